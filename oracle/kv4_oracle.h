@@ -1,0 +1,108 @@
+/*
+ * kv4_oracle.h -- plain fp64 CPU oracle for decode attention over a KV4-RL
+ * compressed KV cache (paged INT4 + INT8 sink/recent side cache).
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg load this library. It shares no code, header or table with
+ * the CUDA library; the only contract between the two is the stated byte
+ * layout and the stated quantiser, both written out independently on each side.
+ *
+ * Sources (web pages, cited by title and section):
+ *  [KV4RL]  "[Paper review] KV4-RL: Unlocking Faster Asynchronous Rollouts for
+ *           RLVR with INT4 KV Cache Quantization", sec. 1 (Selective Protection)
+ *           and sec. 3 (Method & Key Results): full context in paged INT4,
+ *           first 16 + most recent 128 positions in an INT8 side cache, the two
+ *           regions attended separately and joined by an exact softmax merge.
+ *  [SMD]    "How to compress the KV cache in RL post-training? Shadow Mask
+ *           Distillation" (arXiv 2605.06850), sec. 1 and Figure 1: the retained
+ *           index set is recorded as a binary mask and applied inside attention.
+ *  [KVP]    promo of arXiv 2602.10238 ("learning to evict"), core-mechanism
+ *           section: score every token, rank, truncate at a 10%..90% budget,
+ *           one ranking per attention head.
+ * Quantiser details the pages leave open (symmetric INT4 per 32-element group
+ * along head_dim with an fp16 scale; per-token INT8 with an fp16 scale;
+ * scale rounded toward +inf; codes rounded to nearest-even) are this project's
+ * stated readings.
+ */
+#ifndef KV4_ORACLE_H
+#define KV4_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+  int32_t B;        /* sequences */
+  int32_t Hq;       /* query heads */
+  int32_t Hkv;      /* KV heads; Hq % Hkv == 0 */
+  int32_t D;        /* head_dim, a multiple of 32 */
+  int32_t sink;     /* INT8 sink positions (16 in KV4-RL) */
+  int32_t recent;   /* INT8 recent window (128 in KV4-RL) */
+} kv4o_shape;
+
+/* ---- number formats ---- */
+uint16_t kv4o_fp16_round_up(double y);          /* smallest fp16 >= y (y >= 0); +inf bits if none */
+double   kv4o_fp16_to_double(uint16_t bits);
+double   kv4o_bf16_to_double(uint16_t bits);
+double   kv4o_round_half_even(double x);
+
+/* ---- quantiser ---- */
+/* Symmetric INT4 over n elements (a group of 32): s = RU_fp16(max|x|/7),
+ * c = RNE(x/s) in [-7,7]. Returns 1 if the scale overflowed fp16 (then
+ * s = 0x7BFF and codes are clamped), else 0. */
+int kv4o_quant_int4(const uint16_t *x_bf16, int n, uint16_t *scale_bits, int8_t *codes);
+/* Symmetric INT8 over n elements (one token row): s = RU_fp16(max|x|/127),
+ * c = RNE(x/s) in [-127,127]. Same overflow rule. */
+int kv4o_quant_int8(const uint16_t *x_bf16, int n, uint16_t *scale_bits, int8_t *codes);
+
+/* ---- byte layout (offsets inside one head block of one physical page) ---- */
+int64_t kv4o_page_head_bytes(int D);                       /* 18*D */
+int64_t kv4o_k_code_byte(int D, int r, int d, int *nibble); /* r = slot 0..15 */
+int64_t kv4o_v_code_byte(int D, int r, int d, int *nibble);
+int64_t kv4o_k_scale_byte(int D, int r, int grp);
+int64_t kv4o_v_scale_byte(int D, int r, int grp);
+int64_t kv4o_side_head_bytes(int D, int sink, int recent); /* INT8 block per (seq, head) */
+
+/* Write the byte image that appending positions [0, lens[b]) of every sequence
+ * leaves in the page pool and the side cache. k, v: bf16 bits [B][Lmax][Hkv][D].
+ * page_table: [B][pt_stride]. Bytes not written are left untouched.
+ * Returns the OR of range flags (1 = a scale overflowed). */
+int kv4o_write_cache(const kv4o_shape *sh, const uint16_t *k, const uint16_t *v, int Lmax,
+                     const int32_t *lens, const int32_t *page_table, int pt_stride,
+                     uint8_t *pool, int64_t pool_bytes, uint8_t *side, int64_t side_bytes);
+
+/* Dequantised K and V rows of (sequence b, KV head h) as attention sees them:
+ * INT8 values for positions in the protected set, INT4 values elsewhere.
+ * khat, vhat: [lens[b]][D] doubles. */
+void kv4o_dequant_rows(const kv4o_shape *sh, const uint16_t *k, const uint16_t *v, int Lmax,
+                       const int32_t *lens, int b, int h, double *khat, double *vhat);
+
+/* ---- attention ---- */
+/* Softmax attention of every query head over the retained positions.
+ * q: bf16 bits [B][Hq][D]. mask: NULL or bits [B][Hkv][mask_stride] (bit p of
+ * word p/32 set = position p retained). mode 0: KV4 values (INT4 + INT8
+ * protection); mode 1: the bf16 values themselves. out: [B][Hq][D]. */
+void kv4o_decode(const kv4o_shape *sh, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                 int Lmax, const int32_t *lens, const uint32_t *mask, int mask_stride,
+                 float softmax_scale, int mode, double *out);
+
+/* Partial over an arbitrary set of n rows: m = max s, l = sum e^(s-m),
+ * o = sum e^(s-m) v / l. Empty set: m = -inf, l = 0, o = 0. */
+void kv4o_attend_rows(int D, const double *q, const double *krows, const double *vrows, int n,
+                      double scale, double *m, double *l, double *o);
+/* Exact merge of C partials: M = max m_c, W_c = l_c e^(m_c - M),
+ * out = sum W_c o_c / sum W_c. All empty: out = 0. */
+void kv4o_merge(int D, int C, const double *m, const double *l, const double *o, double *out);
+
+/* ---- retained-position selection ---- */
+/* Per (b, h): forced set F = first min(sink, L) and last min(recent, L)
+ * positions; k = floor(L * permille / 1000); keep F plus the max(0, k - |F|)
+ * best other positions by (score descending, index ascending). */
+void kv4o_topk(const float *scores, int64_t score_stride, const int32_t *lens, int B, int Hkv,
+               int permille, int sink, int recent, uint32_t *mask, int mask_stride, int32_t *count);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
