@@ -1,0 +1,471 @@
+// kv4_api.cu -- the extern "C" boundary of libkv4 (declared in include/kv4.h).
+//
+// Host-side argument validation, workspace layout, worker planning and kernel
+// launches on the caller's stream. No device memory is allocated except the
+// 4-byte error word of a kv4_cache.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "../../include/kv4.h"
+#include "kv4_common.cuh"
+#include "kv4_internal.h"
+
+using namespace kv4;
+
+struct kv4_cache {
+  kv4_config cfg;
+  uint8_t *pool;
+  size_t pool_bytes;
+  uint8_t *side;
+  size_t side_bytes;
+  uint32_t *err;
+  int device;
+  int num_sms;
+  long long wait_cap;
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+long long page_head_bytes(int D) { return 18LL * D; }
+
+long long side_head_bytes(int D, int sink, int recent) {
+  const long long rows = sink + recent;
+  return (long long)round_up((size_t)(2 * rows * D + 4 * rows), 16);
+}
+
+int slot_o_off(int G) { return (int)round_up((size_t)(2 * G), 4); }
+int slot_floats(int G, int D) { return slot_o_off(G) + G * D; }
+
+kv4_status check_config(const kv4_config *c) {
+  if (!c) return KV4_ERR_INVALID;
+  if (c->num_kv_heads < 1 || c->max_seqs < 1 || c->num_pages < 1) return KV4_ERR_INVALID;
+  if (c->page_tokens != kPageTokens || c->group != kGroup) return KV4_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return KV4_ERR_UNSUPPORTED;
+  if (c->sink < 0 || c->sink > 16 || c->recent < 0 || c->recent > 128) return KV4_ERR_UNSUPPORTED;
+  return KV4_OK;
+}
+
+// Per (D, G, format) launch geometry, computed once per process.
+struct Geometry {
+  bool ready = false;
+  cudaError_t err = cudaSuccess;
+  DecodeLaunch l{};
+};
+
+std::mutex g_mu;
+Geometry g_geo[2][3][2];   // [D=64,128][G=1,2,4][int4, bf16]
+int g_num_sms = 0;
+
+int gidx(int G) { return G == 1 ? 0 : (G == 2 ? 1 : 2); }
+
+cudaError_t geometry(int D, int G, bool bf16, DecodeLaunch *out, int *num_sms) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  Geometry &g = g_geo[D == 128][gidx(G)][bf16];
+  if (!g.ready) {
+    g.err = decode_prepare(D, G, bf16, &g.l);
+    g.ready = true;
+  }
+  if (g.err != cudaSuccess) return g.err;
+  *out = g.l;
+  *num_sms = g_num_sms;
+  return cudaSuccess;
+}
+
+int default_workers(const DecodeLaunch &l, int num_sms) { return num_sms * l.blocks_per_sm * kWarps; }
+
+int resolve_workers(int requested, const DecodeLaunch &l, int num_sms) {
+  int nw = requested > 0 ? requested : default_workers(l, num_sms);
+  return (nw + kWarps - 1) / kWarps * kWarps;
+}
+
+size_t decode_ws_bytes(int B, int Hkv, int G, int D, int nw, bool has8) {
+  const size_t slot = (size_t)slot_floats(G, D) * 4;
+  size_t bytes = round_up((size_t)(B + 1) * 8, kAlign);
+  if (has8) bytes += round_up((size_t)B * Hkv * slot, kAlign);
+  bytes += round_up(((size_t)B * Hkv + nw) * slot, kAlign);
+  return bytes;
+}
+
+void carve_workspace(DecodeParams &p, void *ws, int D, bool has8) {
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  const size_t slot = (size_t)p.slot_floats * 4;
+  p.plan = reinterpret_cast<long long *>(w);
+  w += round_up((size_t)(p.B + 1) * 8, kAlign);
+  p.slots8 = reinterpret_cast<float *>(w);
+  if (has8) w += round_up((size_t)p.B * p.Hkv * slot, kAlign);
+  p.slots4 = reinterpret_cast<float *>(w);
+  (void)D;
+}
+
+kv4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA; }
+
+// Timing hook state: per kind, a fixed pool of event pairs filled in call order.
+struct Timing {
+  bool on = false;
+  int max_records = 0;
+  int used[2] = {0, 0};
+  std::vector<cudaEvent_t> ev[2];   // 2 * max_records events per kind
+};
+Timing g_timing;
+std::mutex g_timing_mu;
+
+void timing_pair(int kind, cudaEvent_t *e0, cudaEvent_t *e1) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  *e0 = *e1 = nullptr;
+  if (!g_timing.on || g_timing.used[kind] >= g_timing.max_records) return;
+  const int i = g_timing.used[kind]++;
+  *e0 = g_timing.ev[kind][2 * i];
+  *e1 = g_timing.ev[kind][2 * i + 1];
+}
+
+void timing_free() {
+  for (int k = 0; k < 2; ++k) {
+    for (cudaEvent_t e : g_timing.ev[k]) cudaEventDestroy(e);
+    g_timing.ev[k].clear();
+    g_timing.used[k] = 0;
+  }
+  g_timing.on = false;
+  g_timing.max_records = 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kv4_status_string(kv4_status s) {
+  switch (s) {
+    case KV4_OK: return "KV4_OK";
+    case KV4_ERR_INVALID: return "KV4_ERR_INVALID";
+    case KV4_ERR_UNSUPPORTED: return "KV4_ERR_UNSUPPORTED";
+    case KV4_ERR_CAPACITY: return "KV4_ERR_CAPACITY";
+    case KV4_ERR_BOUNDS: return "KV4_ERR_BOUNDS";
+    case KV4_ERR_RANGE: return "KV4_ERR_RANGE";
+    case KV4_ERR_TIMEOUT: return "KV4_ERR_TIMEOUT";
+    case KV4_ERR_CUDA: return "KV4_ERR_CUDA";
+  }
+  return "KV4_ERR_UNKNOWN";
+}
+
+kv4_status kv4_cache_bytes(const kv4_config *cfg, size_t *page_pool_bytes, size_t *side_cache_bytes) {
+  const kv4_status st = check_config(cfg);
+  if (st != KV4_OK) return st;
+  if (!page_pool_bytes || !side_cache_bytes) return KV4_ERR_INVALID;
+  *page_pool_bytes = (size_t)cfg->num_pages * cfg->num_kv_heads * page_head_bytes(cfg->head_dim);
+  *side_cache_bytes =
+      (size_t)cfg->max_seqs * cfg->num_kv_heads * side_head_bytes(cfg->head_dim, cfg->sink, cfg->recent);
+  return KV4_OK;
+}
+
+kv4_status kv4_cache_create(const kv4_config *cfg, void *page_pool, size_t pool_bytes, void *side_cache,
+                            size_t side_bytes, kv4_cache **out) {
+  size_t need_pool = 0, need_side = 0;
+  const kv4_status st = kv4_cache_bytes(cfg, &need_pool, &need_side);
+  if (st != KV4_OK) return st;
+  if (!out || !page_pool || pool_bytes < need_pool) return KV4_ERR_INVALID;
+  if (need_side > 0 && (!side_cache || side_bytes < need_side)) return KV4_ERR_INVALID;
+  if (!aligned(page_pool, 16) || (side_cache && !aligned(side_cache, 16))) return KV4_ERR_INVALID;
+  kv4_cache *c = new kv4_cache();
+  c->cfg = *cfg;
+  c->pool = static_cast<uint8_t *>(page_pool);
+  c->pool_bytes = pool_bytes;
+  c->side = static_cast<uint8_t *>(side_cache);
+  c->side_bytes = side_bytes;
+  c->wait_cap = kDefaultWaitCycles;
+  cudaError_t e = cudaGetDevice(&c->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+  if (e == cudaSuccess) e = cudaMalloc(&c->err, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(c->err, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) {
+    if (c->err) cudaFree(c->err);
+    delete c;
+    return KV4_ERR_CUDA;
+  }
+  *out = c;
+  return KV4_OK;
+}
+
+void kv4_cache_destroy(kv4_cache *cache) {
+  if (!cache) return;
+  if (cache->err) cudaFree(cache->err);
+  delete cache;
+}
+
+kv4_status kv4_append(kv4_cache *cache, void *stream, const void *k_new, const void *v_new,
+                      const int32_t *new_offsets, const int32_t *seq_lens_old, const int32_t *page_table,
+                      int32_t pt_stride, int32_t B, int64_t total_new) {
+  if (!cache) return KV4_ERR_INVALID;
+  if (B < 0 || total_new < 0 || pt_stride < 1) return KV4_ERR_INVALID;
+  if (B == 0 || total_new == 0) return KV4_OK;
+  if (B > cache->cfg.max_seqs) return KV4_ERR_CAPACITY;
+  if (!k_new || !v_new || !new_offsets || !seq_lens_old || !page_table) return KV4_ERR_INVALID;
+  const int D = cache->cfg.head_dim;
+  if (!aligned(k_new, 8) || !aligned(v_new, 8)) return KV4_ERR_INVALID;
+  AppendParams p{};
+  p.k = static_cast<const __nv_bfloat16 *>(k_new);
+  p.v = static_cast<const __nv_bfloat16 *>(v_new);
+  p.offsets = new_offsets;
+  p.lens_old = seq_lens_old;
+  p.page_table = page_table;
+  p.pt_stride = pt_stride;
+  p.B = B;
+  p.Hkv = cache->cfg.num_kv_heads;
+  p.sink = cache->cfg.sink;
+  p.recent = cache->cfg.recent;
+  p.num_pages = cache->cfg.num_pages;
+  p.T = total_new;
+  p.pool = cache->pool;
+  p.side = cache->side;
+  p.head_bytes = page_head_bytes(D);
+  p.page_bytes = p.head_bytes * p.Hkv;
+  p.side_stride = side_head_bytes(D, p.sink, p.recent);
+  p.err = cache->err;
+  return cuda_status(launch_append(p, D, static_cast<cudaStream_t>(stream)));
+}
+
+kv4_status kv4_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t num_q_heads, int32_t num_workers,
+                               size_t *bytes) {
+  if (!cache || !bytes || B < 0 || num_workers < 0) return KV4_ERR_INVALID;
+  const int Hkv = cache->cfg.num_kv_heads;
+  if (num_q_heads < 1 || num_q_heads % Hkv) return KV4_ERR_INVALID;
+  const int G = num_q_heads / Hkv;
+  if (G != 1 && G != 2 && G != 4) return KV4_ERR_UNSUPPORTED;
+  DecodeLaunch l{};
+  int sms = 0;
+  if (geometry(cache->cfg.head_dim, G, false, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
+  const int nw = resolve_workers(num_workers, l, sms);
+  const bool has8 = cache->cfg.sink + cache->cfg.recent > 0;
+  *bytes = decode_ws_bytes(B, Hkv, G, cache->cfg.head_dim, nw, has8);
+  return KV4_OK;
+}
+
+kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_t Hq, const int32_t *seq_lens,
+                           const int32_t *page_table, int32_t pt_stride, const uint32_t *retain_mask,
+                           int32_t mask_stride, float softmax_scale, int32_t num_workers, void *workspace,
+                           size_t ws_bytes, void *out, int32_t out_is_fp32, int32_t B) {
+  if (!cache || B < 0 || pt_stride < 1 || num_workers < 0) return KV4_ERR_INVALID;
+  if (B == 0) return KV4_OK;
+  if (B > cache->cfg.max_seqs) return KV4_ERR_CAPACITY;
+  const int Hkv = cache->cfg.num_kv_heads, D = cache->cfg.head_dim;
+  if (Hq < 1 || Hq % Hkv) return KV4_ERR_INVALID;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4) return KV4_ERR_UNSUPPORTED;
+  if (!q || !seq_lens || !page_table || !workspace || !out) return KV4_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 16)) return KV4_ERR_INVALID;
+  if (retain_mask && (long long)mask_stride * 32 < (long long)pt_stride * kPageTokens) return KV4_ERR_INVALID;
+  if (!isfinite(softmax_scale)) return KV4_ERR_INVALID;
+  DecodeLaunch l{};
+  int sms = 0;
+  if (geometry(D, G, false, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
+  const int nw = resolve_workers(num_workers, l, sms);
+  const bool has8 = cache->cfg.sink + cache->cfg.recent > 0;
+  if (ws_bytes < decode_ws_bytes(B, Hkv, G, D, nw, has8)) return KV4_ERR_INVALID;
+
+  DecodeParams p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.sink = cache->cfg.sink;
+  p.recent = cache->cfg.recent;
+  p.num_pages = cache->cfg.num_pages;
+  p.pt_stride = pt_stride;
+  p.mask_stride = mask_stride;
+  p.num_workers = nw;
+  p.slot_floats = slot_floats(G, D);
+  p.slot_o_off = slot_o_off(G);
+  p.int8_units = has8 ? 1 : 0;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.seq_lens = seq_lens;
+  p.page_table = page_table;
+  p.mask = retain_mask;
+  p.pool = cache->pool;
+  p.side = cache->side;
+  p.head_bytes = page_head_bytes(D);
+  p.page_bytes = p.head_bytes * Hkv;
+  p.side_stride = side_head_bytes(D, p.sink, p.recent);
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  p.out_fp32 = out_is_fp32 ? 1 : 0;
+  p.err = cache->err;
+  p.wait_cap = cache->wait_cap;
+  carve_workspace(p, workspace, D, has8);
+  cudaEvent_t e0, e1;
+  timing_pair(0, &e0, &e1);
+  return cuda_status(launch_decode(p, D, false, static_cast<cudaStream_t>(stream), e0, e1));
+}
+
+kv4_status kv_topk_retain(void *stream, const float *scores, int64_t score_stride, const int32_t *seq_lens,
+                          int32_t B, int32_t Hkv, int32_t budget_permille, int32_t sink, int32_t recent,
+                          uint32_t *mask_out, int32_t mask_stride, int32_t *count_out, int32_t max_len) {
+  if (B < 0 || Hkv < 1 || max_len < 0) return KV4_ERR_INVALID;
+  if (B == 0) return KV4_OK;
+  if (!scores || !seq_lens || !mask_out) return KV4_ERR_INVALID;
+  if (budget_permille < 0 || budget_permille > 1000 || sink < 0 || recent < 0) return KV4_ERR_INVALID;
+  if (score_stride < max_len || (long long)mask_stride * 32 < max_len) return KV4_ERR_INVALID;
+  if (max_len > 1500000) return KV4_ERR_UNSUPPORTED;
+  TopkParams p{};
+  p.scores = scores;
+  p.score_stride = score_stride;
+  p.seq_lens = seq_lens;
+  p.B = B;
+  p.Hkv = Hkv;
+  p.permille = budget_permille;
+  p.sink = sink;
+  p.recent = recent;
+  p.max_len = max_len;
+  p.mask_stride = mask_stride;
+  p.mask = mask_out;
+  p.count = count_out;
+  return cuda_status(launch_topk(p, static_cast<cudaStream_t>(stream)));
+}
+
+kv4_status bf16_paged_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t num_workers,
+                                      size_t *bytes) {
+  if (!bytes || B < 0 || Hkv < 1 || Hq < 1 || Hq % Hkv || num_workers < 0) return KV4_ERR_INVALID;
+  const int G = Hq / Hkv;
+  if ((G != 1 && G != 2 && G != 4) || (D != 64 && D != 128)) return KV4_ERR_UNSUPPORTED;
+  DecodeLaunch l{};
+  int sms = 0;
+  if (geometry(D, G, true, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
+  *bytes = decode_ws_bytes(B, Hkv, G, D, resolve_workers(num_workers, l, sms), false);
+  return KV4_OK;
+}
+
+kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32_t Hkv, int32_t D,
+                                  const void *kv_pages, int32_t num_pages, const int32_t *page_table,
+                                  int32_t pt_stride, const int32_t *seq_lens, float softmax_scale,
+                                  int32_t num_workers, void *workspace, size_t ws_bytes, void *out,
+                                  int32_t out_is_fp32, int32_t B, uint32_t *error_word) {
+  if (B < 0 || Hkv < 1 || Hq < 1 || Hq % Hkv || pt_stride < 1 || num_pages < 1 || num_workers < 0)
+    return KV4_ERR_INVALID;
+  if (B == 0) return KV4_OK;
+  const int G = Hq / Hkv;
+  if ((G != 1 && G != 2 && G != 4) || (D != 64 && D != 128)) return KV4_ERR_UNSUPPORTED;
+  if (!q || !kv_pages || !page_table || !seq_lens || !workspace || !out) return KV4_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 16) || !aligned(kv_pages, 16))
+    return KV4_ERR_INVALID;
+  if (!isfinite(softmax_scale)) return KV4_ERR_INVALID;
+  DecodeLaunch l{};
+  int sms = 0;
+  if (geometry(D, G, true, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
+  const int nw = resolve_workers(num_workers, l, sms);
+  if (ws_bytes < decode_ws_bytes(B, Hkv, G, D, nw, false)) return KV4_ERR_INVALID;
+  DecodeParams p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.num_pages = num_pages;
+  p.pt_stride = pt_stride;
+  p.num_workers = nw;
+  p.slot_floats = slot_floats(G, D);
+  p.slot_o_off = slot_o_off(G);
+  p.int8_units = 0;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.seq_lens = seq_lens;
+  p.page_table = page_table;
+  p.pool = static_cast<const uint8_t *>(kv_pages);
+  p.head_bytes = 64LL * D;
+  p.page_bytes = p.head_bytes * Hkv;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  p.out_fp32 = out_is_fp32 ? 1 : 0;
+  p.err = error_word;
+  p.wait_cap = kDefaultWaitCycles;
+  carve_workspace(p, workspace, D, false);
+  cudaEvent_t e0, e1;
+  timing_pair(1, &e0, &e1);
+  return cuda_status(launch_decode(p, D, true, static_cast<cudaStream_t>(stream), e0, e1));
+}
+
+kv4_status kv4_get_error(kv4_cache *cache, void *stream, uint32_t *bits) {
+  if (!cache) return KV4_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t w = 0;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&w, cache->err, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(cache->err, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) return KV4_ERR_CUDA;
+  if (bits) *bits = w;
+  if (w & (1u << KV4_ERR_TIMEOUT)) return KV4_ERR_TIMEOUT;
+  if (w & (1u << KV4_ERR_BOUNDS)) return KV4_ERR_BOUNDS;
+  if (w & (1u << KV4_ERR_CAPACITY)) return KV4_ERR_CAPACITY;
+  if (w & (1u << KV4_ERR_RANGE)) return KV4_ERR_RANGE;
+  return KV4_OK;
+}
+
+kv4_status kv4_debug_set_wait_limit(kv4_cache *cache, int64_t cycles) {
+  if (!cache) return KV4_ERR_INVALID;
+  cache->wait_cap = cycles < 0 ? kDefaultWaitCycles : cycles;
+  return KV4_OK;
+}
+
+kv4_status kv4_device_info(int32_t *num_sms, int32_t *default_workers_out) {
+  DecodeLaunch l{};
+  int sms = 0;
+  if (geometry(128, 4, false, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
+  if (num_sms) *num_sms = sms;
+  if (default_workers_out) *default_workers_out = default_workers(l, sms);
+  return KV4_OK;
+}
+
+kv4_status kv4_timing_enable(int32_t max_records) {
+  if (max_records < 1) return KV4_ERR_INVALID;
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  timing_free();
+  for (int k = 0; k < 2; ++k) {
+    g_timing.ev[k].resize(2 * (size_t)max_records, nullptr);
+    for (auto &e : g_timing.ev[k]) {
+      if (cudaEventCreate(&e) != cudaSuccess) {
+        timing_free();
+        return KV4_ERR_CUDA;
+      }
+    }
+  }
+  g_timing.max_records = max_records;
+  g_timing.on = true;
+  return KV4_OK;
+}
+
+kv4_status kv4_timing_read(int32_t kind, double *total_ms, int32_t *count) {
+  if (kind < 0 || kind > 1 || !total_ms || !count) return KV4_ERR_INVALID;
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  double sum = 0.0;
+  const int n = g_timing.used[kind];
+  for (int i = 0; i < n; ++i) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(g_timing.ev[kind][2 * i + 1]) != cudaSuccess) return KV4_ERR_CUDA;
+    if (cudaEventElapsedTime(&ms, g_timing.ev[kind][2 * i], g_timing.ev[kind][2 * i + 1]) != cudaSuccess)
+      return KV4_ERR_CUDA;
+    sum += ms;
+  }
+  g_timing.used[kind] = 0;
+  *total_ms = sum;
+  *count = n;
+  return KV4_OK;
+}
+
+kv4_status kv4_timing_disable(void) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  timing_free();
+  return KV4_OK;
+}
+
+}  // extern "C"

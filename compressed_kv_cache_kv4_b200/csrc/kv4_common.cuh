@@ -1,0 +1,169 @@
+// kv4_common.cuh -- device helpers shared by the libkv4 kernels (sm_100a).
+//
+// Inline PTX for: mbarrier + 1-D bulk copies (the TMA engine, no multicast),
+// warp-level bf16 tensor-core MMA (m16n8k16) and 8x8 fragment transposes,
+// LOP3 nibble -> bf16 unpacking, ex2.approx.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kv4 {
+
+constexpr int kPageTokens = 16;
+constexpr int kGroup = 32;
+constexpr int kWarps = 4;                       // warps per CTA in the decode kernels
+constexpr long long kDefaultWaitCycles = 1ll << 32;
+
+// Device error bits: bit (1 << status) for the kv4_status values of kv4.h.
+constexpr uint32_t kErrCapacity = 1u << 3;
+constexpr uint32_t kErrBounds = 1u << 4;
+constexpr uint32_t kErrRange = 1u << 5;
+constexpr uint32_t kErrTimeout = 1u << 6;
+
+__device__ __forceinline__ void set_error(uint32_t *err, uint32_t bit) {
+  if (err) atomicOr(err, bit);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier + bulk copy
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, for at most `cap` SM cycles.
+// cap <= 0 gives up immediately unless the phase is already complete.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, long long cap) {
+  if (mbar_try_wait(bar, parity)) return true;
+  if (cap <= 0) return false;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > cap) return false;
+  }
+  return true;
+}
+
+// 1-D bulk copy global -> shared through the TMA engine; completion is
+// counted in bytes on `bar`. dst, src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// ---------------------------------------------------------------- tensor-core fragments
+// D = A * B + C with A 16x16 (row), B 16x8 (col) bf16, C/D fp32.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 matrix of 16-bit elements held one row per 4 lanes.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+  uint32_t d;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// Two signed 4-bit codes at bits 0-3 and 16-19 of w -> bf16x2 of the codes.
+// LOP3 computes (w & 0x000F000F) ^ 0x43084308: flipping bit 3 turns the
+// two's-complement nibble c into c + 8, and 0x43 above it makes the bf16
+// value 128 + (c + 8). Subtracting 136 (bf16 0x4308) is exact.
+__device__ __forceinline__ uint32_t i4x2_to_bf16x2(uint32_t w) {
+  uint32_t t, d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x000F000Fu), "r"(0x43084308u));
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(t), "r"(0x43084308u));
+  return d;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ float half_bits_to_f32(uint16_t h) {
+  return __half2float(__ushort_as_half(h));
+}
+
+// ---------------------------------------------------------------- region arithmetic
+// Effective length: negative or beyond the page-table capacity counts as empty.
+__device__ __forceinline__ int eff_len(int L, int cap) { return (L < 0 || L > cap) ? 0 : L; }
+
+// INT4-attended positions are [sink, L - recent); the rest of [0, L) is the
+// INT8-protected set (KV4-RL review, sec. 3). Pages of the INT4 region:
+// [sink/16, ceil((L - recent)/16)).
+__device__ __forceinline__ int int4_first_page(int sink) { return sink / kPageTokens; }
+__device__ __forceinline__ int int4_num_pages(int L, int sink, int recent) {
+  const int hi = L - recent;
+  if (hi <= sink) return 0;
+  return (hi + kPageTokens - 1) / kPageTokens - sink / kPageTokens;
+}
+
+// Static split of the flat (sequence, KV head, page) space among `nw` workers.
+// Worker w owns [seg_start(w), seg_start(w+1)); workers with more INT8 units get
+// proportionally fewer INT4 page-heads (an INT8 unit weighs `w8` page-heads).
+__device__ __forceinline__ long long seg_start(long long w, long long T4, long long U8, long long nw,
+                                               long long w8) {
+  if (w >= nw) return T4;
+  if (U8 == 0 || T4 < (w8 + 1) * nw) return w * T4 / nw;
+  const long long total = T4 + w8 * U8;
+  const long long cum8 = w * (U8 / nw) + (w < U8 % nw ? w : U8 % nw);
+  return w * total / nw - w8 * cum8;
+}
+
+}  // namespace kv4

@@ -1,0 +1,68 @@
+// kv4_internal.h -- kernel parameter blocks and launchers inside libkv4.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kv4 {
+
+struct AppendParams {
+  const __nv_bfloat16 *k;   // [T][Hkv][D]
+  const __nv_bfloat16 *v;
+  const int32_t *offsets;   // [B+1]
+  const int32_t *lens_old;  // [B]
+  const int32_t *page_table;
+  int pt_stride, B, Hkv, sink, recent, num_pages;
+  long long T;
+  uint8_t *pool;
+  uint8_t *side;
+  long long page_bytes, head_bytes, side_stride;
+  uint32_t *err;
+};
+
+struct DecodeParams {
+  int B, Hq, Hkv, G, sink, recent, num_pages, pt_stride, mask_stride;
+  int num_workers, slot_floats, slot_o_off, int8_units;
+  const __nv_bfloat16 *q;       // [B][Hq][D]
+  const int32_t *seq_lens;      // [B]
+  const int32_t *page_table;    // [B][pt_stride]
+  const uint32_t *mask;         // nullable [B][Hkv][mask_stride]
+  const uint8_t *pool;          // INT4 or bf16 pages
+  const uint8_t *side;          // INT8 side blocks
+  long long page_bytes, head_bytes, side_stride;
+  float scale_log2;             // softmax_scale * log2(e)
+  long long *plan;              // [B+1] prefix of attended page-heads
+  float *slots8;                // [B*Hkv][slot_floats]
+  float *slots4;                // [B*Hkv + num_workers][slot_floats]
+  void *out;
+  int out_fp32;
+  uint32_t *err;
+  long long wait_cap;           // 0 = simulate a copy that never lands
+};
+
+struct TopkParams {
+  const float *scores;
+  long long score_stride;
+  const int32_t *seq_lens;
+  int B, Hkv, permille, sink, recent, max_len, mask_stride;
+  uint32_t *mask;
+  int32_t *count;
+};
+
+// Weight of one INT8 unit (<= 144 positions of one KV head, fp32 SIMT) in
+// INT4 page-head units when splitting work among workers.
+constexpr long long kInt8UnitWeight = 16;
+
+struct DecodeLaunch {
+  int smem_bytes;
+  int blocks_per_sm;
+};
+
+cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream);
+cudaError_t decode_prepare(int D, int G, bool bf16, DecodeLaunch *out);
+cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t stream, cudaEvent_t ev0,
+                          cudaEvent_t ev1);
+cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream);
+
+}  // namespace kv4

@@ -1,0 +1,164 @@
+// kv_topk.cu -- per (sequence, KV head) retained-position mask.
+//
+// KVP promo (arXiv 2602.10238), core mechanism, and TTKV promo (arXiv
+// 2604.19769), insight 1: eviction is ranking -- score each position, sort,
+// truncate at the budget; one ranking per attention head serves every budget.
+// KV4-RL review, sec. 3: the first 16 and the last 128 positions are always
+// kept. Shadow Mask Distillation, sec. 1: the result is a binary mask.
+//
+// One CTA per row. Scores become order-preserving 32-bit keys (larger score ->
+// larger key, -0 folded into +0). A 4-pass 8-bit radix select finds the key T
+// of the k-th best non-forced position in O(L) work; positions with key > T
+// are kept, and among keys == T the lowest indices fill the remainder (a scan
+// over 32-position tiles gives each tie its rank in index order). The row is
+// held in shared memory when it fits, otherwise re-read from global memory on
+// each pass.
+#include "kv4_common.cuh"
+#include "kv4_internal.h"
+
+namespace kv4 {
+
+constexpr int kTopkThreads = 512;
+constexpr int kTopkSmemKeys = 49152;   // rows up to this length are staged in shared memory
+
+__device__ __forceinline__ uint32_t score_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int use_smem) {
+  extern __shared__ __align__(16) uint32_t dyn[];
+  __shared__ uint32_t hist[256];
+  __shared__ int sh_digit, sh_rem;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NWARP = kTopkThreads / 32;
+  const int row = blockIdx.x;
+  const int b = row / p.Hkv;
+  int L = p.seq_lens[b];
+  L = L < 0 ? 0 : (L > p.max_len ? p.max_len : L);
+  const float *srow = p.scores + (long long)row * p.score_stride;
+  const int S = p.sink, R = p.recent;
+  const int nt = (L + 31) / 32;
+  uint32_t *keys = dyn;                                   // [max_len] when use_smem
+  int *tile_rank = reinterpret_cast<int *>(dyn + (use_smem ? p.max_len : 0));   // [nt]
+
+  auto forced = [&](int pos) { return pos < S || pos >= L - R; };
+  auto key_at = [&](int pos) { return use_smem ? keys[pos] : score_key(srow[pos]); };
+
+  const int nF = L <= S ? L : S + min(R, L - S);
+  const long long kb = (long long)L * p.permille / 1000;
+  long long ksel = kb - nF;
+  if (ksel < 0) ksel = 0;
+  if (ksel > L - nF) ksel = L - nF;
+
+  if (use_smem)
+    for (int i = tid; i < L; i += kTopkThreads) keys[i] = score_key(srow[i]);
+  __syncthreads();
+
+  // mode: 0 = select none, 1 = select all, 2 = threshold
+  int mode = ksel == 0 ? 0 : (ksel == L - nF ? 1 : 2);
+  uint32_t T = 0;
+  int need_eq = 0;
+  if (mode == 2) {
+    uint32_t prefix = 0, pmask = 0;
+    int rem = static_cast<int>(ksel);
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < L; i += kTopkThreads) {
+        if (forced(i)) continue;
+        const uint32_t k = key_at(i);
+        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l owns bins 255-8l .. 248-8l (descending)
+        int tot = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tot += hist[255 - 8 * lane - i];
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int c = incl - tot;   // keys in bins above this lane's range
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int bin = 255 - 8 * lane - i;
+          const int hcount = hist[bin];
+          if (c < rem && rem <= c + hcount) {
+            sh_digit = bin;
+            sh_rem = rem - c;
+          }
+          c += hcount;
+        }
+      }
+      __syncthreads();
+      prefix |= static_cast<uint32_t>(sh_digit) << shift;
+      pmask |= 255u << shift;
+      rem = sh_rem;
+      __syncthreads();
+    }
+    T = prefix;
+    need_eq = rem;
+    // ranks of the ties in index order: count per 32-position tile, then scan
+    for (int w = warp; w < nt; w += NWARP) {
+      const int pos = 32 * w + lane;
+      const bool eq = pos < L && !forced(pos) && key_at(pos) == T;
+      const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+      if (lane == 0) tile_rank[w] = __popc(bal);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int carry = 0;
+      for (int base = 0; base < nt; base += 32) {
+        const int w = base + lane;
+        const int v = w < nt ? tile_rank[w] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (w < nt) tile_rank[w] = carry + incl - v;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    __syncthreads();
+  }
+
+  uint32_t *mrow = p.mask + (long long)row * p.mask_stride;
+  for (int w = warp; w < nt; w += NWARP) {
+    const int pos = 32 * w + lane;
+    bool sel = false, eq = false;
+    if (pos < L) {
+      if (forced(pos) || mode == 1) {
+        sel = true;
+      } else if (mode == 2) {
+        const uint32_t k = key_at(pos);
+        sel = k > T;
+        eq = k == T;
+      }
+    }
+    const uint32_t eqbal = __ballot_sync(0xffffffffu, eq);
+    if (eq) sel = tile_rank[w] + __popc(eqbal & ((1u << lane) - 1u)) < need_eq;
+    const uint32_t word = __ballot_sync(0xffffffffu, sel);
+    if (lane == 0) mrow[w] = word;
+  }
+  if (tid == 0 && p.count) p.count[row] = nF + static_cast<int>(ksel);
+}
+
+cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream) {
+  const int rows = p.B * p.Hkv;
+  if (rows == 0) return cudaSuccess;
+  const int use_smem = p.max_len <= kTopkSmemKeys ? 1 : 0;
+  const size_t smem = (use_smem ? (size_t)p.max_len * 4 : 0) + (size_t)((p.max_len + 31) / 32) * 4;
+  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_kernel<<<rows, kTopkThreads, smem, stream>>>(p, use_smem);
+  return cudaGetLastError();
+}
+
+}  // namespace kv4

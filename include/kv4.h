@@ -1,0 +1,231 @@
+/*
+ * kv4.h -- C ABI of libkv4: decode-step attention over a KV4-RL compressed KV
+ * cache on NVIDIA B200 (sm_100a).
+ *
+ * The method (cited by page title and section):
+ *  [KV4RL] "[Paper review] KV4-RL: Unlocking Faster Asynchronous Rollouts for
+ *          RLVR with INT4 KV Cache Quantization", sec. 1 (Selective Protection)
+ *          and sec. 3 (Method & Key Results). The full context is stored as
+ *          paged INT4 K/V; the first 16 ("attention sink") and the 128 most
+ *          recent positions are also held in an INT8 side cache; the INT4 and
+ *          INT8 regions are attended independently and their partial
+ *          (max, sum, output) triples are joined by an exact softmax merge, so
+ *          no full-precision cache is ever rebuilt.
+ *  [SMD]   "How to compress the KV cache in RL post-training? Shadow Mask
+ *          Distillation" (arXiv 2605.06850), sec. 1 and Figure 1: eviction is
+ *          recorded as a binary mask of retained positions and applied inside
+ *          attention instead of slicing tensors.
+ *  [KVP]   promo of arXiv 2602.10238 ("learning to evict"), core-mechanism
+ *          section, and the TTKV promo (arXiv 2604.19769), insight 1: score each
+ *          position, rank, truncate at a budget, per attention head.
+ * Stated readings where the pages are silent: symmetric INT4 codes in [-7, 7]
+ * per group of 32 consecutive head_dim elements with one fp16 scale; per-token
+ * INT8 codes in [-127, 127] with one fp16 scale; scales are max|x|/qmax rounded
+ * toward +inf to fp16; codes are x/scale rounded to nearest-even.
+ *
+ * Conventions for every call:
+ *  - All pointers named *_dev or documented "device" are device memory owned by
+ *    the caller; the library never allocates device memory except the 4-byte
+ *    error word owned by a kv4_cache.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL =
+ *    the legacy default stream) unless stated otherwise.
+ *  - Argument errors are detected on the host before any launch and return
+ *    KV4_ERR_INVALID / KV4_ERR_UNSUPPORTED with nothing enqueued.
+ *  - Data errors found on the device (a page id outside the pool, a length
+ *    beyond the page-table capacity, a scale that overflows fp16, a bounded
+ *    wait that ran out) set a bit in the cache's device error word; the kernel
+ *    skips the offending work and returns normally. kv4_get_error() reports it.
+ *  - A failed launch returns KV4_ERR_CUDA.
+ */
+#ifndef KV4_H
+#define KV4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KV4_OK = 0,
+  KV4_ERR_INVALID = 1,      /* bad argument (null, misaligned, inconsistent sizes) */
+  KV4_ERR_UNSUPPORTED = 2,  /* valid but not built (head_dim, GQA group, sink/recent) */
+  KV4_ERR_CAPACITY = 3,     /* a length exceeds the page-table / side-cache capacity */
+  KV4_ERR_BOUNDS = 4,       /* a page id outside [0, num_pages) */
+  KV4_ERR_RANGE = 5,        /* a value too large for an fp16 scale (|x| > 458,528) */
+  KV4_ERR_TIMEOUT = 6,      /* a bounded device wait ran out */
+  KV4_ERR_CUDA = 7          /* a CUDA runtime call failed */
+} kv4_status;
+
+/* Geometry of one compressed cache (one attention layer). */
+typedef struct {
+  int32_t num_kv_heads;  /* Hkv >= 1 */
+  int32_t head_dim;      /* D: 64 or 128 */
+  int32_t page_tokens;   /* positions per page: must be 16 */
+  int32_t group;         /* INT4 group along head_dim: must be 32 */
+  int32_t sink;          /* INT8 sink positions: 0..16 (16 in KV4-RL) */
+  int32_t recent;        /* INT8 recent window: 0..128 (128 in KV4-RL) */
+  int32_t max_seqs;      /* sequence slots in the side cache */
+  int32_t num_pages;     /* physical pages in the pool */
+} kv4_config;
+
+typedef struct kv4_cache kv4_cache;   /* opaque host handle */
+
+/* Human-readable name of a status. Never NULL. */
+const char *kv4_status_string(kv4_status s);
+
+/*
+ * kv4_cache_bytes -- sizes of the two caller-owned device buffers.
+ *  page_pool_bytes: num_pages pages. One page holds 16 positions of every KV
+ *    head: per head a block of 18*D bytes = K codes 8D | V codes 8D |
+ *    K scales D | V scales D (INT4 nibbles in the register-fragment order the
+ *    decode kernel consumes; fp16 scales [slot][group]).
+ *  side_cache_bytes: max_seqs * Hkv INT8 blocks, one per (sequence, KV head):
+ *    rows 0..sink-1 hold sink positions, rows sink..sink+recent-1 the ring
+ *    (position p in ring row p mod recent); K codes | V codes | K scales | V
+ *    scales, padded to 16 bytes.
+ * [KV4RL] sec. 3 (paged INT4 full context; bounded INT8 side cache).
+ * Host only; no CUDA call.
+ */
+kv4_status kv4_cache_bytes(const kv4_config *cfg, size_t *page_pool_bytes, size_t *side_cache_bytes);
+
+/*
+ * kv4_cache_create -- bind caller-owned device buffers into a cache handle.
+ *  page_pool, side_cache: device, 256-byte aligned, at least the sizes above.
+ *  The handle keeps the pointers (no copy, no ownership) and allocates one
+ *  4-byte device error word on the current device. Contents of the buffers
+ *  are not touched. Returns KV4_ERR_CUDA if the device query or allocation fails.
+ */
+kv4_status kv4_cache_create(const kv4_config *cfg, void *page_pool, size_t pool_bytes,
+                            void *side_cache, size_t side_bytes, kv4_cache **out);
+
+/* Free the handle and its error word (not the caller's buffers). NULL is a no-op. */
+void kv4_cache_destroy(kv4_cache *cache);
+
+/*
+ * kv4_append -- quantise new K/V positions into the cache ([KV4RL] sec. 3).
+ *  k_new, v_new: device bf16 [T][Hkv][D], the new positions of all sequences
+ *    concatenated; sequence b owns rows new_offsets[b] .. new_offsets[b+1]-1.
+ *  new_offsets: device int32 [B+1], non-decreasing, new_offsets[0] = 0.
+ *  seq_lens_old: device int32 [B], positions already cached (read only; the
+ *    caller adds the new counts afterwards).
+ *  page_table: device int32 [B][pt_stride]; logical page p/16 of sequence b
+ *    must be mapped before position p is appended.
+ *  total_new: T, the host-known number of new rows (sizes the launch).
+ * Position p = seq_lens_old[b] + j gets INT4 codes in slot p%16 of page
+ * page_table[b][p/16]; INT8 codes in sink row p if p < sink; and INT8 codes in
+ * ring row p mod recent if p >= (new length) - recent (only the last occupant
+ * of a ring row writes, so multi-token appends are race-free).
+ */
+kv4_status kv4_append(kv4_cache *cache, void *stream, const void *k_new, const void *v_new,
+                      const int32_t *new_offsets, const int32_t *seq_lens_old,
+                      const int32_t *page_table, int32_t pt_stride, int32_t B, int64_t total_new);
+
+/*
+ * kv4_workspace_bytes -- device scratch needed by kv4_decode_attn for B
+ * sequences and Hq query heads with `num_workers` parallel workers (0 = the
+ * library's default for this device). Host only.
+ */
+kv4_status kv4_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t num_q_heads,
+                               int32_t num_workers, size_t *bytes);
+
+/*
+ * kv4_decode_attn -- one decode step of attention for every sequence and query
+ * head over the compressed cache.
+ *  q: device bf16 [B][Hq][D]; query head hq reads KV head hq / (Hq/Hkv).
+ *  seq_lens: device int32 [B], lengths after this step's append.
+ *  retain_mask: NULL, or device uint32 [B][Hkv][mask_stride]; bit p%32 of word
+ *    p/32 set = position p retained ([SMD] Figure 1). Positions with a clear bit
+ *    are excluded; pages with no retained position are not read.
+ *  softmax_scale: tau, scores are tau * q.k.
+ *  num_workers: 0 = default; otherwise the number of warp workers among which
+ *    the INT4 pages are split (results agree within rounding for any value).
+ *  workspace: device, >= kv4_workspace_bytes(), 256-byte aligned.
+ *  out: device [B][Hq][D], bf16 (out_is_fp32 = 0) or fp32 (1).
+ * The INT4 region [sink, L - recent) and the INT8 region (the rest) are
+ * attended separately into (max, sum, output) partials and merged exactly
+ * ([KV4RL] sec. 3). An empty retained set gives an output of 0.
+ */
+kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_t Hq,
+                           const int32_t *seq_lens, const int32_t *page_table, int32_t pt_stride,
+                           const uint32_t *retain_mask, int32_t mask_stride, float softmax_scale,
+                           int32_t num_workers, void *workspace, size_t ws_bytes, void *out,
+                           int32_t out_is_fp32, int32_t B);
+
+/*
+ * kv_topk_retain -- per (sequence, KV head) retained-position mask ([KVP] core
+ * mechanism; [SMD] sec. 1).
+ *  scores: device fp32 [B][Hkv][score_stride], one score per position.
+ *  Forced set F: positions < sink and positions >= L - recent.
+ *  k = floor(L * budget_permille / 1000); F plus the max(0, k - |F|) other
+ *  positions with the highest scores (ties: lower index first) are retained.
+ *  mask_out: device uint32 [B][Hkv][mask_stride]; words 0..ceil(L/32)-1 are
+ *    written (bits >= L zero); later words are not touched.
+ *  count_out: NULL or device int32 [B][Hkv], the retained count.
+ *  max_len: host upper bound on seq_lens (sizes the launch); must be
+ *    <= score_stride and <= 32 * mask_stride.
+ * Scores must not be NaN; -0 and +0 compare equal.
+ */
+kv4_status kv_topk_retain(void *stream, const float *scores, int64_t score_stride,
+                          const int32_t *seq_lens, int32_t B, int32_t Hkv, int32_t budget_permille,
+                          int32_t sink, int32_t recent, uint32_t *mask_out, int32_t mask_stride,
+                          int32_t *count_out, int32_t max_len);
+
+/*
+ * bf16_paged_workspace_bytes / bf16_paged_decode_attn -- the uncompressed
+ * comparison ([KV4RL] sec. 3 compares against BF16 rollouts): the same decode
+ * attention over bf16 pages. One page holds 16 positions of every KV head: per
+ * head a block K[16][D] bf16 then V[16][D] bf16 (64*D bytes).
+ *  kv_pages: device, num_pages pages. error_word: NULL or a device uint32 that
+ *  receives KV4_ERR_BOUNDS / KV4_ERR_CAPACITY bits (1 << status).
+ * Other arguments as kv4_decode_attn.
+ */
+kv4_status bf16_paged_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
+                                      int32_t num_workers, size_t *bytes);
+kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32_t Hkv, int32_t D,
+                                  const void *kv_pages, int32_t num_pages, const int32_t *page_table,
+                                  int32_t pt_stride, const int32_t *seq_lens, float softmax_scale,
+                                  int32_t num_workers, void *workspace, size_t ws_bytes, void *out,
+                                  int32_t out_is_fp32, int32_t B, uint32_t *error_word);
+
+/*
+ * kv4_get_error -- synchronise `stream`, then read and clear the cache's device
+ * error word. Returns KV4_OK if no device error was recorded, else the most
+ * severe recorded status (TIMEOUT > BOUNDS > CAPACITY > RANGE). *bits (optional)
+ * receives the raw word: bit (1 << status) per recorded status.
+ */
+kv4_status kv4_get_error(kv4_cache *cache, void *stream, uint32_t *bits);
+
+/*
+ * kv4_debug_set_wait_limit -- test hook for the bounded device waits of this
+ * cache's decode calls, in SM clock cycles.
+ *   cycles = 0:  the first wait on a page copy gives up at once and records
+ *                KV4_ERR_TIMEOUT; the worker then drains the copies it has in
+ *                flight (with the default limit) and stops.
+ *   cycles > 0:  that limit.
+ *   cycles < 0:  the default limit (about 2^32 cycles, ~2 s).
+ * Host only.
+ */
+kv4_status kv4_debug_set_wait_limit(kv4_cache *cache, int64_t cycles);
+
+/*
+ * Kernel timing hook (host only). While enabled, every kv4_decode_attn and
+ * bf16_paged_decode_attn call records a pair of CUDA events on its stream
+ * immediately before and after its split-K worker kernel, for up to
+ * `max_records` calls per kind. kv4_timing_read synchronises those events and
+ * returns the summed worker-kernel time in milliseconds and the number of
+ * recorded calls for `kind` (0 = kv4_decode_attn, 1 = bf16_paged_decode_attn),
+ * then clears the records. kv4_timing_disable frees the events.
+ */
+kv4_status kv4_timing_enable(int32_t max_records);
+kv4_status kv4_timing_read(int32_t kind, double *total_ms, int32_t *count);
+kv4_status kv4_timing_disable(void);
+
+/* Number of multiprocessors and default worker count the library uses. */
+kv4_status kv4_device_info(int32_t *num_sms, int32_t *default_workers);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KV4_H */
