@@ -38,9 +38,10 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 long long page_head_bytes(int D) { return 18LL * D; }
 
+// INT8 side block of one (sequence, KV head): a sink page (when sink > 0) and
+// recent/16 ring pages of 32*D + 64 bytes each.
 long long side_head_bytes(int D, int sink, int recent) {
-  const long long rows = sink + recent;
-  return (long long)round_up((size_t)(2 * rows * D + 4 * rows), 16);
+  return (long long)((sink > 0 ? 1 : 0) + recent / 16) * (32LL * D + 64);
 }
 
 int slot_o_off(int G) { return (int)round_up((size_t)(2 * G), 4); }
@@ -51,7 +52,7 @@ kv4_status check_config(const kv4_config *c) {
   if (c->num_kv_heads < 1 || c->max_seqs < 1 || c->num_pages < 1) return KV4_ERR_INVALID;
   if (c->page_tokens != kPageTokens || c->group != kGroup) return KV4_ERR_UNSUPPORTED;
   if (c->head_dim != 64 && c->head_dim != 128) return KV4_ERR_UNSUPPORTED;
-  if (c->sink < 0 || c->sink > 16 || c->recent < 0 || c->recent > 128) return KV4_ERR_UNSUPPORTED;
+  if (c->sink < 0 || c->sink > 16 || c->recent < 0 || c->recent > 128 || c->recent % 16) return KV4_ERR_UNSUPPORTED;
   return KV4_OK;
 }
 
@@ -95,23 +96,22 @@ int resolve_workers(int requested, const DecodeLaunch &l, int num_sms) {
   return (nw + kWarps - 1) / kWarps * kWarps;
 }
 
-size_t decode_ws_bytes(int B, int Hkv, int G, int D, int nw, bool has8) {
+// Workspace: plan int32 [B+1] | segs int64 [nw+1] | partial slots
+// [2*B*Hkv + nw][slot_floats] (INT8 ranges, then INT4 ranges, each offset by
+// the worker index).
+size_t decode_ws_bytes(int B, int Hkv, int G, int D, int nw) {
   const size_t slot = (size_t)slot_floats(G, D) * 4;
-  size_t bytes = round_up((size_t)(B + 1) * 8, kAlign);
-  if (has8) bytes += round_up((size_t)B * Hkv * slot, kAlign);
-  bytes += round_up(((size_t)B * Hkv + nw) * slot, kAlign);
-  return bytes;
+  return round_up((size_t)(B + 1) * 4, kAlign) + round_up((size_t)(nw + 1) * 8, kAlign) +
+         round_up(((size_t)2 * B * Hkv + nw) * slot, kAlign);
 }
 
-void carve_workspace(DecodeParams &p, void *ws, int D, bool has8) {
+void carve_workspace(DecodeParams &p, void *ws) {
   uint8_t *w = static_cast<uint8_t *>(ws);
-  const size_t slot = (size_t)p.slot_floats * 4;
-  p.plan = reinterpret_cast<long long *>(w);
-  w += round_up((size_t)(p.B + 1) * 8, kAlign);
-  p.slots8 = reinterpret_cast<float *>(w);
-  if (has8) w += round_up((size_t)p.B * p.Hkv * slot, kAlign);
-  p.slots4 = reinterpret_cast<float *>(w);
-  (void)D;
+  p.plan = reinterpret_cast<int *>(w);
+  w += round_up((size_t)(p.B + 1) * 4, kAlign);
+  p.segs = reinterpret_cast<long long *>(w);
+  w += round_up((size_t)(p.num_workers + 1) * 8, kAlign);
+  p.slots = reinterpret_cast<float *>(w);
 }
 
 kv4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA; }
@@ -214,7 +214,8 @@ kv4_status kv4_append(kv4_cache *cache, void *stream, const void *k_new, const v
   if (B < 0 || total_new < 0 || pt_stride < 1) return KV4_ERR_INVALID;
   if (B == 0 || total_new == 0) return KV4_OK;
   if (B > cache->cfg.max_seqs) return KV4_ERR_CAPACITY;
-  if (!k_new || !v_new || !new_offsets || !seq_lens_old || !page_table) return KV4_ERR_INVALID;
+  if (!k_new || !v_new || !seq_lens_old || !page_table) return KV4_ERR_INVALID;
+  if (!new_offsets && total_new != B) return KV4_ERR_INVALID;
   const int D = cache->cfg.head_dim;
   if (!aligned(k_new, 8) || !aligned(v_new, 8)) return KV4_ERR_INVALID;
   AppendParams p{};
@@ -250,8 +251,7 @@ kv4_status kv4_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t num_q_
   int sms = 0;
   if (geometry(cache->cfg.head_dim, G, false, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
   const int nw = resolve_workers(num_workers, l, sms);
-  const bool has8 = cache->cfg.sink + cache->cfg.recent > 0;
-  *bytes = decode_ws_bytes(B, Hkv, G, cache->cfg.head_dim, nw, has8);
+  *bytes = decode_ws_bytes(B, Hkv, G, cache->cfg.head_dim, nw);
   return KV4_OK;
 }
 
@@ -262,6 +262,7 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   if (!cache || B < 0 || pt_stride < 1 || num_workers < 0) return KV4_ERR_INVALID;
   if (B == 0) return KV4_OK;
   if (B > cache->cfg.max_seqs) return KV4_ERR_CAPACITY;
+  if (B > kMaxBatch) return KV4_ERR_UNSUPPORTED;
   const int Hkv = cache->cfg.num_kv_heads, D = cache->cfg.head_dim;
   if (Hq < 1 || Hq % Hkv) return KV4_ERR_INVALID;
   const int G = Hq / Hkv;
@@ -275,7 +276,7 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   if (geometry(D, G, false, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
   const int nw = resolve_workers(num_workers, l, sms);
   const bool has8 = cache->cfg.sink + cache->cfg.recent > 0;
-  if (ws_bytes < decode_ws_bytes(B, Hkv, G, D, nw, has8)) return KV4_ERR_INVALID;
+  if (ws_bytes < decode_ws_bytes(B, Hkv, G, D, nw)) return KV4_ERR_INVALID;
 
   DecodeParams p{};
   p.B = B;
@@ -305,7 +306,7 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   p.out_fp32 = out_is_fp32 ? 1 : 0;
   p.err = cache->err;
   p.wait_cap = cache->wait_cap;
-  carve_workspace(p, workspace, D, has8);
+  carve_workspace(p, workspace);
   cudaEvent_t e0, e1;
   timing_pair(0, &e0, &e1);
   return cuda_status(launch_decode(p, D, false, static_cast<cudaStream_t>(stream), e0, e1));
@@ -344,7 +345,7 @@ kv4_status bf16_paged_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_
   DecodeLaunch l{};
   int sms = 0;
   if (geometry(D, G, true, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
-  *bytes = decode_ws_bytes(B, Hkv, G, D, resolve_workers(num_workers, l, sms), false);
+  *bytes = decode_ws_bytes(B, Hkv, G, D, resolve_workers(num_workers, l, sms));
   return KV4_OK;
 }
 
@@ -356,6 +357,7 @@ kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32
   if (B < 0 || Hkv < 1 || Hq < 1 || Hq % Hkv || pt_stride < 1 || num_pages < 1 || num_workers < 0)
     return KV4_ERR_INVALID;
   if (B == 0) return KV4_OK;
+  if (B > kMaxBatch) return KV4_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
   if ((G != 1 && G != 2 && G != 4) || (D != 64 && D != 128)) return KV4_ERR_UNSUPPORTED;
   if (!q || !kv_pages || !page_table || !seq_lens || !workspace || !out) return KV4_ERR_INVALID;
@@ -366,7 +368,7 @@ kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32
   int sms = 0;
   if (geometry(D, G, true, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
   const int nw = resolve_workers(num_workers, l, sms);
-  if (ws_bytes < decode_ws_bytes(B, Hkv, G, D, nw, false)) return KV4_ERR_INVALID;
+  if (ws_bytes < decode_ws_bytes(B, Hkv, G, D, nw)) return KV4_ERR_INVALID;
   DecodeParams p{};
   p.B = B;
   p.Hq = Hq;
@@ -389,7 +391,7 @@ kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32
   p.out_fp32 = out_is_fp32 ? 1 : 0;
   p.err = error_word;
   p.wait_cap = kDefaultWaitCycles;
-  carve_workspace(p, workspace, D, false);
+  carve_workspace(p, workspace);
   cudaEvent_t e0, e1;
   timing_pair(1, &e0, &e1);
   return cuda_status(launch_decode(p, D, true, static_cast<cudaStream_t>(stream), e0, e1));

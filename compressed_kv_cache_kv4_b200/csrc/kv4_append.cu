@@ -7,24 +7,34 @@
 // head_dim elements, INT8 per token row; scale = max|x| / qmax rounded toward
 // +inf to fp16; code = x / scale rounded to nearest-even.
 //
-// One warp per (new position, KV head). Lane l holds D/32 consecutive
-// elements. fp32 IEEE division followed by round-up to fp16 equals rounding
-// the exact quotient a/7 (a/127) up: a bf16 numerator over 7 (127) is never an
-// fp16 value unless exact, so the fp32 rounding cannot land on the boundary.
-// x/scale in fp32 is at least 2^-10 away from any half-integer it is not equal
-// to, so rintf of the fp32 quotient is the exact nearest-even code.
+// One warp per (new position, KV head); lane l holds D/32 consecutive elements.
+//
+// Scale: fp32 IEEE division then round-up to fp16 equals rounding the exact
+// quotient a/7 (a/127) up: for a bf16 numerator the quotient is either exact
+// or has a periodic binary expansion whose bits past the fp16 precision are
+// never all zero, so the fp32 rounding cannot land on an fp16 value.
+// Code: x/s differs from every half-integer it is not equal to by at least
+// 2^-10, while x * RN(1/s) differs from x/s by less than 2^-20, so rounding
+// x * RN(1/s) to the nearest integer is exact except at true half-way points;
+// those are detected exactly through the residual c*s - x (exact in fp32) and
+// resolved to the even code.
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
 
 namespace kv4 {
 
-template <int D>
-struct AppendLane {
-  static constexpr int EPL = D / 32;          // elements per lane
-  static constexpr int LPG = kGroup / EPL;    // lanes per INT4 group
-};
-
 __device__ __forceinline__ uint32_t nib(int c) { return static_cast<uint32_t>(c) & 0xFu; }
+
+// Nearest-even integer to x/s (s > 0), given r = RN(1/s).
+__device__ __forceinline__ float round_code(float x, float s, float r) {
+  float c = rintf(x * r);
+  const float d = fmaf(c, s, -x);   // c*s - x, exact
+  if (2.f * fabsf(d) == s) {        // half-way: x/s = c - sign(d)/2
+    const float other = c - copysignf(1.f, d);
+    c = (fmodf(c, 2.f) == 0.f) ? c : other;
+  }
+  return c;
+}
 
 // Quantise this lane's EPL values with a scale shared by `span` lanes
 // (span = lanes per group for INT4, 32 for INT8). Returns the fp16 scale bits.
@@ -40,43 +50,48 @@ __device__ __forceinline__ uint16_t quant_lane(const float (&x)[EPL], int span, 
     for (int e = 0; e < EPL; ++e) c[e] = 0;
     return 0;
   }
-  __half hs = __float2half_ru(__fdiv_rn(a, qmax));
-  uint16_t bits = __half_as_ushort(hs);
+  uint16_t bits = __half_as_ushort(__float2half_ru(__fdiv_rn(a, qmax)));
   if (bits == 0x7C00u) {           // a/qmax > 65504: saturate and flag
     bits = 0x7BFFu;
     set_error(err, kErrRange);
   }
   const float s = half_bits_to_f32(bits);
-  const int q = static_cast<int>(qmax);
+  const float r = __frcp_rn(s);
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
-    int v = static_cast<int>(rintf(__fdiv_rn(x[e], s)));
-    c[e] = v > q ? q : (v < -q ? -q : v);
+    const float v = fminf(fmaxf(round_code(x[e], s, r), -qmax), qmax);
+    c[e] = static_cast<int>(v);
   }
   return bits;
 }
 
 template <int D>
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
-  constexpr int EPL = AppendLane<D>::EPL;
-  constexpr int LPG = AppendLane<D>::LPG;
+  constexpr int EPL = D / 32;              // elements per lane
+  constexpr int LPG = kGroup / EPL;        // lanes per INT4 group
   const int lane = threadIdx.x & 31;
   const long long task = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (task >= p.T * p.Hkv) return;
   const long long j = task / p.Hkv;
   const int h = static_cast<int>(task % p.Hkv);
 
-  // sequence owning row j: largest b with offsets[b] <= j
-  int lo = 0, hi = p.B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.offsets[mid] <= j) lo = mid;
-    else hi = mid - 1;
+  int b, pos, L_new;
+  if (p.offsets) {
+    // sequence owning row j: largest b with offsets[b] <= j
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.offsets[mid] <= j) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+    pos = p.lens_old[b] + static_cast<int>(j - p.offsets[b]);
+    L_new = p.lens_old[b] + (p.offsets[b + 1] - p.offsets[b]);
+  } else {
+    b = static_cast<int>(j);   // one new position per sequence
+    pos = p.lens_old[b];
+    L_new = pos + 1;
   }
-  const int b = lo;
-  const int n_new = p.offsets[b + 1] - p.offsets[b];
-  const int pos = p.lens_old[b] + static_cast<int>(j - p.offsets[b]);
-  const int L_new = p.lens_old[b] + n_new;
   if (pos < 0 || pos >= p.pt_stride * kPageTokens) {
     if (lane == 0) set_error(p.err, kErrCapacity);
     return;
@@ -93,9 +108,9 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
 
   const int S = p.sink, R = p.recent;
   const int sink_row = pos < S ? pos : -1;
-  const int ring_row = (R > 0 && pos >= L_new - R) ? S + pos % R : -1;
-  const int rows = S + R;
+  const int ring_row = (R > 0 && pos >= L_new - R) ? (S > 0 ? 16 : 0) + pos % R : -1;
   uint8_t *sblk = p.side + ((long long)b * p.Hkv + h) * p.side_stride;
+  const long long spage = 32LL * D + 64;
 
 #pragma unroll
   for (int kv = 0; kv < 2; ++kv) {
@@ -128,8 +143,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
       }
       if (d0 % kGroup == 0) *reinterpret_cast<uint16_t *>(blk + 16 * D + 2 * (r * (D / 32) + grp)) = s4;
     } else {
-      // V: the byte of (slot r, element d) pairs d and d+8; its partner lane is
-      // 8/EPL lanes up.
+      // V: the byte of (slot r, element d) pairs d and d+8, held 8/EPL lanes up
       int partner[EPL];
 #pragma unroll
       for (int e = 0; e < EPL; ++e) partner[e] = __shfl_down_sync(0xffffffffu, c[e], 8 / EPL);
@@ -138,8 +152,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
         for (int e = 0; e < EPL; ++e) {
           const int d = d0 + e;
           const int m = d / 16, g = d % 8, tt = (r % 8) / 2;
-          const int lanev = 4 * g + tt;
-          const int word = (m / 4) * 128 + lanev * 4 + (m % 4);
+          const int word = (m / 4) * 128 + (4 * g + tt) * 4 + (m % 4);
           blk[8 * D + 4 * word + 2 * (r % 2) + r / 8] = static_cast<uint8_t>(nib(c[e]) | nib(partner[e]) << 4);
         }
       }
@@ -150,18 +163,47 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     if (sink_row >= 0 || ring_row >= 0) {
       int c8[EPL];
       const uint16_t s8 = quant_lane<EPL>(x, 32, 127.f, c8, p.err);
-      uint32_t packed = 0;
+      int partner8[EPL];
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) packed |= (static_cast<uint32_t>(c8[e]) & 0xFFu) << (8 * e);
+      for (int e = 0; e < EPL; ++e) partner8[e] = __shfl_down_sync(0xffffffffu, c8[e], 8 / EPL);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const int row = which == 0 ? sink_row : ring_row;
         if (row < 0) continue;
-        uint8_t *cdst = sblk + (long long)kv * rows * D + (long long)row * D + d0;
-        if constexpr (EPL == 4) *reinterpret_cast<uint32_t *>(cdst) = packed;
-        else *reinterpret_cast<uint16_t *>(cdst) = static_cast<uint16_t>(packed);
-        if (lane == 0)
-          *reinterpret_cast<uint16_t *>(sblk + 2LL * rows * D + 2LL * kv * rows + 2LL * row) = s8;
+        uint8_t *pg = sblk + (long long)(row / 16) * spage;
+        const int rr = row % 16;
+        if (kv == 0) {
+          // K row rr, element d: lane 4*(rr%8) + d/(D/4), word (rr/8)*(D/16) + (d%(D/4))/4, byte d%4
+          const int t = d0 / (D / 4), jw = (d0 % (D / 4)) / 4;
+          const int lanek = 4 * (rr % 8) + t;
+          const int w = (rr / 8) * (D / 16) + jw;
+          uint8_t *dst = pg + (w / 4) * 512 + lanek * 16 + (w % 4) * 4 + d0 % 4;
+          if constexpr (EPL == 4) {
+            uint32_t packed = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) packed |= (static_cast<uint32_t>(c8[e]) & 0xFFu) << (8 * e);
+            *reinterpret_cast<uint32_t *>(dst) = packed;
+          } else {
+            *reinterpret_cast<uint16_t *>(dst) =
+                static_cast<uint16_t>((static_cast<uint32_t>(c8[0]) & 0xFFu) | (static_cast<uint32_t>(c8[1]) & 0xFFu) << 8);
+          }
+          if (lane == 0) *reinterpret_cast<uint16_t *>(pg + 16 * D + 2 * rr) = s8;
+        } else {
+          // V row rr, element d: lane 4*(d%8) + (rr%8)/2, word 2*(d/16) + rr/8,
+          // bytes 2*(rr%2) + {0: d, 1: d+8}
+          if ((d0 % 16) < 8) {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) {
+              const int d = d0 + e;
+              const int lanev = 4 * (d % 8) + (rr % 8) / 2;
+              const int w = 2 * (d / 16) + rr / 8;
+              const uint32_t pair = (static_cast<uint32_t>(c8[e]) & 0xFFu) | (static_cast<uint32_t>(partner8[e]) & 0xFFu) << 8;
+              *reinterpret_cast<uint16_t *>(pg + 16 * D + 64 + (w / 4) * 512 + lanev * 16 + (w % 4) * 4 +
+                                            2 * (rr % 2)) = static_cast<uint16_t>(pair);
+            }
+          }
+          if (lane == 0) *reinterpret_cast<uint16_t *>(pg + 16 * D + 32 + 2 * rr) = s8;
+        }
       }
     }
   }

@@ -122,6 +122,33 @@ __device__ __forceinline__ uint32_t i4x2_to_bf16x2(uint32_t w) {
   return d;
 }
 
+// Same LOP3 without the subtraction: bf16x2 of 136 + c (the offset is removed
+// elsewhere, e.g. through the MMA accumulator's initial value).
+__device__ __forceinline__ uint32_t i4x2_biased(uint32_t w) {
+  uint32_t t;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x000F000Fu), "r"(0x43084308u));
+  return t;
+}
+
+// Two signed 8-bit codes at bits 0-7 and 16-23 of w -> fp16x2 of the codes.
+// LOP3 computes (w & 0x00FF00FF) ^ 0x64806480: flipping bit 7 turns c into
+// c + 128, and 0x64 above it makes the fp16 value 1024 + (c + 128).
+// Subtracting 1152 (fp16 0x6480) is exact.
+__device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t w) {
+  uint32_t t, d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x00FF00FFu), "r"(0x64806480u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(t), "r"(0x64806480u));
+  return d;
+}
+
+// D = A * B + C with A 16x16 (row), B 16x8 (col) fp16, C/D fp32.
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -131,6 +158,18 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float f16lo_to_f32(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(v & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16hi_to_f32(uint32_t v) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
 }
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
@@ -152,18 +191,6 @@ __device__ __forceinline__ int int4_num_pages(int L, int sink, int recent) {
   const int hi = L - recent;
   if (hi <= sink) return 0;
   return (hi + kPageTokens - 1) / kPageTokens - sink / kPageTokens;
-}
-
-// Static split of the flat (sequence, KV head, page) space among `nw` workers.
-// Worker w owns [seg_start(w), seg_start(w+1)); workers with more INT8 units get
-// proportionally fewer INT4 page-heads (an INT8 unit weighs `w8` page-heads).
-__device__ __forceinline__ long long seg_start(long long w, long long T4, long long U8, long long nw,
-                                               long long w8) {
-  if (w >= nw) return T4;
-  if (U8 == 0 || T4 < (w8 + 1) * nw) return w * T4 / nw;
-  const long long total = T4 + w8 * U8;
-  const long long cum8 = w * (U8 / nw) + (w < U8 % nw ? w : U8 % nw);
-  return w * total / nw - w8 * cum8;
 }
 
 }  // namespace kv4

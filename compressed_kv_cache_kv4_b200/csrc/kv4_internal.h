@@ -32,9 +32,9 @@ struct DecodeParams {
   const uint8_t *side;          // INT8 side blocks
   long long page_bytes, head_bytes, side_stride;
   float scale_log2;             // softmax_scale * log2(e)
-  long long *plan;              // [B+1] prefix of attended page-heads
-  float *slots8;                // [B*Hkv][slot_floats]
-  float *slots4;                // [B*Hkv + num_workers][slot_floats]
+  int *plan;                    // [B+1] prefix of attended INT4/bf16 page-heads
+  long long *segs;              // [num_workers+1] first item of each worker
+  float *slots;                 // [2*B*Hkv + num_workers][slot_floats] partials
   void *out;
   int out_fp32;
   uint32_t *err;
@@ -50,9 +50,8 @@ struct TopkParams {
   int32_t *count;
 };
 
-// Weight of one INT8 unit (<= 144 positions of one KV head, fp32 SIMT) in
-// INT4 page-head units when splitting work among workers.
-constexpr long long kInt8UnitWeight = 16;
+// Largest batch kv4_decode_attn accepts (the per-CTA plan lives in shared memory).
+constexpr int kMaxBatch = 8192;
 
 struct DecodeLaunch {
   int smem_bytes;
@@ -61,6 +60,7 @@ struct DecodeLaunch {
 
 cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream);
 cudaError_t decode_prepare(int D, int G, bool bf16, DecodeLaunch *out);
+int decode_smem_bytes(int D, bool bf16, int B);
 cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t stream, cudaEvent_t ev0,
                           cudaEvent_t ev1);
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream);

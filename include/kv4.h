@@ -65,7 +65,7 @@ typedef struct {
   int32_t page_tokens;   /* positions per page: must be 16 */
   int32_t group;         /* INT4 group along head_dim: must be 32 */
   int32_t sink;          /* INT8 sink positions: 0..16 (16 in KV4-RL) */
-  int32_t recent;        /* INT8 recent window: 0..128 (128 in KV4-RL) */
+  int32_t recent;        /* INT8 recent window: 0..128, a multiple of 16 (128 in KV4-RL) */
   int32_t max_seqs;      /* sequence slots in the side cache */
   int32_t num_pages;     /* physical pages in the pool */
 } kv4_config;
@@ -81,10 +81,12 @@ const char *kv4_status_string(kv4_status s);
  *    head: per head a block of 18*D bytes = K codes 8D | V codes 8D |
  *    K scales D | V scales D (INT4 nibbles in the register-fragment order the
  *    decode kernel consumes; fp16 scales [slot][group]).
- *  side_cache_bytes: max_seqs * Hkv INT8 blocks, one per (sequence, KV head):
- *    rows 0..sink-1 hold sink positions, rows sink..sink+recent-1 the ring
- *    (position p in ring row p mod recent); K codes | V codes | K scales | V
- *    scales, padded to 16 bytes.
+ *  side_cache_bytes: max_seqs * Hkv INT8 blocks, one per (sequence, KV head).
+ *    A block is a sequence of 16-row pages: a sink page when sink > 0 (position
+ *    p < sink in row p), then recent/16 ring pages (position p in ring slot
+ *    p mod recent). A page is K codes 16*D | K scales 16 x fp16 | V scales
+ *    16 x fp16 | V codes 16*D (32*D + 64 bytes), codes in the register-fragment
+ *    order of the fp16 decode tiles.
  * [KV4RL] sec. 3 (paged INT4 full context; bounded INT8 side cache).
  * Host only; no CUDA call.
  */
@@ -107,7 +109,9 @@ void kv4_cache_destroy(kv4_cache *cache);
  * kv4_append -- quantise new K/V positions into the cache ([KV4RL] sec. 3).
  *  k_new, v_new: device bf16 [T][Hkv][D], the new positions of all sequences
  *    concatenated; sequence b owns rows new_offsets[b] .. new_offsets[b+1]-1.
- *  new_offsets: device int32 [B+1], non-decreasing, new_offsets[0] = 0.
+ *  new_offsets: device int32 [B+1], non-decreasing, new_offsets[0] = 0; or
+ *    NULL for the decode-step case of exactly one new position per sequence
+ *    (then total_new must equal B and row b belongs to sequence b).
  *  seq_lens_old: device int32 [B], positions already cached (read only; the
  *    caller adds the new counts afterwards).
  *  page_table: device int32 [B][pt_stride]; logical page p/16 of sequence b
@@ -125,7 +129,8 @@ kv4_status kv4_append(kv4_cache *cache, void *stream, const void *k_new, const v
 /*
  * kv4_workspace_bytes -- device scratch needed by kv4_decode_attn for B
  * sequences and Hq query heads with `num_workers` parallel workers (0 = the
- * library's default for this device). Host only.
+ * library's default for this device). Queries the current device once per
+ * process (kernel attributes and occupancy); enqueues nothing.
  */
 kv4_status kv4_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t num_q_heads,
                                int32_t num_workers, size_t *bytes);

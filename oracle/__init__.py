@@ -50,6 +50,16 @@ def lib():
             f.argtypes = [C.c_int, C.c_int, C.c_int]
         L.kv4o_side_head_bytes.restype = C.c_int64
         L.kv4o_side_head_bytes.argtypes = [C.c_int, C.c_int, C.c_int]
+        L.kv4o_side_pages.restype = C.c_int
+        L.kv4o_side_pages.argtypes = [C.c_int, C.c_int]
+        L.kv4o_side_page_bytes.restype = C.c_int64
+        L.kv4o_side_page_bytes.argtypes = [C.c_int]
+        for f in (L.kv4o_side_k_byte, L.kv4o_side_v_byte):
+            f.restype = C.c_int64
+            f.argtypes = [C.c_int, C.c_int, C.c_int]
+        for f in (L.kv4o_side_ks_byte, L.kv4o_side_vs_byte):
+            f.restype = C.c_int64
+            f.argtypes = [C.c_int, C.c_int]
         L.kv4o_write_cache.restype = C.c_int
         L.kv4o_write_cache.argtypes = [C.POINTER(Shape), P, P, C.c_int, P, P, C.c_int,
                                        P, C.c_int64, P, C.c_int64]
@@ -139,6 +149,30 @@ def v_scale_byte(D, r, grp):
 
 def side_head_bytes(D, sink, recent):
     return int(lib().kv4o_side_head_bytes(D, sink, recent))
+
+
+def side_pages(sink, recent):
+    return int(lib().kv4o_side_pages(sink, recent))
+
+
+def side_page_bytes(D):
+    return int(lib().kv4o_side_page_bytes(D))
+
+
+def side_k_byte(D, row, d):
+    return int(lib().kv4o_side_k_byte(D, row, d))
+
+
+def side_v_byte(D, row, d):
+    return int(lib().kv4o_side_v_byte(D, row, d))
+
+
+def side_ks_byte(D, row):
+    return int(lib().kv4o_side_ks_byte(D, row))
+
+
+def side_vs_byte(D, row):
+    return int(lib().kv4o_side_vs_byte(D, row))
 
 
 def shape(B, Hq, Hkv, D, sink=16, recent=128):

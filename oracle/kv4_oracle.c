@@ -144,14 +144,47 @@ int64_t kv4o_v_code_byte(int D, int r, int d, int *nibble) {
 int64_t kv4o_k_scale_byte(int D, int r, int grp) { return 16LL * D + 2LL * (r * (D / 32) + grp); }
 int64_t kv4o_v_scale_byte(int D, int r, int grp) { return 17LL * D + 2LL * (r * (D / 32) + grp); }
 
-/* INT8 side block per (sequence, KV head): rows 0..S-1 are sink slots,
- * rows S..S+R-1 are ring slots (position p lives in ring slot p mod R).
- *   [K codes (S+R)*D][V codes (S+R)*D][K scales (S+R) fp16][V scales (S+R) fp16]
- * rounded up to a multiple of 16 bytes. */
+/* INT8 side block per (sequence, KV head): a sequence of 16-row pages. With
+ * sink > 0 the first page holds sink rows 0..15 (position p < sink in row p);
+ * then recent/16 ring pages hold ring slots 0..recent-1 (position p in slot
+ * p mod recent, page 16-slot blocks in slot order). Each page is
+ *   [K codes 16*D][K scales 16 x fp16][V scales 16 x fp16][V codes 16*D]
+ * and the codes of a page are in register-fragment order:
+ *   K row r, element d: t = d / (D/4), j = (d % (D/4)) / 4, e = d % 4,
+ *     lane = 4*(r%8) + t, word w = (r/8)*(D/16) + j,
+ *     byte = (w/4)*512 + lane*16 + (w%4)*4 + e.
+ *   V row r, element d: m = d/16, g = d%8, lane = 4*g + (r%8)/2,
+ *     word w = 2*m + r/8, byte = (w/4)*512 + lane*16 + (w%4)*4 + 2*(r%2) + (d%16)/8.
+ */
+int kv4o_side_pages(int sink, int recent) { return (sink > 0 ? 1 : 0) + recent / 16; }
+int64_t kv4o_side_page_bytes(int D) { return 32LL * D + 64; }
 int64_t kv4o_side_head_bytes(int D, int sink, int recent) {
-  int64_t rows = sink + recent;
-  int64_t b = 2 * rows * D + 4 * rows;
-  return (b + 15) / 16 * 16;
+  return kv4o_side_pages(sink, recent) * kv4o_side_page_bytes(D);
+}
+
+int64_t kv4o_side_k_byte(int D, int row, int d) {
+  const int r = row % 16;
+  const int t = d / (D / 4), j = (d % (D / 4)) / 4, e = d % 4;
+  const int lane = 4 * (r % 8) + t;
+  const int w = (r / 8) * (D / 16) + j;
+  return (int64_t)(row / 16) * kv4o_side_page_bytes(D) + (w / 4) * 512 + lane * 16 + (w % 4) * 4 + e;
+}
+
+int64_t kv4o_side_v_byte(int D, int row, int d) {
+  const int r = row % 16;
+  const int m = d / 16, g = d % 8;
+  const int lane = 4 * g + (r % 8) / 2;
+  const int w = 2 * m + r / 8;
+  return (int64_t)(row / 16) * kv4o_side_page_bytes(D) + 16LL * D + 64 + (w / 4) * 512 + lane * 16 +
+         (w % 4) * 4 + 2 * (r % 2) + (d % 16) / 8;
+}
+
+int64_t kv4o_side_ks_byte(int D, int row) {
+  return (int64_t)(row / 16) * kv4o_side_page_bytes(D) + 16LL * D + 2 * (row % 16);
+}
+
+int64_t kv4o_side_vs_byte(int D, int row) {
+  return (int64_t)(row / 16) * kv4o_side_page_bytes(D) + 16LL * D + 32 + 2 * (row % 16);
 }
 
 static void put_nibble(uint8_t *p, int nibble, int code) {
@@ -208,21 +241,22 @@ int kv4o_write_cache(const kv4o_shape *sh, const uint16_t *k, const uint16_t *v,
           }
           put_u16(blk + kv4o_v_scale_byte(D, r, grp), sc);
         }
-        /* INT8 side cache: sink slot for p < S; ring slot p mod R for the
-         * last R positions. */
+        /* INT8 side cache: sink row p for p < S; ring slot p mod R for the
+         * last R positions. Rows count from the block start: the sink page
+         * (16 rows) comes first when S > 0. */
         uint8_t *sb = side + ((int64_t)b * Hkv + h) * side_stride;
-        const int64_t rows = S + R;
+        const int ring0 = S > 0 ? 16 : 0;
         int row = -1;
         for (int pass = 0; pass < 2; ++pass) {
           if (pass == 0) row = (p < S) ? p : -1;
-          else row = (R > 0 && p >= L - R) ? S + p % R : -1;
+          else row = (R > 0 && p >= L - R) ? ring0 + p % R : -1;
           if (row < 0) continue;
           flags |= kv4o_quant_int8(krow, D, &sc, codes);
-          for (int d = 0; d < D; ++d) sb[(int64_t)row * D + d] = (uint8_t)codes[d];
-          put_u16(sb + 2 * rows * D + 2 * row, sc);
+          for (int d = 0; d < D; ++d) sb[kv4o_side_k_byte(D, row, d)] = (uint8_t)codes[d];
+          put_u16(sb + kv4o_side_ks_byte(D, row), sc);
           flags |= kv4o_quant_int8(vrow, D, &sc, codes);
-          for (int d = 0; d < D; ++d) sb[rows * D + (int64_t)row * D + d] = (uint8_t)codes[d];
-          put_u16(sb + 2 * rows * D + 2 * rows + 2 * row, sc);
+          for (int d = 0; d < D; ++d) sb[kv4o_side_v_byte(D, row, d)] = (uint8_t)codes[d];
+          put_u16(sb + kv4o_side_vs_byte(D, row), sc);
         }
       }
     }

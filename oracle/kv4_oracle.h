@@ -63,6 +63,12 @@ int64_t kv4o_v_code_byte(int D, int r, int d, int *nibble);
 int64_t kv4o_k_scale_byte(int D, int r, int grp);
 int64_t kv4o_v_scale_byte(int D, int r, int grp);
 int64_t kv4o_side_head_bytes(int D, int sink, int recent); /* INT8 block per (seq, head) */
+int     kv4o_side_pages(int sink, int recent);             /* 16-row pages per block */
+int64_t kv4o_side_page_bytes(int D);                       /* 32*D + 64 */
+int64_t kv4o_side_k_byte(int D, int row, int d);           /* offsets inside one block */
+int64_t kv4o_side_v_byte(int D, int row, int d);
+int64_t kv4o_side_ks_byte(int D, int row);
+int64_t kv4o_side_vs_byte(int D, int row);
 
 /* Write the byte image that appending positions [0, lens[b]) of every sequence
  * leaves in the page pool and the side cache. k, v: bf16 bits [B][Lmax][Hkv][D].

@@ -277,3 +277,33 @@ def test_range_overflow_flag():
     assert flags == 1
     assert np.array_equal(c.cache.pool.cpu().numpy(), pool)
     assert np.array_equal(c.cache.side.cpu().numpy(), side)
+
+
+def test_append_exact_ties():
+    """Rows built so that x/scale is exactly k + 1/2 for many elements (INT4 and
+    INT8 scales that are powers of two): codes must round half to even."""
+    wl = small_wl([40], seed=35, Hq=4, Hkv=1)
+    c = Case(wl)
+    D = wl.D
+    rng = np.random.default_rng(0)
+    rows = []
+    for p in range(40):
+        e = float(2.0 ** int(rng.integers(-6, 4)))
+        row = np.zeros(D, np.float32)
+        for grp in range(D // 32):
+            vals = (rng.integers(-7, 7, size=32) + 0.5) * e          # ties for an INT4 scale of e
+            vals[int(rng.integers(0, 32))] = 7 * e * (1 if rng.random() < 0.5 else -1)
+            row[32 * grp: 32 * grp + 32] = vals
+        if p % 2:                                                   # INT8 ties: max 127 e
+            row = ((rng.integers(-127, 127, size=D) + 0.5) * e).astype(np.float32)
+            row[int(rng.integers(0, D))] = 127 * e
+        rows.append(row)
+    kt = torch.as_tensor(np.stack(rows)[:, None, :]).to(torch.bfloat16)
+    assert torch.equal(kt.float(), torch.as_tensor(np.stack(rows)[:, None, :]))   # exact in bf16
+    c.k = kt
+    c.v = -kt
+    c.make_cache()
+    c.append_all()
+    pool, side, _ = c.oracle_cache()
+    assert np.array_equal(c.cache.pool.cpu().numpy(), pool)
+    assert np.array_equal(c.cache.side.cpu().numpy(), side)

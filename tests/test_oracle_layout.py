@@ -32,9 +32,33 @@ def test_hand_computed_offsets():
     assert O.v_scale_byte(128, 3, 2) == 2176 + 28
     # D = 64: rows of 32 bytes, chunks of 8 bytes
     assert O.k_code_byte(64, 1, 40) == (32 + 8 + 4 + 0, 0)
-    # INT8 side block for 16 + 128 rows at D = 128: 2*144*128 + 4*144 = 37440 bytes
-    assert O.side_head_bytes(128, 16, 128) == 37440
-    assert O.side_head_bytes(64, 16, 128) == 19008
+    # INT8 side block: 1 sink page + 8 ring pages of 2*(16*D + 32) bytes
+    assert O.side_head_bytes(128, 16, 128) == 9 * 4160 == 37440
+    assert O.side_head_bytes(64, 16, 128) == 9 * 2112 and O.side_page_bytes(128) == 4160
+    assert O.side_head_bytes(128, 0, 0) == 0 and O.side_pages(0, 128) == 8
+    # side K, row 21 (ring page 1, row 5), element 70: t = 2, j = 1, e = 2; lane 22,
+    # word 1 -> 4160 + 0*512 + 22*16 + 4 + 2
+    assert O.side_k_byte(128, 21, 70) == 4160 + 352 + 6
+    # side V, row 9, element 37: m = 2, g = 5, t = 0, odd row, r/8 = 1 -> lane 20,
+    # word 5 -> 2112 (after K codes and both scale arrays) + 512 + 320 + 4 + 2 + 0
+    assert O.side_v_byte(128, 9, 37) == 2112 + 512 + 320 + 4 + 2
+    assert O.side_ks_byte(128, 17) == 4160 + 2048 + 2
+    assert O.side_vs_byte(128, 17) == 4160 + 2048 + 32 + 2
+
+
+def test_side_layout_is_a_bijection():
+    for D in (64, 128):
+        pb = O.side_page_bytes(D)
+        seen = set()
+        for row in range(16):
+            for d in range(D):
+                seen.add(O.side_k_byte(D, row, d))
+                seen.add(O.side_v_byte(D, row, d))
+            seen.add(O.side_ks_byte(D, row))
+            seen.add(O.side_ks_byte(D, row) + 1)
+            seen.add(O.side_vs_byte(D, row))
+            seen.add(O.side_vs_byte(D, row) + 1)
+        assert seen == set(range(pb))
 
 
 def test_layout_is_a_bijection():
@@ -104,6 +128,37 @@ def test_writer_matches_quantiser_through_fragment_view():
                     assert vs[r, grp] == sc and np.array_equal(V[r, 32 * grp: 32 * grp + 32], codes)
 
 
+def _decode_side_page_via_fragments(page, D):
+    """Read one INT8 side page the way the fp16 tensor-core fragments read it."""
+    w = page.view(np.uint32)
+    nk = 4 * D                                   # K codes: 16*D bytes = 4*D words
+    K = np.zeros((16, D), np.int32)
+    V = np.zeros((16, D), np.int32)
+    kw = w[: nk].reshape(D // 32, 32, 4)          # [chunk][lane][word in chunk]
+    vw = w[nk + 16: 2 * nk + 16].reshape(D // 32, 32, 4)
+    sb = lambda x, k: ((int(x) >> (8 * k)) & 0xFF) - (256 if (int(x) >> (8 * k)) & 0x80 else 0)
+    for lane in range(32):
+        g, t = lane // 4, lane % 4
+        for wi in range(D // 8):
+            # K: words 0..D/16-1 are row g, the rest row g+8; word j holds elements
+            # t*D/4 + 4j + (0..3) in bytes 0..3
+            x = kw[wi // 4, lane, wi % 4]
+            row = g + 8 * (wi // (D // 16))
+            j = wi % (D // 16)
+            for e in range(4):
+                K[row, t * (D // 4) + 4 * j + e] = sb(x, e)
+            # V: word 2m + r8 holds (slot 2t+8r8, dim 16m+g), (2t+8r8, 16m+g+8),
+            # (2t+8r8+1, 16m+g), (2t+8r8+1, 16m+g+8) in bytes 0..3
+            y = vw[wi // 4, lane, wi % 4]
+            m, r8 = wi // 2, wi % 2
+            for e, (tok, dd) in enumerate([(2 * t + 8 * r8, g), (2 * t + 8 * r8, g + 8),
+                                           (2 * t + 8 * r8 + 1, g), (2 * t + 8 * r8 + 1, g + 8)]):
+                V[tok, 16 * m + dd] = sb(y, e)
+    ks = page[16 * D: 16 * D + 32].view(np.uint16)
+    vs = page[16 * D + 32: 16 * D + 64].view(np.uint16)
+    return K, V, ks, vs
+
+
 def test_side_cache_sink_and_ring():
     wl = synth.workload("tiny")
     k, v, off = synth.gen_kv(wl)
@@ -113,23 +168,24 @@ def test_side_cache_sink_and_ring():
     vb = synth.bf16_bits(synth.pad_batch(v, off, range(wl.B)))
     _, side, _ = O.write_cache(sh, kb, vb, wl.lens, pt, npages, fill=0x5A)
     S, R, D = wl.sink, wl.recent, wl.D
-    rows = S + R
     stride = O.side_head_bytes(D, S, R)
+    pb = O.side_page_bytes(D)
     for b in range(wl.B):
         L = int(wl.lens[b])
         for h in range(wl.Hkv):
             blk = side[(b * wl.Hkv + h) * stride: (b * wl.Hkv + h + 1) * stride]
-            kc = blk[: rows * D].view(np.int8).reshape(rows, D)
-            vc = blk[rows * D: 2 * rows * D].view(np.int8).reshape(rows, D)
-            ksc = blk[2 * rows * D: 2 * rows * D + 2 * rows].view(np.uint16)
-            # sink rows hold positions 0..15
+            pages = [_decode_side_page_via_fragments(blk[i * pb: (i + 1) * pb], D) for i in range(stride // pb)]
+            # sink rows (page 0) hold positions 0..15
             for p in range(min(S, L)):
                 sc, codes, _ = O.quant_int8(kb[b, p, h])
-                assert ksc[p] == sc and np.array_equal(kc[p], codes)
-            # ring slot p % R holds the latest position with that residue
+                assert pages[0][2][p] == sc and np.array_equal(pages[0][0][p], codes)
+            # ring slot p % R (page 1 + slot/16) holds the latest position with that residue
             for p in range(max(0, L - R), L):
+                slot = p % R
                 sc, codes, _ = O.quant_int8(vb[b, p, h])
-                assert np.array_equal(vc[S + p % R], codes)
-            # slots never written keep the fill byte (sequence of 37 tokens)
+                pg = pages[1 + slot // 16]
+                assert pg[3][slot % 16] == sc and np.array_equal(pg[1][slot % 16], codes)
+            # ring slots never written keep the fill byte (sequence of 37 tokens)
             if L < R:
-                assert np.all(blk[(S + L) * D: (S + R) * D].view(np.uint8) == 0x5A)
+                for slot in range(L, R):
+                    assert blk[O.side_k_byte(D, 16 + slot, 0)] == 0x5A
