@@ -7,7 +7,8 @@
 // head_dim elements, INT8 per token row; scale = max|x| / qmax rounded toward
 // +inf to fp16; code = x / scale rounded to nearest-even.
 //
-// One warp per (new position, KV head); lane l holds D/32 consecutive elements.
+// One warp per (new position, KV head, K or V); lane l holds D/32 consecutive
+// elements.
 //
 // Scale: fp32 IEEE division then round-up to fp16 equals rounding the exact
 // quotient a/7 (a/127) up: for a bf16 numerator the quotient is either exact
@@ -71,9 +72,12 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   constexpr int LPG = kGroup / EPL;        // lanes per INT4 group
   const int lane = threadIdx.x & 31;
   const long long task = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (task >= p.T * p.Hkv) return;
-  const long long j = task / p.Hkv;
-  const int h = static_cast<int>(task % p.Hkv);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (task >= p.T * p.Hkv * 2) return;
+  const int kv = static_cast<int>(task & 1);   // 0: K, 1: V
+  const long long j = (task >> 1) / p.Hkv;
+  const int h = static_cast<int>((task >> 1) % p.Hkv);
 
   int b, pos, L_new;
   if (p.offsets) {
@@ -98,7 +102,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   }
   const int page = p.page_table[(long long)b * p.pt_stride + pos / kPageTokens];
   if (page < 0 || page >= p.num_pages) {
-    if (lane == 0) set_error(p.err, kErrBounds);
+    if (lane == 0 && kv == 0) set_error(p.err, kErrBounds);
     return;
   }
   const int r = pos % kPageTokens;
@@ -112,8 +116,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   uint8_t *sblk = p.side + ((long long)b * p.Hkv + h) * p.side_stride;
   const long long spage = 32LL * D + 64;
 
-#pragma unroll
-  for (int kv = 0; kv < 2; ++kv) {
+  {
     const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + (j * p.Hkv + h) * D + d0;
     float x[EPL];
     if constexpr (EPL == 4) {
@@ -210,13 +213,12 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
 }
 
 cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream) {
-  const long long tasks = p.T * p.Hkv;
+  const long long tasks = p.T * p.Hkv * 2;
   if (tasks == 0) return cudaSuccess;
   const int warps_per_block = 8;
-  const long long blocks = (tasks + warps_per_block - 1) / warps_per_block;
-  if (D == 128) append_kernel<128><<<(unsigned)blocks, 32 * warps_per_block, 0, stream>>>(p);
-  else append_kernel<64><<<(unsigned)blocks, 32 * warps_per_block, 0, stream>>>(p);
-  return cudaGetLastError();
+  const unsigned blocks = static_cast<unsigned>((tasks + warps_per_block - 1) / warps_per_block);
+  if (D == 128) return launch_pdl(append_kernel<128>, dim3(blocks), dim3(32 * warps_per_block), 0, stream, p);
+  return launch_pdl(append_kernel<64>, dim3(blocks), dim3(32 * warps_per_block), 0, stream, p);
 }
 
 }  // namespace kv4

@@ -31,6 +31,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Wait until the grids this one depends on (earlier work in the stream) have
+// completed and their writes are visible; a no-op without the launch attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next grid in the stream to start launching (it still waits in pdl_wait).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier + bulk copy
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -170,6 +177,11 @@ __device__ __forceinline__ float f16lo_to_f32(uint32_t v) {
 }
 __device__ __forceinline__ float f16hi_to_f32(uint32_t v) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(v >> 16)));
+}
+
+// Both fp16 halves of a 32-bit word as floats (low half in .x).
+__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<const __half2 *>(&v));
 }
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }

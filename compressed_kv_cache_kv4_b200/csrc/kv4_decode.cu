@@ -19,7 +19,8 @@
 //                  bf16 in registers), fp16 tiles for INT8 pages (int8 codes are
 //                  exact in fp16). Each worker writes one (m, l, o) partial per
 //                  (region, sequence, KV head) piece of its segment.
-//   merge_kernel   one warp per (sequence, query head) merges the partials.
+//   merge_kernel   one warp per (sequence, KV head) merges the partials of all
+//                  its query heads exactly.
 //
 // Softmax bookkeeping runs in the log2 domain (scores scaled by tau*log2 e).
 // P.V takes P*scale_V as two 16-bit terms (hi + lo), which carries 16 (bf16)
@@ -31,18 +32,32 @@
 
 namespace kv4 {
 
+#ifndef KV4_INT4_STAGES
+#define KV4_INT4_STAGES 4
+#endif
+#ifndef KV4_MIN_BLOCKS
+#define KV4_MIN_BLOCKS 4
+#endif
+
 template <int D, bool kBF16>
 struct Cfg {
-  static constexpr int NS = kBF16 ? 3 : 4;                  // stages per warp
+  static constexpr int NS = kBF16 ? 3 : KV4_INT4_STAGES;    // stages per warp
   static constexpr int ROWB = 2 * D + 16;                   // padded bf16 row in shared memory
   static constexpr int STAGE = kBF16 ? 2 * kPageTokens * ROWB : 18 * D;
   static constexpr int WARP_SMEM = NS * STAGE;
-  static constexpr int RINGS = kWarps * (WARP_SMEM + NS * 8);
+  // per-warp query operands: [chunk][lane][16 bytes]; INT4 pieces use D/32
+  // chunks of q fragments and (D/32 + 1)/2 chunks of accumulator starts,
+  // INT8 pieces D/32 chunks of fp16 q fragments
+  static constexpr int QCHUNKS = kBF16 ? 0 : D / 32 + (D / 32 + 1) / 2;
+  static constexpr int QBYTES = QCHUNKS * 512;
+  static constexpr int RINGS = kWarps * (WARP_SMEM + NS * 8 + QBYTES);
 };
 
 // Weights of one item when splitting work among workers: an INT4 page-head
 // (18*D bytes) counts 4, an INT8 side page (32*D + 64 bytes) counts 7.
 constexpr long long kW4 = 4, kW8 = 7;
+
+// (sequence, KV head) merges a worker postpones to the end of its segment.
 
 // First item of worker w among nw: items 0..T8-1 are INT8 pages (weight kW8),
 // then T4 INT4/bf16 pages (weight kW4); worker w starts at the first item whose
@@ -55,7 +70,7 @@ __device__ __forceinline__ long long worker_first_item(long long w, long long nw
   return T8 + (a - kW8 * T8 + kW4 - 1) / kW4;
 }
 
-__device__ __forceinline__ int side_pages(int sink, int recent) { return (sink > 0 ? 1 : 0) + recent / 16; }
+__host__ __device__ __forceinline__ int side_pages(int sink, int recent) { return (sink > 0 ? 1 : 0) + recent / 16; }
 
 // ---------------------------------------------------------------------------
 // Partial slot: m[G] | l[G] | pad | o[G][D]   (m in log2 units, o normalised)
@@ -110,28 +125,30 @@ __device__ __forceinline__ void softmax_update(SoftmaxState<NMT> &st, const floa
     }
     st.m[1] = mx1;
   }
-  const float r0 = st.m[0] == -INFINITY ? 0.f : st.m[0];
-  const float r1 = st.m[1] == -INFINITY ? 0.f : st.m[1];
-  pr[0] = ex2(s[0] - r0);
-  pr[1] = ex2(s[1] - r1);
-  pr[2] = ex2(s[2] - r0);
-  pr[3] = ex2(s[3] - r1);
-  st.l[0] += pr[0] + pr[2];
-  st.l[1] += pr[1] + pr[3];
+  const float2 r = make_float2(st.m[0] == -INFINITY ? 0.f : st.m[0], st.m[1] == -INFINITY ? 0.f : st.m[1]);
+  const float2 d01 = __fadd2_rn(make_float2(s[0], s[1]), make_float2(-r.x, -r.y));
+  const float2 d23 = __fadd2_rn(make_float2(s[2], s[3]), make_float2(-r.x, -r.y));
+  pr[0] = ex2(d01.x);
+  pr[1] = ex2(d01.y);
+  pr[2] = ex2(d23.x);
+  pr[3] = ex2(d23.y);
+  const float2 l = __fadd2_rn(make_float2(st.l[0], st.l[1]),
+                              __fadd2_rn(make_float2(pr[0], pr[1]), make_float2(pr[2], pr[3])));
+  st.l[0] = l.x;
+  st.l[1] = l.y;
 }
 
 // Weights w for (token g, col 2t/2t+1) and (token g+8, ...) -> the B fragment
 // (k = tokens, n = columns) of the P.V tile. Lanes with t < 2 contribute the
 // 16-bit rounding of w ("hi" columns 0-3); lanes with t >= 2 the 16-bit
 // rounding of the remainder ("lo" columns 4-7).
-__device__ __forceinline__ void weights_bf16(float w0, float w1, float w2, float w3, float lo_sel, uint32_t &b0,
-                                             uint32_t &b1) {
-  uint32_t h01 = pack_bf16x2(w0, w1);
-  uint32_t h23 = pack_bf16x2(w2, w3);
-  h01 = pack_bf16x2(fmaf(-lo_sel, bf16lo_to_f32(h01), w0), fmaf(-lo_sel, bf16hi_to_f32(h01), w1));
-  h23 = pack_bf16x2(fmaf(-lo_sel, bf16lo_to_f32(h23), w2), fmaf(-lo_sel, bf16hi_to_f32(h23), w3));
-  b0 = movmatrix_t(h01);
-  b1 = movmatrix_t(h23);
+__device__ __forceinline__ void weights_bf16(float2 w01, float2 w23, float2 neg_sel, uint32_t &b0, uint32_t &b1) {
+  uint32_t h01 = pack_bf16x2(w01.x, w01.y);
+  uint32_t h23 = pack_bf16x2(w23.x, w23.y);
+  const float2 r01 = __ffma2_rn(neg_sel, make_float2(bf16lo_to_f32(h01), bf16hi_to_f32(h01)), w01);
+  const float2 r23 = __ffma2_rn(neg_sel, make_float2(bf16lo_to_f32(h23), bf16hi_to_f32(h23)), w23);
+  b0 = movmatrix_t(pack_bf16x2(r01.x, r01.y));
+  b1 = movmatrix_t(pack_bf16x2(r23.x, r23.y));
 }
 
 __device__ __forceinline__ void weights_f16(float w0, float w1, float w2, float w3, float lo_sel, uint32_t &b0,
@@ -254,6 +271,12 @@ __device__ __forceinline__ void load_batch(PageCursor &c, int base, const int32_
 
 __device__ __forceinline__ int next_page(PageCursor &c, int &pid, const int32_t *ptrow, int lo_tok, int hi_tok,
                                          const uint32_t *mrow, const DecodeParams &p, int lane) {
+  // common case: the next page is in the loaded batch and has work
+  const int idx0 = c.cursor - c.batch_base;
+  if (c.cursor < c.pg1 && idx0 < 32 && ((c.okbits >> idx0) & 1u)) {
+    pid = __shfl_sync(0xffffffffu, c.pid_reg, idx0);
+    return c.cursor++;
+  }
   while (c.cursor < c.pg1) {
     if (c.cursor >= c.batch_base + 32) load_batch(c, c.cursor, ptrow, lo_tok, hi_tok, mrow, p, lane);
     const int idx = c.cursor - c.batch_base;
@@ -283,25 +306,27 @@ __device__ __forceinline__ int next_page(PageCursor &c, int &pid, const int32_t 
 // ---------------------------------------------------------------------------
 template <int D, int G>
 __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, int pg1, uint8_t *wsm,
-                           uint64_t *bars, uint32_t &phase, float *slot, int lane) {
+                           uint64_t *bars, uint8_t *qsm, uint32_t &phase, float *slot, int lane) {
   using C = Cfg<D, false>;
   constexpr int NS = C::NS, NG = D / 32, NMT = D / 16, NSW = (NG + 1) / 2;
   const int g = lane >> 2, t = lane & 3;
 
-  uint32_t qf[NG][2][2];
-  float qinit[NG][2];   // -136 * sum of q over group i, for columns 2t and 2t+1
+  // q as the B operand, and -136 * (sum of q over group i) for columns 2t and
+  // 2t+1, parked in the warp's shared-memory q area for the whole piece
   {
     const int head = g & 3;
     const bool hv = head < G;
     const uint4 *qh = reinterpret_cast<const uint4 *>(p.q + ((long long)b * p.Hq + h * G + (hv ? head : 0)) * D);
+    float qinit[NG][2];
 #pragma unroll
     for (int i = 0; i < NG; ++i) {
       const uint4 e = hv ? qh[4 * i + t] : make_uint4(0, 0, 0, 0);
       // e.x = (e0, e1), e.y = (e2, e3), e.z = (e4, e5), e.w = (e6, e7)
-      qf[i][0][0] = __byte_perm(e.x, e.z, 0x5410);   // (e0, e4)
-      qf[i][0][1] = __byte_perm(e.x, e.z, 0x7632);   // (e1, e5)
-      qf[i][1][0] = __byte_perm(e.y, e.w, 0x5410);   // (e2, e6)
-      qf[i][1][1] = __byte_perm(e.y, e.w, 0x7632);   // (e3, e7)
+      *reinterpret_cast<uint4 *>(qsm + i * 512 + lane * 16) =
+          make_uint4(__byte_perm(e.x, e.z, 0x5410),    // (e0, e4)
+                     __byte_perm(e.x, e.z, 0x7632),    // (e1, e5)
+                     __byte_perm(e.y, e.w, 0x5410),    // (e2, e6)
+                     __byte_perm(e.y, e.w, 0x7632));   // (e3, e7)
       float part = bf16lo_to_f32(e.x) + bf16hi_to_f32(e.x) + bf16lo_to_f32(e.y) + bf16hi_to_f32(e.y) +
                    bf16lo_to_f32(e.z) + bf16hi_to_f32(e.z) + bf16lo_to_f32(e.w) + bf16hi_to_f32(e.w);
       part += __shfl_xor_sync(0xffffffffu, part, 1);
@@ -310,13 +335,21 @@ __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
       qinit[i][0] = -136.f * __shfl_sync(0xffffffffu, part, 8 * t);
       qinit[i][1] = -136.f * __shfl_sync(0xffffffffu, part, 8 * t + 4);
     }
+#pragma unroll
+    for (int c = 0; c < (NG + 1) / 2; ++c) {
+      const float a0 = qinit[2 * c][0], a1 = qinit[2 * c][1];
+      const float a2 = 2 * c + 1 < NG ? qinit[(2 * c + 1) % NG][0] : 0.f;
+      const float a3 = 2 * c + 1 < NG ? qinit[(2 * c + 1) % NG][1] : 0.f;
+      *reinterpret_cast<float4 *>(qsm + (NG + c) * 512 + lane * 16) = make_float4(a0, a1, a2, a3);
+    }
+    __syncwarp();
   }
 
   const int lo_tok = p.sink, hi_tok = L - p.recent;
   const uint32_t *mrow = p.mask ? p.mask + ((long long)b * p.Hkv + h) * p.mask_stride : nullptr;
   const int32_t *ptrow = p.page_table + (long long)b * p.pt_stride;
   const uint8_t *hbase = p.pool + (long long)h * p.head_bytes;
-  const float lo_sel = t >= 2 ? 1.f : 0.f;
+  const float2 neg_sel = t >= 2 ? make_float2(-1.f, -1.f) : make_float2(0.f, 0.f);
 
   SoftmaxState<NMT> st;
   st.reset();
@@ -365,27 +398,41 @@ __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
       vsw0[0] = *reinterpret_cast<const uint32_t *>(stg + 17 * D + g * 4);
       vsw1[0] = *reinterpret_cast<const uint32_t *>(stg + 17 * D + (g + 8) * 4);
     }
-    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    float ks0[NG], ks1[NG], vs0a[NG], vs1a[NG];
+#pragma unroll
+    for (int c = 0; c < NSW; ++c) {
+      const float2 a0 = f16x2_to_f32x2(ksw0[c]), a1 = f16x2_to_f32x2(ksw1[c]);
+      const float2 b0 = f16x2_to_f32x2(vsw0[c]), b1 = f16x2_to_f32x2(vsw1[c]);
+      ks0[2 * c] = a0.x; ks1[2 * c] = a1.x; vs0a[2 * c] = b0.x; vs1a[2 * c] = b1.x;
+      if (2 * c + 1 < NG) {
+        ks0[2 * c + 1] = a0.y; ks1[2 * c + 1] = a1.y; vs0a[2 * c + 1] = b0.y; vs1a[2 * c + 1] = b1.y;
+      }
+    }
+    float2 sc01 = make_float2(0.f, 0.f), sc23 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < NG; ++i) {
-      float acc[4] = {qinit[i][0], qinit[i][1], qinit[i][0], qinit[i][1]};
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const uint32_t a[4] = {i4x2_biased(kw0[i] >> (8 * j)), i4x2_biased(kw1[i] >> (8 * j)),
-                               i4x2_biased(kw0[i] >> (8 * j + 4)), i4x2_biased(kw1[i] >> (8 * j + 4))};
-        mma_bf16(acc, a, qf[i][j][0], qf[i][j][1]);
+      const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + i * 512 + lane * 16);
+      const float2 qi = *reinterpret_cast<const float2 *>(qsm + (NG + i / 2) * 512 + lane * 16 + (i & 1) * 8);
+      float acc[4] = {qi.x, qi.y, qi.x, qi.y};
+      {
+        const uint32_t a[4] = {i4x2_biased(kw0[i]), i4x2_biased(kw1[i]), i4x2_biased(kw0[i] >> 4),
+                               i4x2_biased(kw1[i] >> 4)};
+        mma_bf16(acc, a, qv.x, qv.y);
       }
-      const float k0 = (i & 1) ? f16hi_to_f32(ksw0[i >> 1]) : f16lo_to_f32(ksw0[i >> 1]);
-      const float k1 = (i & 1) ? f16hi_to_f32(ksw1[i >> 1]) : f16lo_to_f32(ksw1[i >> 1]);
-      sc[0] = fmaf(k0, acc[0], sc[0]);
-      sc[1] = fmaf(k0, acc[1], sc[1]);
-      sc[2] = fmaf(k1, acc[2], sc[2]);
-      sc[3] = fmaf(k1, acc[3], sc[3]);
+      {
+        const uint32_t a[4] = {i4x2_biased(kw0[i] >> 8), i4x2_biased(kw1[i] >> 8), i4x2_biased(kw0[i] >> 12),
+                               i4x2_biased(kw1[i] >> 12)};
+        mma_bf16(acc, a, qv.z, qv.w);
+      }
+      const float k0 = ks0[i], k1 = ks1[i];
+      sc01 = __ffma2_rn(make_float2(k0, k0), make_float2(acc[0], acc[1]), sc01);
+      sc23 = __ffma2_rn(make_float2(k1, k1), make_float2(acc[2], acc[3]), sc23);
     }
     // ---- which of the page's slots are attended (all of them on interior pages)
-    float sl[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) sl[k] = sc[k] * p.scale_log2;
+    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+    sc01 = __fmul2_rn(sc01, sl2);
+    sc23 = __fmul2_rn(sc23, sl2);
+    float sl[4] = {sc01.x, sc01.y, sc23.x, sc23.y};
     if (mrow || pg * kPageTokens < lo_tok || pg * kPageTokens + kPageTokens > hi_tok) {
       const int tok0 = pg * kPageTokens + g, tok1 = tok0 + 8;
       bool v0 = tok0 >= lo_tok && tok0 < hi_tok;
@@ -405,9 +452,9 @@ __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
     uint32_t wb[NG][2];
 #pragma unroll
     for (int i = 0; i < NG; ++i) {
-      const float vs0 = (i & 1) ? f16hi_to_f32(vsw0[i >> 1]) : f16lo_to_f32(vsw0[i >> 1]);
-      const float vs1 = (i & 1) ? f16hi_to_f32(vsw1[i >> 1]) : f16lo_to_f32(vsw1[i >> 1]);
-      weights_bf16(pr[0] * vs0, pr[1] * vs0, pr[2] * vs1, pr[3] * vs1, lo_sel, wb[i][0], wb[i][1]);
+      const float vs0 = vs0a[i], vs1 = vs1a[i];
+      weights_bf16(__fmul2_rn(make_float2(pr[0], pr[1]), make_float2(vs0, vs0)),
+                   __fmul2_rn(make_float2(pr[2], pr[3]), make_float2(vs1, vs1)), neg_sel, wb[i][0], wb[i][1]);
     }
     uint32_t vw[NMT];
 #pragma unroll
@@ -454,7 +501,7 @@ __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
 // ---------------------------------------------------------------------------
 template <int D, int G>
 __device__ bool int8_piece(const DecodeParams &p, int b, int h, int L, int j0, int j1, uint8_t *wsm,
-                           uint64_t *bars, uint32_t &phase, float *slot, int lane) {
+                           uint64_t *bars, uint8_t *qsm, uint32_t &phase, float *slot, int lane) {
   using C = Cfg<D, false>;
   constexpr int NS = C::NS, NJ = D / 16, NMT = D / 16, NW = D / 8;   // MMAs, M-tiles, words per lane
   constexpr int KHALF = 16 * D + 64, VHALF = 16 * D;
@@ -463,7 +510,7 @@ __device__ bool int8_piece(const DecodeParams &p, int b, int h, int L, int j0, i
   const int js = S > 0 ? 1 : 0;
   const int r0 = max(S, L - R);
 
-  uint32_t qf[NJ][2];
+  // fp16 q fragments of MMA j at q area chunk j/2, words 2*(j%2) + {0, 1}
   {
     const int head = g & 3;
     const bool hv = head < G;
@@ -473,14 +520,17 @@ __device__ bool int8_piece(const DecodeParams &p, int b, int h, int L, int j0, i
     for (int j = 0; j < NJ; ++j) {
       const int d = t * (D / 4) + 4 * j;
       const uint32_t e01 = hv ? qh[d / 2] : 0u, e23 = hv ? qh[d / 2 + 1] : 0u;
-      qf[j][0] = pack_f16x2(bf16lo_to_f32(e01), bf16lo_to_f32(e23));   // (q[d], q[d+2])
-      qf[j][1] = pack_f16x2(bf16hi_to_f32(e01), bf16hi_to_f32(e23));   // (q[d+1], q[d+3])
+      *reinterpret_cast<uint2 *>(qsm + (j / 2) * 512 + lane * 16 + (j % 2) * 8) =
+          make_uint2(pack_f16x2(bf16lo_to_f32(e01), bf16lo_to_f32(e23)),    // (q[d], q[d+2])
+                     pack_f16x2(bf16hi_to_f32(e01), bf16hi_to_f32(e23)));   // (q[d+1], q[d+3])
     }
+    __syncwarp();
   }
   const uint32_t *mrow = p.mask ? p.mask + ((long long)b * p.Hkv + h) * p.mask_stride : nullptr;
   const uint8_t *blk = p.side + ((long long)b * p.Hkv + h) * p.side_stride;
   const long long page_bytes8 = 32LL * D + 64;
   const float lo_sel = t >= 2 ? 1.f : 0.f;
+  (void)G;
 
   // position held by row r of page j, or -1 when the row is not attended
   auto row_pos = [&](int j, int r) -> int {
@@ -546,10 +596,14 @@ __device__ bool int8_piece(const DecodeParams &p, int b, int h, int L, int j0, i
       }
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int jj = 0; jj < NJ; ++jj) {
-        const uint32_t a[4] = {i8x2_to_f16x2(kw[jj]), i8x2_to_f16x2(kw[NJ + jj]), i8x2_to_f16x2(kw[jj] >> 8),
-                               i8x2_to_f16x2(kw[NJ + jj] >> 8)};
-        mma_f16(acc, a, qf[jj][0], qf[jj][1]);
+      for (int jj = 0; jj < NJ; jj += 2) {
+        const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + (jj / 2) * 512 + lane * 16);
+        const uint32_t a0[4] = {i8x2_to_f16x2(kw[jj]), i8x2_to_f16x2(kw[NJ + jj]), i8x2_to_f16x2(kw[jj] >> 8),
+                                i8x2_to_f16x2(kw[NJ + jj] >> 8)};
+        mma_f16(acc, a0, qv.x, qv.y);
+        const uint32_t a1[4] = {i8x2_to_f16x2(kw[jj + 1]), i8x2_to_f16x2(kw[NJ + jj + 1]),
+                                i8x2_to_f16x2(kw[jj + 1] >> 8), i8x2_to_f16x2(kw[NJ + jj + 1] >> 8)};
+        mma_f16(acc, a1, qv.z, qv.w);
       }
       const __half *ks = reinterpret_cast<const __half *>(stg + 16 * D);
       const __half *vs = reinterpret_cast<const __half *>(stg + 16 * D + 32);
@@ -620,7 +674,7 @@ __device__ bool bf16_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
   }
   const int32_t *ptrow = p.page_table + (long long)b * p.pt_stride;
   const uint8_t *hbase = p.pool + (long long)h * p.head_bytes;
-  const float lo_sel = t >= 2 ? 1.f : 0.f;
+  const float2 neg_sel = t >= 2 ? make_float2(-1.f, -1.f) : make_float2(0.f, 0.f);
 
   SoftmaxState<NMT> st;
   st.reset();
@@ -670,7 +724,7 @@ __device__ bool bf16_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
     float pr[4];
     softmax_update<NMT, 8>(st, sl, pr);
     uint32_t wb0, wb1;
-    weights_bf16(pr[0], pr[1], pr[2], pr[3], lo_sel, wb0, wb1);
+    weights_bf16(make_float2(pr[0], pr[1]), make_float2(pr[2], pr[3]), neg_sel, wb0, wb1);
 #pragma unroll
     for (int mt = 0; mt < NMT; ++mt) {
       uint32_t a[4];
@@ -691,15 +745,149 @@ __device__ bool bf16_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
 }
 
 // ---------------------------------------------------------------------------
+// The exact merge of one (sequence, KV head).
+// ---------------------------------------------------------------------------
+
+// out[b][h*G + g] for every query head g: M = max m_c, W_c = l_c 2^(m_c - M),
+// out = sum W_c o_c / sum W_c over the partials of (b, h) (0 if none). The
+// partials of a range sit in slots range + w for the contiguous workers
+// w = first[range] .. last[range]. Loads in three rounds: the range bounds,
+// every partial's (m, l) (lane k: partial k), then the output vectors (lane:
+// query head lane / (32/G), D*G/32 consecutive elements). All reads bypass L1:
+// the partials were written by other SMs.
+template <int D, int G>
+__device__ void merge_bh(const DecodeParams &p, int b, int h, int np8, int per, long long T8, long long T4,
+                         int lane) {
+  constexpr int LPH = 32 / G, DPL = D / LPH;
+  const int gq = lane / LPH, d0 = (lane % LPH) * DPL;
+  const long long nbh = (long long)p.B * p.Hkv;
+  const long long r = (long long)b * p.Hkv + h;
+  const long long f8 = np8 > 0 ? __ldcg(&p.first[r]) : 0, l8 = np8 > 0 ? __ldcg(&p.last[r]) : -1;
+  const long long f4 = per > 0 ? __ldcg(&p.first[nbh + r]) : 0, l4 = per > 0 ? __ldcg(&p.last[nbh + r]) : -1;
+  const int n8 = static_cast<int>(l8 - f8 + 1), n = n8 + static_cast<int>(l4 - f4 + 1);
+  float M = -INFINITY, den = 0.f, acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  for (int c0 = 0; c0 < n; c0 += 32) {
+    const int k = c0 + lane;
+    long long slot_idx = -1, w = -1;
+    if (k < n8) {
+      w = f8 + k;
+      slot_idx = r + w;
+    } else if (k < n) {
+      w = f4 + (k - n8);
+      slot_idx = nbh + r + w;
+    }
+    // a worker with an empty segment wrote no partial
+    if (w >= 0 && worker_first_item(w, p.num_workers, T8, T4) == worker_first_item(w + 1, p.num_workers, T8, T4))
+      slot_idx = -1;
+    // lane k: (m, l) of partial k for all heads
+    float mk[G], lk[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      mk[g] = -INFINITY;
+      lk[g] = 0.f;
+    }
+    if (slot_idx >= 0) {
+      const float *slot = p.slots + slot_idx * p.slot_floats;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        lk[g] = __ldcg(slot + G + g);
+        mk[g] = __ldcg(slot + g);
+      }
+    }
+    // every lane needs, for its head gq, the (m, l) of each partial kk: read
+    // them from lane kk with shuffles; first the head max, then the weights
+    float mc = -INFINITY;
+    const uint32_t pmask = __ballot_sync(0xffffffffu, slot_idx >= 0);
+    uint32_t rem = pmask;
+    while (rem) {
+      const int kk = __ffs(rem) - 1;
+      rem &= rem - 1;
+      float mg = -INFINITY, lg = 0.f;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float mv = __shfl_sync(0xffffffffu, mk[g], kk);
+        const float lv = __shfl_sync(0xffffffffu, lk[g], kk);
+        if (g == gq) {
+          mg = mv;
+          lg = lv;
+        }
+      }
+      if (lg > 0.f) mc = fmaxf(mc, mg);
+    }
+    if (mc > M) {
+      const float f = ex2(M - mc);
+      den *= f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] *= f;
+      M = mc;
+    }
+    rem = pmask;
+    while (rem) {
+      const int kk = __ffs(rem) - 1;
+      rem &= rem - 1;
+      float mg = -INFINITY, lg = 0.f;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float mv = __shfl_sync(0xffffffffu, mk[g], kk);
+        const float lv = __shfl_sync(0xffffffffu, lk[g], kk);
+        if (g == gq) {
+          mg = mv;
+          lg = lv;
+        }
+      }
+      const long long si = __shfl_sync(0xffffffffu, slot_idx, kk);
+      if (!(lg > 0.f)) continue;
+      const float wk = lg * ex2(mg - M);
+      den += wk;
+      const float2 *o = reinterpret_cast<const float2 *>(p.slots + si * p.slot_floats + p.slot_o_off + gq * D + d0);
+#pragma unroll
+      for (int e = 0; e < DPL / 2; ++e) {
+        const float2 v = __ldcg(o + e);
+        acc[2 * e + 0] = fmaf(wk, v.x, acc[2 * e + 0]);
+        acc[2 * e + 1] = fmaf(wk, v.y, acc[2 * e + 1]);
+      }
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const long long obase = ((long long)b * p.Hq + (long long)h * G + gq) * D + d0;
+  if (p.out_fp32) {
+    float2 *o = reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + obase);
+#pragma unroll
+    for (int e = 0; e < DPL / 2; ++e) o[e] = make_float2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  } else {
+    uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + obase);
+#pragma unroll
+    for (int e = 0; e < DPL / 2; ++e) o[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  }
+}
+
+// One warp per (sequence, KV head), after the worker grid has finished.
+template <int D, int G>
+__global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
+  const long long task = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (task >= (long long)p.B * p.Hkv) return;
+  const int b = static_cast<int>(task / p.Hkv), h = static_cast<int>(task % p.Hkv);
+  const int per = (__ldcg(&p.plan[b + 1]) - __ldcg(&p.plan[b])) / p.Hkv;
+  const long long T8 = (long long)p.B * p.Hkv * np8, T4 = __ldcg(&p.plan[p.B]);
+  merge_bh<D, G>(p, b, h, np8, per, T8, T4, lane);
+}
+
+// ---------------------------------------------------------------------------
 // Persistent worker kernel.
 // ---------------------------------------------------------------------------
 template <int D, int G, bool kBF16>
-__global__ void __launch_bounds__(kWarps * 32, 4) decode_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) decode_kernel(DecodeParams p) {
   using C = Cfg<D, kBF16>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t *wsm = smem + warp * C::WARP_SMEM;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kWarps * C::WARP_SMEM) + warp * C::NS;
+  uint8_t *qsm = smem + kWarps * (C::WARP_SMEM + C::NS * 8) + warp * C::QBYTES;
   int *plan = reinterpret_cast<int *>(smem + C::RINGS);   // [B + 1]
   __shared__ int wtot[kWarps];
 
@@ -708,6 +896,8 @@ __global__ void __launch_bounds__(kWarps * 32, 4) decode_kernel(DecodeParams p) 
     for (int s = 0; s < C::NS; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
+  pdl_wait();                 // inputs and cache writes of earlier grids are visible from here
+  pdl_launch_dependents();    // the merge grid may queue behind the workers
 
   // plan[b] = sum over b' < b of (attended pages of b') * Hkv, computed by the CTA
   const int cap = p.pt_stride * kPageTokens;
@@ -754,11 +944,11 @@ __global__ void __launch_bounds__(kWarps * 32, 4) decode_kernel(DecodeParams p) 
     p.segs[wid] = x;
     if (wid == NWk - 1) p.segs[NWk] = z;
   }
+  const long long nbh = (long long)p.B * p.Hkv;
   if (x >= z) return;
 
   uint32_t phase = 0;
   const int first_page = kBF16 ? 0 : int4_first_page(p.sink);
-  const long long nbh = (long long)p.B * p.Hkv;
   int b = 0;
   bool located = false;
   while (x < z) {
@@ -772,8 +962,12 @@ __global__ void __launch_bounds__(kWarps * 32, 4) decode_kernel(DecodeParams p) 
         const long long e = min(z, (long long)(r8 + 1) * np8);
         const int L = eff_len(p.seq_lens[r8 / p.Hkv], cap);
         float *slot = p.slots + ((long long)r8 + wid) * p.slot_floats;
-        ok = int8_piece<D, G>(p, r8 / p.Hkv, r8 % p.Hkv, L, j0, j0 + static_cast<int>(e - x), wsm, bars, phase,
-                              slot, lane);
+        if (lane == 0) {
+          if (j0 == 0) p.first[r8] = static_cast<int>(wid);
+          if (e == (long long)(r8 + 1) * np8) p.last[r8] = static_cast<int>(wid);
+        }
+        ok = int8_piece<D, G>(p, r8 / p.Hkv, r8 % p.Hkv, L, j0, j0 + static_cast<int>(e - x), wsm, bars, qsm,
+                              phase, slot, lane);
         x = e;
       }
     } else {
@@ -797,81 +991,15 @@ __global__ void __launch_bounds__(kWarps * 32, 4) decode_kernel(DecodeParams p) 
       float *slot = p.slots + (nbh + (long long)b * p.Hkv + h + wid) * p.slot_floats;
       const int pg0 = first_page + off;
       const int pg1 = pg0 + static_cast<int>(e - x);
+      if (lane == 0) {
+        if (off == 0) p.first[nbh + (long long)b * p.Hkv + h] = static_cast<int>(wid);
+        if (e == T8 + plan[b] + (long long)(h + 1) * per) p.last[nbh + (long long)b * p.Hkv + h] = static_cast<int>(wid);
+      }
       if constexpr (kBF16) ok = bf16_piece<D, G>(p, b, h, L, pg0, pg1, wsm, bars, phase, slot, lane);
-      else ok = int4_piece<D, G>(p, b, h, L, pg0, pg1, wsm, bars, phase, slot, lane);
+      else ok = int4_piece<D, G>(p, b, h, L, pg0, pg1, wsm, bars, qsm, phase, slot, lane);
       x = e;
     }
     if (!ok) return;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Exact merge of the partials of one (sequence, query head):
-// M = max m_c, W_c = l_c 2^(m_c - M), out = sum W_c o_c / sum W_c.
-// ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
-  constexpr int EPL = D / 32;
-  const long long task = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (task >= (long long)p.B * p.Hq) return;
-  const int b = static_cast<int>(task / p.Hq), hq = static_cast<int>(task % p.Hq);
-  const int h = hq / p.G, gq = hq % p.G;
-  const int r = b * p.Hkv + h;
-  const long long NW = p.num_workers;
-  const long long nbh = (long long)p.B * p.Hkv;
-  const long long T8 = nbh * np8;
-  float M = -INFINITY, den = 0.f, acc[EPL];
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
-  auto add = [&](const float *slot) {
-    const float l = slot[p.G + gq];
-    if (!(l > 0.f)) return;
-    const float m = slot[gq];
-    if (m > M) {
-      const float f = ex2(M - m);
-      den *= f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) acc[e] *= f;
-      M = m;
-    }
-    const float w = l * ex2(m - M);
-    den += w;
-    const float *o = slot + p.slot_o_off + gq * D + lane * EPL;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, o[e], acc[e]);
-  };
-  // items [start, end) of one range -> the partials of the workers that own them
-  auto add_range = [&](long long start, long long end, long long range) {
-    long long lo = 0, hi = NW - 1;   // largest w with segs[w] <= start
-    while (lo < hi) {
-      const long long mid = (lo + hi + 1) >> 1;
-      if (p.segs[mid] <= start) lo = mid;
-      else hi = mid - 1;
-    }
-    long long a = p.segs[lo];
-    for (long long w = lo; w < NW && a < end; ++w) {
-      const long long a1 = p.segs[w + 1];
-      if (a1 > a && a1 > start) add(p.slots + (range + w) * p.slot_floats);
-      a = a1;
-    }
-  };
-  if (np8 > 0) add_range((long long)r * np8, (long long)(r + 1) * np8, r);
-  const int per = (p.plan[b + 1] - p.plan[b]) / p.Hkv;
-  if (per > 0) {
-    const long long start = T8 + p.plan[b] + (long long)h * per;
-    add_range(start, start + per, nbh + r);
-  }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  const long long obase = ((long long)b * p.Hq + hq) * D + lane * EPL;
-  if (p.out_fp32) {
-    float *o = reinterpret_cast<float *>(p.out) + obase;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) o[e] = acc[e] * inv;
-  } else {
-    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out) + obase;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) o[e] = __float2bfloat16_rn(acc[e] * inv);
   }
 }
 
@@ -917,36 +1045,42 @@ cudaError_t decode_prepare(int D, int G, bool bf16, DecodeLaunch *out) {
 }
 
 template <int D, int G, bool kBF16>
-static void launch_main(const DecodeParams &p, cudaStream_t stream) {
-  decode_kernel<D, G, kBF16><<<p.num_workers / kWarps, kWarps * 32, decode_smem_bytes(D, kBF16, p.B), stream>>>(p);
+static cudaError_t launch_main(const DecodeParams &p, cudaStream_t stream) {
+  return launch_pdl(decode_kernel<D, G, kBF16>, dim3(p.num_workers / kWarps), dim3(kWarps * 32),
+                    decode_smem_bytes(D, kBF16, p.B), stream, p);
 }
 
 template <int D, bool kBF16>
-static void launch_main_d(const DecodeParams &p, cudaStream_t stream) {
+static cudaError_t launch_main_d(const DecodeParams &p, cudaStream_t stream) {
   switch (p.G) {
-    case 1: launch_main<D, 1, kBF16>(p, stream); break;
-    case 2: launch_main<D, 2, kBF16>(p, stream); break;
-    default: launch_main<D, 4, kBF16>(p, stream); break;
+    case 1: return launch_main<D, 1, kBF16>(p, stream);
+    case 2: return launch_main<D, 2, kBF16>(p, stream);
+    default: return launch_main<D, 4, kBF16>(p, stream);
+  }
+}
+
+template <int D>
+static cudaError_t launch_merge(const DecodeParams &p, int np8, cudaStream_t stream) {
+  const long long warps = (long long)p.B * p.Hkv;
+  if (warps == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>((warps + 3) / 4);
+  switch (p.G) {
+    case 1: return launch_pdl(merge_kernel<D, 1>, dim3(blocks), dim3(128), 0, stream, p, np8);
+    case 2: return launch_pdl(merge_kernel<D, 2>, dim3(blocks), dim3(128), 0, stream, p, np8);
+    default: return launch_pdl(merge_kernel<D, 4>, dim3(blocks), dim3(128), 0, stream, p, np8);
   }
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t stream, cudaEvent_t ev0,
                           cudaEvent_t ev1) {
   if (ev0) cudaEventRecord(ev0, stream);
-  if (D == 128) {
-    if (bf16) launch_main_d<128, true>(p, stream);
-    else launch_main_d<128, false>(p, stream);
-  } else {
-    if (bf16) launch_main_d<64, true>(p, stream);
-    else launch_main_d<64, false>(p, stream);
-  }
+  cudaError_t e;
+  if (D == 128) e = bf16 ? launch_main_d<128, true>(p, stream) : launch_main_d<128, false>(p, stream);
+  else e = bf16 ? launch_main_d<64, true>(p, stream) : launch_main_d<64, false>(p, stream);
+  if (e != cudaSuccess) return e;
   if (ev1) cudaEventRecord(ev1, stream);
-  const long long warps = (long long)p.B * p.Hq;
-  const unsigned blocks = static_cast<unsigned>((warps + 3) / 4);
-  const int np8 = (!bf16 && p.int8_units) ? (p.sink > 0 ? 1 : 0) + p.recent / 16 : 0;
-  if (D == 128) merge_kernel<128><<<blocks, 128, 0, stream>>>(p, np8);
-  else merge_kernel<64><<<blocks, 128, 0, stream>>>(p, np8);
-  return cudaGetLastError();
+  const int np8 = (!bf16 && p.int8_units) ? side_pages(p.sink, p.recent) : 0;
+  return D == 128 ? launch_merge<128>(p, np8, stream) : launch_merge<64>(p, np8, stream);
 }
 
 }  // namespace kv4

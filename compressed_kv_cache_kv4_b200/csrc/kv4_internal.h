@@ -34,6 +34,8 @@ struct DecodeParams {
   float scale_log2;             // softmax_scale * log2(e)
   int *plan;                    // [B+1] prefix of attended INT4/bf16 page-heads
   long long *segs;              // [num_workers+1] first item of each worker
+  int *first;                   // [2*B*Hkv] worker owning the first item of each range
+  int *last;                    // [2*B*Hkv] worker owning the last item of each range
   float *slots;                 // [2*B*Hkv + num_workers][slot_floats] partials
   void *out;
   int out_fp32;
@@ -57,6 +59,25 @@ struct DecodeLaunch {
   int smem_bytes;
   int blocks_per_sm;
 };
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous grid in the stream finishes; it calls pdl_wait() before
+// touching anything that grid produced.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream);
 cudaError_t decode_prepare(int D, int G, bool bf16, DecodeLaunch *out);

@@ -33,6 +33,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int us
   __shared__ int sh_digit, sh_rem;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NWARP = kTopkThreads / 32;
+  pdl_wait();
+  pdl_launch_dependents();
   const int row = blockIdx.x;
   const int b = row / p.Hkv;
   int L = p.seq_lens[b];
@@ -157,8 +159,7 @@ cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream) {
   const size_t smem = (use_smem ? (size_t)p.max_len * 4 : 0) + (size_t)((p.max_len + 31) / 32) * 4;
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  topk_kernel<<<rows, kTopkThreads, smem, stream>>>(p, use_smem);
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel, dim3(rows), dim3(kTopkThreads), smem, stream, p, use_smem);
 }
 
 }  // namespace kv4

@@ -84,7 +84,7 @@ def test_decode_tiny_end_to_end():
     assert c.cache.get_error()[0] == K.KV4_OK
 
 
-@pytest.mark.parametrize("D,Hq,Hkv", [(128, 32, 8), (64, 4, 2), (128, 8, 8), (64, 8, 4)])
+@pytest.mark.parametrize("D,Hq,Hkv", [(128, 32, 8), (64, 4, 2), (128, 8, 8), (64, 8, 4), (64, 4, 4), (128, 4, 2)])
 def test_decode_from_oracle_bytes(D, Hq, Hkv):
     """The decode kernel reading bytes written by the oracle's own layout writer."""
     wl = small_wl([1, 16, 17, 100, 144, 145, 160, 161, 700, 2049, 3001], Hq=Hq, Hkv=Hkv, D=D, seed=D + Hq)
