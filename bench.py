@@ -23,9 +23,11 @@ the max over ranks.
 bounded sample of the same workload (the reference arm of the comparison).
 """
 import argparse
+import hashlib
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -92,9 +94,15 @@ def sum_over_ranks(x, ws):
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def aggregate(positions, elapsed_ms, ws):
+    """Whole-job throughput: positions attended on all ranks / the slowest rank's time."""
+    elapsed_max = max_over_ranks(elapsed_ms, ws)
+    return sum_over_ranks(positions, ws) / (elapsed_max / 1e3), elapsed_max
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -157,6 +165,33 @@ def peaks():
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
     except Exception:
         return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+# ---------------------------------------------------------------------------- ncu traffic
+PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_qwen8b.md")
+KERNEL_SOURCES = ["kv4_decode.cu", "kv4_common.cuh", "kv4_internal.h"]
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "compressed_kv_cache_kv4_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def ncu_traffic(wbytes):
+    """DRAM bytes (read + write) of one decode_kernel launch, from the committed
+    ncu summary, scaled from the captured launch's algorithmic bytes to
+    `wbytes`. None if the summary is absent or the kernel sources have changed
+    since the capture."""
+    try:
+        vals = dict(re.findall(r"^- (\w+): (\S+)\s*$", open(PROFILE).read(), re.M))
+        if vals.get("kernel_sources_sha256") != kernel_source_hash():
+            return None
+        return int(round(float(vals["dram_bytes_per_launch"]) * wbytes /
+                         float(vals["algorithmic_bytes_of_captured_launch"])))
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 # ---------------------------------------------------------------------------- byte accounting
@@ -272,11 +307,9 @@ def run_kv4(args, ws, rank):
     st, bits = cache.get_error()
     assert st == K.KV4_OK, ("device error in timed region", st, bits)
 
-    elapsed_max = max_over_ranks(elapsed_ms, ws)
     cyc = [(args.warmup + s) % CYCLE for s in range(args.steps)]
     positions = float(sum(int(lens_pre.astype(np.int64).sum()) + wl.B * (c + 1) for c in cyc))
-    positions_all = sum_over_ranks(positions, ws)
-    value = positions_all / (elapsed_max / 1e3)
+    value, elapsed_max = aggregate(positions, elapsed_ms, ws)
     mean_lens = lens_pre.astype(np.int64) + CYCLE // 2
     wbytes = worker_bytes(mean_lens, wl)
     sbytes = step_bytes(mean_lens, wl)
@@ -290,10 +323,10 @@ def run_kv4(args, ws, rank):
         "step_gbs": sbytes / (elapsed_max / args.steps / 1e3) / 1e9,
         "worker_avg_us": worker_avg_ms * 1e3, "worker_launches": worker_n,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic(wbytes),
                      "kernel": "decode_kernel (split-K worker)", "algorithmic_bytes_per_launch": wbytes,
                      "peak_source": peak_src},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,   # per step: append, decode workers, merge
     }
 
     if rank == 0 and not args.no_secondary and args.workload == "qwen8b":
