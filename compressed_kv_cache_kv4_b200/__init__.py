@@ -59,6 +59,8 @@ def lib():
         "kv4_workspace_bytes": (C.c_int, [_P, _I32, _I32, _I32, C.POINTER(_SZ)]),
         "kv4_decode_attn": (C.c_int, [_P, _P, _P, _I32, _P, _P, _I32, _P, _I32, C.c_float, _I32, _P, _SZ,
                                       _P, _I32, _I32]),
+        "kv4_decode_attn_noalloc": (C.c_int, [_P, _P, _P, _I32, _P, _P, _I32, _P, _I32, C.c_float, _I32,
+                                              _P, _I32, _I32]),
         "kv_topk_retain": (C.c_int, [_P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P, _I32, _P, _I32]),
         "bf16_paged_workspace_bytes": (C.c_int, [_I32, _I32, _I32, _I32, _I32, C.POINTER(_SZ)]),
         "bf16_paged_decode_attn": (C.c_int, [_P, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _P, C.c_float,
@@ -143,6 +145,29 @@ def kv4_decode_attn(handle, q, seq_lens, page_table, softmax_scale, workspace, o
                                num_workers, _ptr(workspace), workspace.numel() * workspace.element_size(),
                                _ptr(out), 1 if out.dtype == torch.float32 else 0, B)
     _check(st, "kv4_decode_attn")
+
+
+# Size of the fixed per-device scratch of kv4_decode_attn_noalloc (KV4_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def kv4_decode_attn_noalloc(handle, q, seq_lens, page_table, softmax_scale, out, retain_mask=None,
+                            num_workers=0, stream=None):
+    """kv4_decode_attn with the library's fixed scratch instead of a caller
+    workspace (for callers that cannot allocate device memory). Calls whose
+    kernels may overlap in time on one device must not be issued: they share
+    the scratch."""
+    B, Hq, _ = q.shape
+    mstride = 0 if retain_mask is None else retain_mask.shape[-1]
+    st = lib().kv4_decode_attn_noalloc(handle, _stream(stream), _ptr(q), Hq, _ptr(seq_lens), _ptr(page_table),
+                                       page_table.shape[1], _ptr(retain_mask), mstride, C.c_float(softmax_scale),
+                                       num_workers, _ptr(out), 1 if out.dtype == torch.float32 else 0, B)
+    if st == KV4_ERR_CAPACITY:
+        need = kv4_workspace_bytes(handle, B, Hq, num_workers)
+        if need > NOALLOC_SCRATCH_BYTES:
+            raise Kv4Error(st, "kv4_decode_attn_noalloc: needs %d bytes of scratch, the fixed area holds %d"
+                           % (need, NOALLOC_SCRATCH_BYTES))
+    _check(st, "kv4_decode_attn_noalloc")
 
 
 def kv_topk_retain(scores, seq_lens, budget_permille, mask_out, count_out=None, sink=16, recent=128,

@@ -195,7 +195,39 @@ kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32
                                   int32_t out_is_fp32, int32_t B, uint32_t *error_word);
 
 /*
- * kv4_get_error -- synchronise `stream`, then read and clear the cache's device
+ * kv4_decode_attn_noalloc -- kv4_decode_attn without a caller workspace. The
+ * pages describe no such call: it serves callers that cannot allocate device
+ * memory for the library, e.g. C code with no access to the application's
+ * device allocator, or a serving loop that must not call cudaMalloc/cudaFree
+ * (which may synchronise the device) between decode steps.
+ *  Scratch: a fixed array of KV4_NOALLOC_SCRATCH_BYTES (16 MiB) per device,
+ *    part of the library's loaded module; no call allocates or frees memory.
+ *    Nothing in it has to start at zero (the kernels write each word before
+ *    reading it).
+ *  Limit: returns KV4_ERR_CAPACITY, with nothing enqueued, when
+ *    kv4_workspace_bytes() for the same (B, Hq, num_workers) exceeds
+ *    KV4_NOALLOC_SCRATCH_BYTES (with Hkv = 8, head_dim = 128, Hq = 32 and the
+ *    default workers on a 148-SM B200: up to about 340 sequences). A smaller
+ *    num_workers lowers the need.
+ *  Set-up: the first call on each device looks up the array's address (this
+ *    makes the CUDA runtime load the library's module on that device); make
+ *    that first call before capturing the stream into a graph. Later calls on
+ *    the device reuse the cached address.
+ *  Concurrency: all calls on one device share the one array. Two calls whose
+ *    kernels may overlap in time (different streams without ordering between
+ *    them, or host threads racing on streams) corrupt each other's partials;
+ *    order them on one stream or with events.
+ * Other arguments, the outputs and the error behaviour are those of
+ * kv4_decode_attn (q, out 16-byte aligned; the cache's device error word).
+ */
+#define KV4_NOALLOC_SCRATCH_BYTES (16u << 20)
+kv4_status kv4_decode_attn_noalloc(kv4_cache *cache, void *stream, const void *q, int32_t Hq,
+                                   const int32_t *seq_lens, const int32_t *page_table, int32_t pt_stride,
+                                   const uint32_t *retain_mask, int32_t mask_stride, float softmax_scale,
+                                   int32_t num_workers, void *out, int32_t out_is_fp32, int32_t B);
+
+/*
+ * kv4_get_error --synchronise `stream`, then read and clear the cache's device
  * error word. Returns KV4_OK if no device error was recorded, else the most
  * severe recorded status (TIMEOUT > BOUNDS > CAPACITY > RANGE). *bits (optional)
  * receives the raw word: bit (1 << status) per recorded status.
