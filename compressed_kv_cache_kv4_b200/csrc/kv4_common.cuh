@@ -205,4 +205,22 @@ __device__ __forceinline__ int int4_num_pages(int L, int sink, int recent) {
   return (hi + kPageTokens - 1) / kPageTokens - sink / kPageTokens;
 }
 
+// ---------------------------------------------------------------- split of the decode work
+// Weights of one item when splitting work among workers: an INT4 page-head
+// (18*D bytes) counts 4, an INT8 side page (32*D + 64 bytes) counts 7.
+constexpr long long kW4 = 4, kW8 = 7;
+
+// First item of worker w among nw: items 0..T8-1 are INT8 pages (weight kW8),
+// then T4 INT4/bf16 pages (weight kW4); worker w starts at the first item whose
+// weighted start is >= floor(w * total / nw).
+__device__ __forceinline__ long long worker_first_item(long long w, long long nw, long long T8, long long T4) {
+  if (w >= nw) return T8 + T4;
+  const long long total = kW8 * T8 + kW4 * T4;
+  const long long a = w * total / nw;
+  if (a <= kW8 * T8) return (a + kW8 - 1) / kW8;
+  return T8 + (a - kW8 * T8 + kW4 - 1) / kW4;
+}
+
+__host__ __device__ __forceinline__ int side_pages(int sink, int recent) { return (sink > 0 ? 1 : 0) + recent / 16; }
+
 }  // namespace kv4

@@ -19,8 +19,8 @@
 //                  bf16 in registers), fp16 tiles for INT8 pages (int8 codes are
 //                  exact in fp16). Each worker writes one (m, l, o) partial per
 //                  (region, sequence, KV head) piece of its segment.
-//   merge_kernel   one warp per (sequence, KV head) merges the partials of all
-//                  its query heads exactly.
+//   merge_kernel   (kv4_merge.cu) one warp per (sequence, query head) merges
+//                  its partials exactly.
 //
 // Softmax bookkeeping runs in the log2 domain (scores scaled by tau*log2 e).
 // P.V takes P*scale_V as two 16-bit terms (hi + lo), which carries 16 (bf16)
@@ -53,24 +53,6 @@ struct Cfg {
   static constexpr int RINGS = kWarps * (WARP_SMEM + NS * 8 + QBYTES);
 };
 
-// Weights of one item when splitting work among workers: an INT4 page-head
-// (18*D bytes) counts 4, an INT8 side page (32*D + 64 bytes) counts 7.
-constexpr long long kW4 = 4, kW8 = 7;
-
-// (sequence, KV head) merges a worker postpones to the end of its segment.
-
-// First item of worker w among nw: items 0..T8-1 are INT8 pages (weight kW8),
-// then T4 INT4/bf16 pages (weight kW4); worker w starts at the first item whose
-// weighted start is >= floor(w * total / nw).
-__device__ __forceinline__ long long worker_first_item(long long w, long long nw, long long T8, long long T4) {
-  if (w >= nw) return T8 + T4;
-  const long long total = kW8 * T8 + kW4 * T4;
-  const long long a = w * total / nw;
-  if (a <= kW8 * T8) return (a + kW8 - 1) / kW8;
-  return T8 + (a - kW8 * T8 + kW4 - 1) / kW4;
-}
-
-__host__ __device__ __forceinline__ int side_pages(int sink, int recent) { return (sink > 0 ? 1 : 0) + recent / 16; }
 
 // ---------------------------------------------------------------------------
 // Partial slot: m[G] | l[G] | pad | o[G][D]   (m in log2 units, o normalised)
@@ -745,139 +727,6 @@ __device__ bool bf16_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
 }
 
 // ---------------------------------------------------------------------------
-// The exact merge of one (sequence, KV head).
-// ---------------------------------------------------------------------------
-
-// out[b][h*G + g] for every query head g: M = max m_c, W_c = l_c 2^(m_c - M),
-// out = sum W_c o_c / sum W_c over the partials of (b, h) (0 if none). The
-// partials of a range sit in slots range + w for the contiguous workers
-// w = first[range] .. last[range]. Loads in three rounds: the range bounds,
-// every partial's (m, l) (lane k: partial k), then the output vectors (lane:
-// query head lane / (32/G), D*G/32 consecutive elements). All reads bypass L1:
-// the partials were written by other SMs.
-template <int D, int G>
-__device__ void merge_bh(const DecodeParams &p, int b, int h, int np8, int per, long long T8, long long T4,
-                         int lane) {
-  constexpr int LPH = 32 / G, DPL = D / LPH;
-  const int gq = lane / LPH, d0 = (lane % LPH) * DPL;
-  const long long nbh = (long long)p.B * p.Hkv;
-  const long long r = (long long)b * p.Hkv + h;
-  const long long f8 = np8 > 0 ? __ldcg(&p.first[r]) : 0, l8 = np8 > 0 ? __ldcg(&p.last[r]) : -1;
-  const long long f4 = per > 0 ? __ldcg(&p.first[nbh + r]) : 0, l4 = per > 0 ? __ldcg(&p.last[nbh + r]) : -1;
-  const int n8 = static_cast<int>(l8 - f8 + 1), n = n8 + static_cast<int>(l4 - f4 + 1);
-  float M = -INFINITY, den = 0.f, acc[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  for (int c0 = 0; c0 < n; c0 += 32) {
-    const int k = c0 + lane;
-    long long slot_idx = -1, w = -1;
-    if (k < n8) {
-      w = f8 + k;
-      slot_idx = r + w;
-    } else if (k < n) {
-      w = f4 + (k - n8);
-      slot_idx = nbh + r + w;
-    }
-    // a worker with an empty segment wrote no partial
-    if (w >= 0 && worker_first_item(w, p.num_workers, T8, T4) == worker_first_item(w + 1, p.num_workers, T8, T4))
-      slot_idx = -1;
-    // lane k: (m, l) of partial k for all heads
-    float mk[G], lk[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      mk[g] = -INFINITY;
-      lk[g] = 0.f;
-    }
-    if (slot_idx >= 0) {
-      const float *slot = p.slots + slot_idx * p.slot_floats;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        lk[g] = __ldcg(slot + G + g);
-        mk[g] = __ldcg(slot + g);
-      }
-    }
-    // every lane needs, for its head gq, the (m, l) of each partial kk: read
-    // them from lane kk with shuffles; first the head max, then the weights
-    float mc = -INFINITY;
-    const uint32_t pmask = __ballot_sync(0xffffffffu, slot_idx >= 0);
-    uint32_t rem = pmask;
-    while (rem) {
-      const int kk = __ffs(rem) - 1;
-      rem &= rem - 1;
-      float mg = -INFINITY, lg = 0.f;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float mv = __shfl_sync(0xffffffffu, mk[g], kk);
-        const float lv = __shfl_sync(0xffffffffu, lk[g], kk);
-        if (g == gq) {
-          mg = mv;
-          lg = lv;
-        }
-      }
-      if (lg > 0.f) mc = fmaxf(mc, mg);
-    }
-    if (mc > M) {
-      const float f = ex2(M - mc);
-      den *= f;
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] *= f;
-      M = mc;
-    }
-    rem = pmask;
-    while (rem) {
-      const int kk = __ffs(rem) - 1;
-      rem &= rem - 1;
-      float mg = -INFINITY, lg = 0.f;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float mv = __shfl_sync(0xffffffffu, mk[g], kk);
-        const float lv = __shfl_sync(0xffffffffu, lk[g], kk);
-        if (g == gq) {
-          mg = mv;
-          lg = lv;
-        }
-      }
-      const long long si = __shfl_sync(0xffffffffu, slot_idx, kk);
-      if (!(lg > 0.f)) continue;
-      const float wk = lg * ex2(mg - M);
-      den += wk;
-      const float2 *o = reinterpret_cast<const float2 *>(p.slots + si * p.slot_floats + p.slot_o_off + gq * D + d0);
-#pragma unroll
-      for (int e = 0; e < DPL / 2; ++e) {
-        const float2 v = __ldcg(o + e);
-        acc[2 * e + 0] = fmaf(wk, v.x, acc[2 * e + 0]);
-        acc[2 * e + 1] = fmaf(wk, v.y, acc[2 * e + 1]);
-      }
-    }
-  }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-  const long long obase = ((long long)b * p.Hq + (long long)h * G + gq) * D + d0;
-  if (p.out_fp32) {
-    float2 *o = reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + obase);
-#pragma unroll
-    for (int e = 0; e < DPL / 2; ++e) o[e] = make_float2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-  } else {
-    uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + obase);
-#pragma unroll
-    for (int e = 0; e < DPL / 2; ++e) o[e] = pack_bf16x2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-  }
-}
-
-// One warp per (sequence, KV head), after the worker grid has finished.
-template <int D, int G>
-__global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
-  const long long task = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  pdl_wait();
-  pdl_launch_dependents();
-  if (task >= (long long)p.B * p.Hkv) return;
-  const int b = static_cast<int>(task / p.Hkv), h = static_cast<int>(task % p.Hkv);
-  const int per = (__ldcg(&p.plan[b + 1]) - __ldcg(&p.plan[b])) / p.Hkv;
-  const long long T8 = (long long)p.B * p.Hkv * np8, T4 = __ldcg(&p.plan[p.B]);
-  merge_bh<D, G>(p, b, h, np8, per, T8, T4, lane);
-}
-
-// ---------------------------------------------------------------------------
 // Persistent worker kernel.
 // ---------------------------------------------------------------------------
 template <int D, int G, bool kBF16>
@@ -1059,18 +908,6 @@ static cudaError_t launch_main_d(const DecodeParams &p, cudaStream_t stream) {
   }
 }
 
-template <int D>
-static cudaError_t launch_merge(const DecodeParams &p, int np8, cudaStream_t stream) {
-  const long long warps = (long long)p.B * p.Hkv;
-  if (warps == 0) return cudaSuccess;
-  const unsigned blocks = static_cast<unsigned>((warps + 3) / 4);
-  switch (p.G) {
-    case 1: return launch_pdl(merge_kernel<D, 1>, dim3(blocks), dim3(128), 0, stream, p, np8);
-    case 2: return launch_pdl(merge_kernel<D, 2>, dim3(blocks), dim3(128), 0, stream, p, np8);
-    default: return launch_pdl(merge_kernel<D, 4>, dim3(blocks), dim3(128), 0, stream, p, np8);
-  }
-}
-
 cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t stream, cudaEvent_t ev0,
                           cudaEvent_t ev1) {
   if (ev0) cudaEventRecord(ev0, stream);
@@ -1080,7 +917,7 @@ cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t 
   if (e != cudaSuccess) return e;
   if (ev1) cudaEventRecord(ev1, stream);
   const int np8 = (!bf16 && p.int8_units) ? side_pages(p.sink, p.recent) : 0;
-  return D == 128 ? launch_merge<128>(p, np8, stream) : launch_merge<64>(p, np8, stream);
+  return launch_merge(p, D, np8, stream);
 }
 
 }  // namespace kv4

@@ -85,5 +85,7 @@ int decode_smem_bytes(int D, bool bf16, int B);
 cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t stream, cudaEvent_t ev0,
                           cudaEvent_t ev1);
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream);
+// Exact merge of the decode partials (np8 = INT8 side pages per (sequence, head)).
+cudaError_t launch_merge(const DecodeParams &p, int D, int np8, cudaStream_t stream);
 
 }  // namespace kv4

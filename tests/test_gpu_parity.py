@@ -98,7 +98,7 @@ def test_decode_from_oracle_bytes(D, Hq, Hkv):
 
 @pytest.mark.parametrize("workers", [4, 8, 12, 60, 0, 4000])
 def test_worker_count_invariance(workers):
-    wl = small_wl([3000, 2, 500, 145, 4100, 900, 1600, 33], seed=11)
+    wl = small_wl([3000, 2, 0, 500, 145, 4100, 900, 1600, 33], seed=11)
     c = Case(wl)
     c.make_cache()
     c.append_all()
@@ -146,7 +146,7 @@ def test_protected_positions_ignore_int4_codes():
 
 
 def test_pure_kv4_mode():
-    wl = small_wl([1, 300, 1700], seed=15, sink=0, recent=0)
+    wl = small_wl([1, 0, 300, 1700], seed=15, sink=0, recent=0)
     c = Case(wl)
     c.make_cache()
     c.append_all()
