@@ -82,30 +82,36 @@ struct SoftmaxState {
 template <int NMT, int kSlack>
 __device__ __forceinline__ void softmax_update(SoftmaxState<NMT> &st, const float (&s)[4], float (&pr)[4]) {
   float mx0 = fmaxf(s[0], s[2]), mx1 = fmaxf(s[1], s[3]);
+  // The page's column max exceeds the reference exactly when some lane's own
+  // max does, so the warp-wide max (three shuffle rounds) is only formed on
+  // pages that move the reference.
+  const bool up = mx0 > st.m[0] + static_cast<float>(kSlack) || mx1 > st.m[1] + static_cast<float>(kSlack);
+  if (__any_sync(0xffffffffu, up)) {
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-  }
-  if (mx0 > st.m[0] + static_cast<float>(kSlack)) {
-    const float f = ex2(st.m[0] - mx0);
-    st.l[0] *= f;
-#pragma unroll
-    for (int mt = 0; mt < NMT; ++mt) {
-      st.o[mt][0] *= f;
-      st.o[mt][2] *= f;
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
-    st.m[0] = mx0;
-  }
-  if (mx1 > st.m[1] + static_cast<float>(kSlack)) {
-    const float f = ex2(st.m[1] - mx1);
-    st.l[1] *= f;
+    if (mx0 > st.m[0] + static_cast<float>(kSlack)) {
+      const float f = ex2(st.m[0] - mx0);
+      st.l[0] *= f;
 #pragma unroll
-    for (int mt = 0; mt < NMT; ++mt) {
-      st.o[mt][1] *= f;
-      st.o[mt][3] *= f;
+      for (int mt = 0; mt < NMT; ++mt) {
+        st.o[mt][0] *= f;
+        st.o[mt][2] *= f;
+      }
+      st.m[0] = mx0;
     }
-    st.m[1] = mx1;
+    if (mx1 > st.m[1] + static_cast<float>(kSlack)) {
+      const float f = ex2(st.m[1] - mx1);
+      st.l[1] *= f;
+#pragma unroll
+      for (int mt = 0; mt < NMT; ++mt) {
+        st.o[mt][1] *= f;
+        st.o[mt][3] *= f;
+      }
+      st.m[1] = mx1;
+    }
   }
   const float2 r = make_float2(st.m[0] == -INFINITY ? 0.f : st.m[0], st.m[1] == -INFINITY ? 0.f : st.m[1]);
   const float2 d01 = __fadd2_rn(make_float2(s[0], s[1]), make_float2(-r.x, -r.y));
