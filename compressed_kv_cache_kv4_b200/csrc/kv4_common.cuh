@@ -137,6 +137,26 @@ __device__ __forceinline__ uint32_t i4x2_biased(uint32_t w) {
   return t;
 }
 
+// Two signed 4-bit codes at bits 0-3 and 16-19 of w -> fp16x2 of the codes.
+// LOP3 computes (w & 0x000F000F) ^ 0x64086408: flipping bit 3 turns c into
+// c + 8 under fp16's 1024, giving 1032 + c; subtracting 1032 is exact.
+__device__ __forceinline__ uint32_t i4x2_lo_to_f16x2(uint32_t w) {
+  uint32_t t, d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x000F000Fu), "r"(0x64086408u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(t), "r"(0x64086408u));
+  return d;
+}
+
+// Two signed 4-bit codes at bits 4-7 and 20-23 of w -> fp16x2, with no shift:
+// fp16 has ten mantissa bits, so under an exponent of 64 (0x5400) the field
+// at bits 4-7 has weight 1. (w & 0x00F000F0) ^ 0x54805480 is 72 + c.
+__device__ __forceinline__ uint32_t i4x2_hi_to_f16x2(uint32_t w) {
+  uint32_t t, d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x00F000F0u), "r"(0x54805480u));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(t), "r"(0x54805480u));
+  return d;
+}
+
 // Two signed 8-bit codes at bits 0-7 and 16-23 of w -> fp16x2 of the codes.
 // LOP3 computes (w & 0x00FF00FF) ^ 0x64806480: flipping bit 7 turns c into
 // c + 128, and 0x64 above it makes the fp16 value 1024 + (c + 128).

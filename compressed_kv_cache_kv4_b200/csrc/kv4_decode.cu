@@ -139,6 +139,16 @@ __device__ __forceinline__ void weights_bf16(float2 w01, float2 w23, float2 neg_
   b1 = movmatrix_t(pack_bf16x2(r23.x, r23.y));
 }
 
+// fp16 variant of weights_bf16 (hi + lo carry 22 significant bits).
+__device__ __forceinline__ void weights_f16x2(float2 w01, float2 w23, float2 neg_sel, uint32_t &b0, uint32_t &b1) {
+  const uint32_t h01 = pack_f16x2(w01.x, w01.y);
+  const uint32_t h23 = pack_f16x2(w23.x, w23.y);
+  const float2 r01 = __ffma2_rn(neg_sel, f16x2_to_f32x2(h01), w01);
+  const float2 r23 = __ffma2_rn(neg_sel, f16x2_to_f32x2(h23), w23);
+  b0 = movmatrix_t(pack_f16x2(r01.x, r01.y));
+  b1 = movmatrix_t(pack_f16x2(r23.x, r23.y));
+}
+
 __device__ __forceinline__ void weights_f16(float w0, float w1, float w2, float w3, float lo_sel, uint32_t &b0,
                                             uint32_t &b1) {
   uint32_t h01 = pack_f16x2(w0, w1);
@@ -433,16 +443,17 @@ __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
       if (!v0) sl[0] = sl[1] = -INFINITY;
       if (!v1) sl[2] = sl[3] = -INFINITY;
     }
+    // exact running max: probabilities <= 1, so P * scale_V fits fp16
     float pr[4];
-    softmax_update<NMT, 8>(st, sl, pr);
+    softmax_update<NMT, 0>(st, sl, pr);
 
     // ---- P.V
     uint32_t wb[NG][2];
 #pragma unroll
     for (int i = 0; i < NG; ++i) {
       const float vs0 = vs0a[i], vs1 = vs1a[i];
-      weights_bf16(__fmul2_rn(make_float2(pr[0], pr[1]), make_float2(vs0, vs0)),
-                   __fmul2_rn(make_float2(pr[2], pr[3]), make_float2(vs1, vs1)), neg_sel, wb[i][0], wb[i][1]);
+      weights_f16x2(__fmul2_rn(make_float2(pr[0], pr[1]), make_float2(vs0, vs0)),
+                    __fmul2_rn(make_float2(pr[2], pr[3]), make_float2(vs1, vs1)), neg_sel, wb[i][0], wb[i][1]);
     }
     uint32_t vw[NMT];
 #pragma unroll
@@ -455,9 +466,10 @@ __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
     }
 #pragma unroll
     for (int mt = 0; mt < NMT; ++mt) {
-      const uint32_t a[4] = {i4x2_to_bf16x2(vw[mt]), i4x2_to_bf16x2(vw[mt] >> 4), i4x2_to_bf16x2(vw[mt] >> 8),
-                             i4x2_to_bf16x2(vw[mt] >> 12)};
-      mma_bf16(st.o[mt], a, wb[mt >> 1][0], wb[mt >> 1][1]);
+      const uint32_t v8 = vw[mt] >> 8;
+      const uint32_t a[4] = {i4x2_lo_to_f16x2(vw[mt]), i4x2_hi_to_f16x2(vw[mt]), i4x2_lo_to_f16x2(v8),
+                             i4x2_hi_to_f16x2(v8)};
+      mma_f16(st.o[mt], a, wb[mt >> 1][0], wb[mt >> 1][1]);
     }
 
     // ---- refill this stage
