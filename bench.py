@@ -173,9 +173,13 @@ KERNEL_SOURCES = ["kv4_decode.cu", "kv4_common.cuh", "kv4_internal.h"]
 
 
 def kernel_source_hash():
+    """sha256 of the decode kernel's sources with comments and whitespace removed."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, "compressed_kv_cache_kv4_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "compressed_kv_cache_kv4_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()
 
 

@@ -15,16 +15,18 @@
 //                  shared-memory stages filled by 1-D bulk copies (TMA engine,
 //                  mbarrier completion, bounded waits). Per page, q.K and P.V
 //                  are small tensor-core tiles (mma.sync m16n8k16, fp32
-//                  accumulate): bf16 tiles for INT4 pages (codes unpacked to
-//                  bf16 in registers), fp16 tiles for INT8 pages (int8 codes are
-//                  exact in fp16). Each worker writes one (m, l, o) partial per
+//                  accumulate): q.K of INT4 pages on bf16 tiles (codes
+//                  unpacked in registers), P.V of INT4 pages and all of the
+//                  INT8 pages on fp16 tiles (the codes are exact in fp16).
+//                  Each worker writes one (m, l, o) partial per
 //                  (region, sequence, KV head) piece of its segment.
 //   merge_kernel   (kv4_merge.cu) one warp per (sequence, query head) merges
 //                  its partials exactly.
 //
 // Softmax bookkeeping runs in the log2 domain (scores scaled by tau*log2 e).
-// P.V takes P*scale_V as two 16-bit terms (hi + lo), which carries 16 (bf16)
-// or 22 (fp16) significant bits into fp32 accumulation.
+// P.V takes P*scale_V as two fp16 terms (hi + lo), which carries 22
+// significant bits into fp32 accumulation; the running max is exact (P <= 1),
+// so P*scale_V stays in the fp16 range.
 #include <math.h>
 
 #include "kv4_common.cuh"
