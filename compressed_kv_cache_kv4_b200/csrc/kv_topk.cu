@@ -10,9 +10,11 @@
 // larger key, -0 folded into +0). A 4-pass 8-bit radix select finds the key T
 // of the k-th best non-forced position in O(L) work; positions with key > T
 // are kept, and among keys == T the lowest indices fill the remainder (a scan
-// over 32-position tiles gives each tie its rank in index order). The row is
-// held in shared memory when it fits, otherwise re-read from global memory on
-// each pass.
+// over 32-position tiles gives each tie its rank in index order). The forced
+// positions are two contiguous ranges, so the passes run over the candidate
+// range between them only, four keys per thread step. The row is held in
+// shared memory when it fits, otherwise re-read from global memory on each
+// pass.
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
 
@@ -27,7 +29,33 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int use_smem) {
+// Keys of candidate positions [c0, c1) in steps of four per thread: f(i, key)
+// for each. With the row in shared memory four keys come from one 16-byte load
+// (c0 rounded down to a multiple of four; lanes skip the indices outside).
+template <bool kSmem, typename F>
+__device__ __forceinline__ void for_candidates(const uint32_t *keys, const float *srow, int c0, int c1, int tid,
+                                               F &&f) {
+  const int base = c0 & ~3;
+  for (int i = base + 4 * tid; i < c1; i += 4 * kTopkThreads) {
+    uint32_t k[4];
+    if constexpr (kSmem) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(keys + i);
+      k[0] = v.x;
+      k[1] = v.y;
+      k[2] = v.z;
+      k[3] = v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) k[e] = i + e < c1 ? score_key(srow[i + e]) : 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (i + e >= c0 && i + e < c1) f(i + e, k[e]);
+  }
+}
+
+template <bool kSmem>
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
   extern __shared__ __align__(16) uint32_t dyn[];
   __shared__ uint32_t hist[256];
   __shared__ int sh_digit, sh_rem;
@@ -42,24 +70,28 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int us
   const float *srow = p.scores + (long long)row * p.score_stride;
   const int S = p.sink, R = p.recent;
   const int nt = (L + 31) / 32;
-  uint32_t *keys = dyn;                                   // [max_len] when use_smem
-  int *tile_rank = reinterpret_cast<int *>(dyn + (use_smem ? p.max_len : 0));   // [nt]
+  // keys [round_up(max_len, 4)] when staged, then the tile ranks [nt]
+  uint32_t *keys = dyn;
+  int *tile_rank = reinterpret_cast<int *>(dyn + (kSmem ? (p.max_len + 3) / 4 * 4 : 0));
 
-  auto forced = [&](int pos) { return pos < S || pos >= L - R; };
-  auto key_at = [&](int pos) { return use_smem ? keys[pos] : score_key(srow[pos]); };
-
-  const int nF = L <= S ? L : S + min(R, L - S);
+  // forced positions are [0, min(S, L)) and [max(S, L - R), L); the candidates
+  // are the positions between them
+  const int c0 = min(S, L), c1 = max(c0, L - R);
+  auto forced = [&](int pos) { return pos < c0 || pos >= c1; };
+  const int nF = L - (c1 - c0);
   const long long kb = (long long)L * p.permille / 1000;
   long long ksel = kb - nF;
   if (ksel < 0) ksel = 0;
-  if (ksel > L - nF) ksel = L - nF;
-
-  if (use_smem)
-    for (int i = tid; i < L; i += kTopkThreads) keys[i] = score_key(srow[i]);
-  __syncthreads();
+  if (ksel > c1 - c0) ksel = c1 - c0;
 
   // mode: 0 = select none, 1 = select all, 2 = threshold
-  int mode = ksel == 0 ? 0 : (ksel == L - nF ? 1 : 2);
+  const int mode = ksel == 0 ? 0 : (ksel == c1 - c0 ? 1 : 2);
+  if (kSmem && mode == 2) {
+    const int base = c0 & ~3;
+    for (int i = base + tid; i < c1; i += kTopkThreads) keys[i] = score_key(srow[i]);
+  }
+  __syncthreads();
+
   uint32_t T = 0;
   int need_eq = 0;
   if (mode == 2) {
@@ -68,11 +100,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int us
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
       __syncthreads();
-      for (int i = tid; i < L; i += kTopkThreads) {
-        if (forced(i)) continue;
-        const uint32_t k = key_at(i);
+      for_candidates<kSmem>(keys, srow, c0, c1, tid, [&](int, uint32_t k) {
         if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
-      }
+      });
       __syncthreads();
       if (warp == 0) {
         // lane l owns bins 255-8l .. 248-8l (descending)
@@ -108,7 +138,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int us
     // ranks of the ties in index order: count per 32-position tile, then scan
     for (int w = warp; w < nt; w += NWARP) {
       const int pos = 32 * w + lane;
-      const bool eq = pos < L && !forced(pos) && key_at(pos) == T;
+      const bool eq = pos >= c0 && pos < c1 && (kSmem ? keys[pos] : score_key(srow[pos])) == T;
       const uint32_t bal = __ballot_sync(0xffffffffu, eq);
       if (lane == 0) tile_rank[w] = __popc(bal);
     }
@@ -139,7 +169,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int us
       if (forced(pos) || mode == 1) {
         sel = true;
       } else if (mode == 2) {
-        const uint32_t k = key_at(pos);
+        const uint32_t k = kSmem ? keys[pos] : score_key(srow[pos]);
         sel = k > T;
         eq = k == T;
       }
@@ -155,11 +185,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int us
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream) {
   const int rows = p.B * p.Hkv;
   if (rows == 0) return cudaSuccess;
-  const int use_smem = p.max_len <= kTopkSmemKeys ? 1 : 0;
-  const size_t smem = (use_smem ? (size_t)p.max_len * 4 : 0) + (size_t)((p.max_len + 31) / 32) * 4;
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool use_smem = p.max_len <= kTopkSmemKeys;
+  const size_t smem = (use_smem ? (size_t)(p.max_len + 3) / 4 * 16 : 0) + (size_t)((p.max_len + 31) / 32) * 4;
+  auto kern = use_smem ? topk_kernel<true> : topk_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(topk_kernel, dim3(rows), dim3(kTopkThreads), smem, stream, p, use_smem);
+  return launch_pdl(kern, dim3(rows), dim3(kTopkThreads), smem, stream, p);
 }
 
 }  // namespace kv4
