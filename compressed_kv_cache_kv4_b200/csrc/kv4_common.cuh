@@ -157,6 +157,14 @@ __device__ __forceinline__ uint32_t i4x2_hi_to_f16x2(uint32_t w) {
   return d;
 }
 
+// The same LOP3 as i4x2_hi_to_f16x2 without the subtraction: fp16x2 of 72 + c
+// for the codes at bits 4-7 and 20-23 (the offset is removed elsewhere).
+__device__ __forceinline__ uint32_t i4x2_hi_biased_f16(uint32_t w) {
+  uint32_t t;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x00F000F0u), "r"(0x54805480u));
+  return t;
+}
+
 // Two signed 8-bit codes at bits 0-7 and 16-23 of w -> fp16x2 of the codes.
 // LOP3 computes (w & 0x00FF00FF) ^ 0x64806480: flipping bit 7 turns c into
 // c + 128, and 0x64 above it makes the fp16 value 1024 + (c + 128).

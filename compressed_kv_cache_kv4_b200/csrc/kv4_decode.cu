@@ -297,11 +297,12 @@ __device__ __forceinline__ int next_page(PageCursor &c, int &pid, const int32_t 
 // INT4 pages of one piece (sequence b, KV head h, pages [pg0, pg1)).
 // Returns false if a bounded wait ran out (the worker must stop).
 //
-// q.K: A = K codes (rows = slots g, g+8), B = q. The MMA of (group i, half j)
-// covers elements 32i+8t+{2j, 2j+4} (k-slots 2t, 2t+1) and 32i+8t+{2j+1, 2j+5}
-// (k-slots 2t+8, 2t+9) -- the nibble order of the K words. The codes enter the
-// MMA as 136 + c (one LOP3); the accumulator starts at -136 * sum(q over the
-// group), which removes the offset.
+// q.K: A = K codes (rows = slots g, g+8), B = q. Per group two MMAs: a bf16
+// one over elements 32i+8t+{0, 4} (k-slots 2t, 2t+1) and {2, 6} (2t+8, 2t+9),
+// whose codes enter as 136 + c, and an fp16 one over {1, 5} and {3, 7}, whose
+// codes enter as 72 + c -- the nibble order of the K words; one shift by 8
+// serves both. The accumulator starts at -(136 * sum of q over the even
+// elements + 72 * sum over the odd ones), which removes the offsets.
 // P.V: A = V^T codes (rows = head_dim, k = slots), B = P * scale_V (hi + lo).
 // ---------------------------------------------------------------------------
 template <int D, int G>
@@ -322,18 +323,21 @@ __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
     for (int i = 0; i < NG; ++i) {
       const uint4 e = hv ? qh[4 * i + t] : make_uint4(0, 0, 0, 0);
       // e.x = (e0, e1), e.y = (e2, e3), e.z = (e4, e5), e.w = (e6, e7)
+      // e.x = (e0, e1), e.y = (e2, e3), e.z = (e4, e5), e.w = (e6, e7). Codes of
+      // even elements enter a bf16 MMA as 136 + c, codes of odd elements an
+      // fp16 MMA as 72 + c (see the q.K below), so the bf16 pairs (e0, e4),
+      // (e2, e6) and the fp16 pairs (e1, e5), (e3, e7) are stored.
+      const float e0 = bf16lo_to_f32(e.x), e1 = bf16hi_to_f32(e.x), e2 = bf16lo_to_f32(e.y), e3 = bf16hi_to_f32(e.y);
+      const float e4 = bf16lo_to_f32(e.z), e5 = bf16hi_to_f32(e.z), e6 = bf16lo_to_f32(e.w), e7 = bf16hi_to_f32(e.w);
       *reinterpret_cast<uint4 *>(qsm + i * 512 + lane * 16) =
-          make_uint4(__byte_perm(e.x, e.z, 0x5410),    // (e0, e4)
-                     __byte_perm(e.x, e.z, 0x7632),    // (e1, e5)
-                     __byte_perm(e.y, e.w, 0x5410),    // (e2, e6)
-                     __byte_perm(e.y, e.w, 0x7632));   // (e3, e7)
-      float part = bf16lo_to_f32(e.x) + bf16hi_to_f32(e.x) + bf16lo_to_f32(e.y) + bf16hi_to_f32(e.y) +
-                   bf16lo_to_f32(e.z) + bf16hi_to_f32(e.z) + bf16lo_to_f32(e.w) + bf16hi_to_f32(e.w);
+          make_uint4(__byte_perm(e.x, e.z, 0x5410), __byte_perm(e.y, e.w, 0x5410), pack_f16x2(e1, e5),
+                     pack_f16x2(e3, e7));
+      float part = -136.f * ((e0 + e2) + (e4 + e6)) - 72.f * ((e1 + e3) + (e5 + e7));
       part += __shfl_xor_sync(0xffffffffu, part, 1);
       part += __shfl_xor_sync(0xffffffffu, part, 2);
-      // lanes 4c..4c+3 hold the group sum of column c; this lane needs columns 2t, 2t+1
-      qinit[i][0] = -136.f * __shfl_sync(0xffffffffu, part, 8 * t);
-      qinit[i][1] = -136.f * __shfl_sync(0xffffffffu, part, 8 * t + 4);
+      // lanes 4c..4c+3 hold the group offset of column c; this lane needs columns 2t, 2t+1
+      qinit[i][0] = __shfl_sync(0xffffffffu, part, 8 * t);
+      qinit[i][1] = __shfl_sync(0xffffffffu, part, 8 * t + 4);
     }
 #pragma unroll
     for (int c = 0; c < (NG + 1) / 2; ++c) {
@@ -414,15 +418,15 @@ __device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
       const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + i * 512 + lane * 16);
       const float2 qi = *reinterpret_cast<const float2 *>(qsm + (NG + i / 2) * 512 + lane * 16 + (i & 1) * 8);
       float acc[4] = {qi.x, qi.y, qi.x, qi.y};
-      {
-        const uint32_t a[4] = {i4x2_biased(kw0[i]), i4x2_biased(kw1[i]), i4x2_biased(kw0[i] >> 4),
-                               i4x2_biased(kw1[i] >> 4)};
+      const uint32_t k80 = kw0[i] >> 8, k81 = kw1[i] >> 8;
+      {   // elements 0, 4 (k-slots 2t, 2t+1) and 2, 6 (2t+8, 2t+9): bf16, 136 + c
+        const uint32_t a[4] = {i4x2_biased(kw0[i]), i4x2_biased(kw1[i]), i4x2_biased(k80), i4x2_biased(k81)};
         mma_bf16(acc, a, qv.x, qv.y);
       }
-      {
-        const uint32_t a[4] = {i4x2_biased(kw0[i] >> 8), i4x2_biased(kw1[i] >> 8), i4x2_biased(kw0[i] >> 12),
-                               i4x2_biased(kw1[i] >> 12)};
-        mma_bf16(acc, a, qv.z, qv.w);
+      {   // elements 1, 5 and 3, 7: fp16, 72 + c (bits 4-7 convert in place)
+        const uint32_t a[4] = {i4x2_hi_biased_f16(kw0[i]), i4x2_hi_biased_f16(kw1[i]), i4x2_hi_biased_f16(k80),
+                               i4x2_hi_biased_f16(k81)};
+        mma_f16(acc, a, qv.z, qv.w);
       }
       const float k0 = ks0[i], k1 = ks1[i];
       sc01 = __ffma2_rn(make_float2(k0, k0), make_float2(acc[0], acc[1]), sc01);
