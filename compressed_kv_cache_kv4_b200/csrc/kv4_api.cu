@@ -96,13 +96,13 @@ int resolve_workers(int requested, const DecodeLaunch &l, int num_sms) {
   return (nw + kWarps - 1) / kWarps * kWarps;
 }
 
-// Workspace: plan int32 [B+1] | segs int64 [nw+1] | first, last int32
+// Workspace: plan int32 [B+1] | first, last int32
 // [2*B*Hkv] each | partial slots [2*B*Hkv + nw][slot_floats] (INT8 ranges,
 // then INT4 ranges, each offset by the worker index). Everything is written
 // before it is read within a call, so the workspace needs no clearing.
 size_t decode_ws_bytes(int B, int Hkv, int G, int D, int nw) {
   const size_t slot = (size_t)slot_floats(G, D) * 4;
-  return round_up((size_t)(B + 1) * 4, kAlign) + round_up((size_t)(nw + 1) * 8, kAlign) +
+  return round_up((size_t)(B + 1) * 4, kAlign) +
          2 * round_up((size_t)2 * B * Hkv * 4, kAlign) +
          round_up(((size_t)2 * B * Hkv + nw) * slot, kAlign);
 }
@@ -111,8 +111,6 @@ void carve_workspace(DecodeParams &p, void *ws) {
   uint8_t *w = static_cast<uint8_t *>(ws);
   p.plan = reinterpret_cast<int *>(w);
   w += round_up((size_t)(p.B + 1) * 4, kAlign);
-  p.segs = reinterpret_cast<long long *>(w);
-  w += round_up((size_t)(p.num_workers + 1) * 8, kAlign);
   p.first = reinterpret_cast<int *>(w);
   w += round_up((size_t)2 * p.B * p.Hkv * 4, kAlign);
   p.last = reinterpret_cast<int *>(w);

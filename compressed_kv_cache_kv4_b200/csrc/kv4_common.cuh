@@ -249,6 +249,14 @@ __device__ __forceinline__ long long worker_first_item(long long w, long long nw
   return T8 + (a - kW8 * T8 + kW4 - 1) / kW4;
 }
 
+// Number of workers that take part: at most one per kW8 weight units of work,
+// so that the share of each of them holds at least one item (a share spans at
+// least kW8 weight units and item starts are at most kW8 apart).
+__device__ __forceinline__ long long active_workers(long long nw, long long T8, long long T4) {
+  const long long cap = (kW8 * T8 + kW4 * T4) / kW8;
+  return cap < 1 ? 1 : (nw < cap ? nw : cap);
+}
+
 __host__ __device__ __forceinline__ int side_pages(int sink, int recent) { return (sink > 0 ? 1 : 0) + recent / 16; }
 
 }  // namespace kv4

@@ -807,16 +807,13 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) decode_kernel(Dec
   }
 
   const long long wid = (long long)blockIdx.x * kWarps + warp;
-  const long long NWk = p.num_workers;
   const int np8 = (!kBF16 && p.int8_units) ? side_pages(p.sink, p.recent) : 0;
   const long long T8 = (long long)p.B * p.Hkv * np8;
   const long long T4 = plan[p.B];
+  const long long NWk = active_workers(p.num_workers, T8, T4);
+  if (wid >= NWk) return;
   long long x = worker_first_item(wid, NWk, T8, T4);
   const long long z = worker_first_item(wid + 1, NWk, T8, T4);
-  if (lane == 0) {
-    p.segs[wid] = x;
-    if (wid == NWk - 1) p.segs[NWk] = z;
-  }
   const long long nbh = (long long)p.B * p.Hkv;
   if (x >= z) return;
 

@@ -33,7 +33,6 @@ struct DecodeParams {
   long long page_bytes, head_bytes, side_stride;
   float scale_log2;             // softmax_scale * log2(e)
   int *plan;                    // [B+1] prefix of attended INT4/bf16 page-heads
-  long long *segs;              // [num_workers+1] first item of each worker
   int *first;                   // [2*B*Hkv] worker owning the first item of each range
   int *last;                    // [2*B*Hkv] worker owning the last item of each range
   float *slots;                 // [2*B*Hkv + num_workers][slot_floats] partials

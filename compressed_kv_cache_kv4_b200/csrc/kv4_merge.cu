@@ -58,7 +58,6 @@ __global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
   if (task >= (long long)p.B * p.Hq) return;
   const int b = static_cast<int>(task / p.Hq), hq = static_cast<int>(task % p.Hq);
   const int h = hq / G, g = hq % G;
-  const long long nw = p.num_workers;
   const long long nbh = (long long)p.B * p.Hkv, r = (long long)b * p.Hkv + h;
 
   // Range bounds and the plan entries, all independent loads.
@@ -67,15 +66,14 @@ __global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
   const int f8 = __ldcg(&p.first[r]), l8 = __ldcg(&p.last[r]);
   const int f4 = __ldcg(&p.first[nbh + r]), l4 = __ldcg(&p.last[nbh + r]);
   const long long T8 = nbh * np8;
+  // the decode kernel's worker count; every one of them owns at least one item
+  const long long nw = active_workers(p.num_workers, T8, T4);
   // A range is used only if it has items; bounds outside [0, nw) (possible only
   // after a worker stopped on an error) drop the range instead of being read.
   const bool ok8 = np8 > 0 && f8 >= 0 && f8 <= l8 && l8 < nw;
   const bool ok4 = pb1 > pb0 && f4 >= 0 && f4 <= l4 && l4 < nw;
   const int n8 = ok8 ? l8 - f8 + 1 : 0;
   const int n = n8 + (ok4 ? l4 - f4 + 1 : 0);
-  // A worker's segment can be empty only if a worker's share of the weighted
-  // items is below the heaviest item; those workers wrote no partial.
-  const bool may_be_empty = kW8 * T8 + kW4 * T4 < kW8 * nw;
 
   float M = -INFINITY, den = 0.f, acc[DPL];
 #pragma unroll
@@ -91,14 +89,10 @@ __global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
       for (int e = 0; e < DPL; ++e) ok[k][e] = 0.f;
       if (i < n) {
         const long long w = i < n8 ? f8 + i : f4 + (i - n8);
-        const bool written =
-            !may_be_empty || worker_first_item(w, nw, T8, T4) != worker_first_item(w + 1, nw, T8, T4);
-        if (written) {
-          const float *slot = p.slots + ((i < n8 ? r : nbh + r) + w) * p.slot_floats;
-          mk[k] = __ldcg(slot + g);
-          lk[k] = __ldcg(slot + G + g);
-          Vec<DPL>::load(slot + p.slot_o_off + g * D + lane * DPL, ok[k]);
-        }
+        const float *slot = p.slots + ((i < n8 ? r : nbh + r) + w) * p.slot_floats;
+        mk[k] = __ldcg(slot + g);
+        lk[k] = __ldcg(slot + G + g);
+        Vec<DPL>::load(slot + p.slot_o_off + g * D + lane * DPL, ok[k]);
       }
     }
     float mc = -INFINITY;
