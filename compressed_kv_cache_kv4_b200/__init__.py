@@ -68,7 +68,7 @@ def lib():
         "kv4_get_error": (C.c_int, [_P, _P, C.POINTER(C.c_uint32)]),
         "kv4_debug_set_wait_limit": (C.c_int, [_P, _I64]),
         "kv4_device_info": (C.c_int, [C.POINTER(_I32), C.POINTER(_I32)]),
-        "kv4_timing_enable": (C.c_int, [_I32]),
+        "kv4_timing_enable": (C.c_int, [_I32, _I32]),
         "kv4_timing_read": (C.c_int, [_I32, C.POINTER(C.c_double), C.POINTER(_I32)]),
         "kv4_timing_disable": (C.c_int, []),
     }
@@ -212,8 +212,8 @@ def kv4_device_info():
     return a.value, b.value
 
 
-def kv4_timing_enable(max_records):
-    _check(lib().kv4_timing_enable(int(max_records)), "kv4_timing_enable")
+def kv4_timing_enable(max_records, every=1):
+    _check(lib().kv4_timing_enable(int(max_records), int(every)), "kv4_timing_enable")
 
 
 def kv4_timing_read(kind):

@@ -124,7 +124,9 @@ kv4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KV4_OK : KV4_E
 struct Timing {
   bool on = false;
   int max_records = 0;
+  int every = 1;          // record every `every`-th call of a kind
   int used[2] = {0, 0};
+  long long calls[2] = {0, 0};
   std::vector<cudaEvent_t> ev[2];   // 2 * max_records events per kind
 };
 Timing g_timing;
@@ -134,6 +136,7 @@ void timing_pair(int kind, cudaEvent_t *e0, cudaEvent_t *e1) {
   std::lock_guard<std::mutex> lk(g_timing_mu);
   *e0 = *e1 = nullptr;
   if (!g_timing.on || g_timing.used[kind] >= g_timing.max_records) return;
+  if (g_timing.calls[kind]++ % g_timing.every != 0) return;
   const int i = g_timing.used[kind]++;
   *e0 = g_timing.ev[kind][2 * i];
   *e1 = g_timing.ev[kind][2 * i + 1];
@@ -144,6 +147,7 @@ void timing_free() {
     for (cudaEvent_t e : g_timing.ev[k]) cudaEventDestroy(e);
     g_timing.ev[k].clear();
     g_timing.used[k] = 0;
+    g_timing.calls[k] = 0;
   }
   g_timing.on = false;
   g_timing.max_records = 0;
@@ -432,8 +436,8 @@ kv4_status kv4_device_info(int32_t *num_sms, int32_t *default_workers_out) {
   return KV4_OK;
 }
 
-kv4_status kv4_timing_enable(int32_t max_records) {
-  if (max_records < 1) return KV4_ERR_INVALID;
+kv4_status kv4_timing_enable(int32_t max_records, int32_t every) {
+  if (max_records < 1 || every < 1) return KV4_ERR_INVALID;
   std::lock_guard<std::mutex> lk(g_timing_mu);
   timing_free();
   for (int k = 0; k < 2; ++k) {
@@ -446,6 +450,7 @@ kv4_status kv4_timing_enable(int32_t max_records) {
     }
   }
   g_timing.max_records = max_records;
+  g_timing.every = every;
   g_timing.on = true;
   return KV4_OK;
 }

@@ -26,7 +26,8 @@
  * Conventions for every call:
  *  - All pointers named *_dev or documented "device" are device memory owned by
  *    the caller; the library never allocates device memory except the 4-byte
- *    error word owned by a kv4_cache.
+ *    error word owned by a kv4_cache (kv4_decode_attn_noalloc's fixed scratch
+ *    is a variable of the library's module, reserved when the module loads).
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL =
  *    the legacy default stream) unless stated otherwise.
  *  - Argument errors are detected on the host before any launch and return
@@ -247,15 +248,18 @@ kv4_status kv4_get_error(kv4_cache *cache, void *stream, uint32_t *bits);
 kv4_status kv4_debug_set_wait_limit(kv4_cache *cache, int64_t cycles);
 
 /*
- * Kernel timing hook (host only). While enabled, every kv4_decode_attn and
- * bf16_paged_decode_attn call records a pair of CUDA events on its stream
- * immediately before and after its split-K worker kernel, for up to
- * `max_records` calls per kind. kv4_timing_read synchronises those events and
- * returns the summed worker-kernel time in milliseconds and the number of
- * recorded calls for `kind` (0 = kv4_decode_attn, 1 = bf16_paged_decode_attn),
- * then clears the records. kv4_timing_disable frees the events.
+ * Kernel timing hook (host only). While enabled, every `every`-th
+ * kv4_decode_attn and bf16_paged_decode_attn call (counted per kind, the first
+ * call included) records a pair of CUDA events on its stream immediately
+ * before and after its split-K worker kernel, for up to `max_records` calls per
+ * kind. An event between two kernels keeps the second from starting early
+ * (programmatic dependent launch), so sampling (every > 1) leaves most calls
+ * undisturbed. kv4_timing_read synchronises those events and returns the summed
+ * worker-kernel time in milliseconds and the number of recorded calls for
+ * `kind` (0 = kv4_decode_attn, 1 = bf16_paged_decode_attn), then clears the
+ * records. kv4_timing_disable frees the events. max_records, every >= 1.
  */
-kv4_status kv4_timing_enable(int32_t max_records);
+kv4_status kv4_timing_enable(int32_t max_records, int32_t every);
 kv4_status kv4_timing_read(int32_t kind, double *total_ms, int32_t *count);
 kv4_status kv4_timing_disable(void);
 
