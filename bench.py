@@ -486,6 +486,16 @@ def secondary(wl, L0, cache, ptd, pt_np, npages, kpre, vpre, offpre, lens_pre, s
                                "kv4_speedup": callb / call}
     del pages
 
+    # prefill: append of every prompt position (rewrites the same bytes each call)
+    offs_t = torch.as_tensor(offpre.astype(np.int32), device="cuda")
+    zeros = torch.zeros(wl.B, dtype=torch.int32, device="cuda")
+    callp, _ = time_calls(lambda: cache.append(kpre, vpre, offs_t, zeros, ptd), 20)
+    T = int(offpre[-1])
+    n8 = int(np.minimum(lens_pre, wl.sink + wl.recent).astype(np.int64).sum())
+    pbytes = T * wl.Hkv * (4 * wl.D + 18 * wl.D // 16) + n8 * wl.Hkv * 2 * (wl.D + 2) + (wl.B + 1) * 4
+    out["prefill_append"] = {"tokens": T, "us": callp * 1e3, "tokens_per_s": T / (callp / 1e3),
+                             "gbs": pbytes / (callp / 1e3) / 1e9, "frac_of_peak": pbytes / (callp / 1e3) / 1e9 / peak}
+
     # eviction workload: top-k (per KV head) + masked decode at 10/30/50/90/100%
     out["evict"] = evict_secondary()
     return out

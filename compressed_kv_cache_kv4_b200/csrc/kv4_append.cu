@@ -7,8 +7,14 @@
 // head_dim elements, INT8 per token row; scale = max|x| / qmax rounded toward
 // +inf to fp16; code = x / scale rounded to nearest-even.
 //
-// One warp per (new position, KV head, K or V); lane l holds D/32 consecutive
-// elements.
+// Two kernels. append_pages_kernel takes every page the append fills
+// completely (a prefill, or a multi-token append that crosses page
+// boundaries): one warp per (page, KV head), lane l quantises row l % 16 of K
+// (l < 16) or V (l >= 16) group by group into a shared-memory image of the
+// 18*D-byte head block, which the warp then writes out with 16-byte stores.
+// append_kernel takes the rest: one warp per (new position, KV head, K or V),
+// lane l holding D/32 consecutive elements, for the INT4 slots of partially
+// filled pages and for every INT8 side-cache row.
 //
 // Scale: fp32 IEEE division then round-up to fp16 equals rounding the exact
 // quotient a/7 (a/127) up: for a bf16 numerator the quotient is either exact
@@ -19,6 +25,8 @@
 // x * RN(1/s) to the nearest integer is exact except at true half-way points;
 // those are detected exactly through the residual c*s - x (exact in fp32) and
 // resolved to the even code.
+#include <algorithm>
+
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
 
@@ -66,22 +74,10 @@ __device__ __forceinline__ uint16_t quant_lane(const float (&x)[EPL], int span, 
   return bits;
 }
 
-template <int D>
-__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
-  constexpr int EPL = D / 32;              // elements per lane
-  constexpr int LPG = kGroup / EPL;        // lanes per INT4 group
-  const int lane = threadIdx.x & 31;
-  const long long task = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  pdl_wait();
-  pdl_launch_dependents();
-  if (task >= p.T * p.Hkv * 2) return;
-  const int kv = static_cast<int>(task & 1);   // 0: K, 1: V
-  const long long j = (task >> 1) / p.Hkv;
-  const int h = static_cast<int>((task >> 1) % p.Hkv);
-
-  int b, pos, L_new;
+// Sequence b owning packed row j, the row's position and the sequence's new length.
+__device__ __forceinline__ void locate_row(const AppendParams &p, long long j, int &b, int &pos, int &L_new) {
   if (p.offsets) {
-    // sequence owning row j: largest b with offsets[b] <= j
+    // largest b with offsets[b] <= j
     int lo = 0, hi = p.B - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -96,10 +92,168 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     pos = p.lens_old[b];
     L_new = pos + 1;
   }
-  if (pos < 0 || pos >= p.pt_stride * kPageTokens) {
-    if (lane == 0) set_error(p.err, kErrCapacity);
-    return;
+}
+
+// Position pos lies in a page that the append [L_old, L_new) fills completely.
+__device__ __forceinline__ bool in_full_page(int pos, int L_old, int L_new) {
+  const int f0 = (L_old + kPageTokens - 1) / kPageTokens * kPageTokens;
+  const int f1 = L_new / kPageTokens * kPageTokens;
+  return pos >= f0 && pos < f1;
+}
+
+// Scale bits and codes of one group of 32 values held by one thread (the same
+// quantiser as quant_lane, without lanes to combine).
+__device__ __forceinline__ uint16_t quant_group32(const float (&x)[kGroup], int (&c)[kGroup], uint32_t *err) {
+  float a = 0.f;
+#pragma unroll
+  for (int e = 0; e < kGroup; ++e) a = fmaxf(a, fabsf(x[e]));
+  if (a == 0.f) {
+#pragma unroll
+    for (int e = 0; e < kGroup; ++e) c[e] = 0;
+    return 0;
   }
+  uint16_t bits = __half_as_ushort(__float2half_ru(__fdiv_rn(a, 7.f)));
+  if (bits == 0x7C00u) {           // a/7 > 65504: saturate and flag
+    bits = 0x7BFFu;
+    set_error(err, kErrRange);
+  }
+  const float s = half_bits_to_f32(bits);
+  const float r = __frcp_rn(s);
+#pragma unroll
+  for (int e = 0; e < kGroup; ++e) c[e] = static_cast<int>(fminf(fmaxf(round_code(x[e], s, r), -7.f), 7.f));
+  return bits;
+}
+
+// One warp per (page the append fills completely, KV head). Every CTA first
+// forms, in shared memory, the prefix over sequences of their completely
+// filled pages, then maps its warps' units onto (sequence, page, head).
+template <int D>
+__global__ void __launch_bounds__(256) append_pages_kernel(AppendParams p) {
+  constexpr int WARPS = 8, NG = D / kGroup;
+  __shared__ __align__(16) uint8_t img[WARPS][18 * D];
+  __shared__ int wtot[WARPS];
+  extern __shared__ int fplan[];   // [B + 1]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_launch_dependents();
+
+  auto full_pages = [&](int b) {
+    const int L_old = p.lens_old[b];
+    if (L_old < 0) return 0;
+    const int L_new = L_old + (p.offsets[b + 1] - p.offsets[b]);
+    const int f0 = (L_old + kPageTokens - 1) / kPageTokens, f1 = L_new / kPageTokens;
+    return f1 > f0 ? f1 - f0 : 0;
+  };
+  const int chunk = (p.B + WARPS * 32 - 1) / (WARPS * 32);
+  const int b0 = min(p.B, tid * chunk), b1 = min(p.B, b0 + chunk);
+  int mine = 0;
+  for (int b = b0; b < b1; ++b) mine += full_pages(b);
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  int run = incl - mine;
+  for (int w = 0; w < warp; ++w) run += wtot[w];
+  for (int b = b0; b < b1; ++b) {
+    fplan[b] = run;
+    run += full_pages(b);
+  }
+  if (tid == WARPS * 32 - 1) fplan[p.B] = run;
+  __syncthreads();
+
+  const long long units = (long long)fplan[p.B] * p.Hkv;
+  uint8_t *im = img[warp];
+  const int r = lane & 15, kv = lane >> 4;
+  for (long long u = (long long)blockIdx.x * WARPS + warp; u < units; u += (long long)gridDim.x * WARPS) {
+    const int unit = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
+    int lo = 0, hi = p.B - 1;   // sequence: largest b with fplan[b] <= unit
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (fplan[mid] <= unit) lo = mid;
+      else hi = mid - 1;
+    }
+    const int b = lo;
+    const int L_old = p.lens_old[b];
+    const int pg = (L_old + kPageTokens - 1) / kPageTokens + (unit - fplan[b]);
+    if (pg >= p.pt_stride) {
+      if (lane == 0) set_error(p.err, kErrCapacity);
+      continue;
+    }
+    const int page = p.page_table[(long long)b * p.pt_stride + pg];
+    if (page < 0 || page >= p.num_pages) {
+      if (lane == 0) set_error(p.err, kErrBounds);
+      continue;
+    }
+    // rows j .. j+15 are the page's slots 0..15 (all new, all of sequence b)
+    const long long j = p.offsets[b] + (pg * kPageTokens - L_old);
+    const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + ((j + r) * p.Hkv + h) * D;
+#pragma unroll 1
+    for (int i = 0; i < NG; ++i) {
+      float x[kGroup];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(src + kGroup * i + 8 * q);
+        x[8 * q + 0] = bf16lo_to_f32(w.x);
+        x[8 * q + 1] = bf16hi_to_f32(w.x);
+        x[8 * q + 2] = bf16lo_to_f32(w.y);
+        x[8 * q + 3] = bf16hi_to_f32(w.y);
+        x[8 * q + 4] = bf16lo_to_f32(w.z);
+        x[8 * q + 5] = bf16hi_to_f32(w.z);
+        x[8 * q + 6] = bf16lo_to_f32(w.w);
+        x[8 * q + 7] = bf16hi_to_f32(w.w);
+      }
+      int c[kGroup];
+      const uint16_t sbits = quant_group32(x, c, p.err);
+      if (kv == 0) {
+        // K: element 32i + 8t + k of row r is nibble k of the word at
+        // r*D/2 + t*D/8 + 4i
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) w |= nib(c[8 * t + k]) << (4 * k);
+          *reinterpret_cast<uint32_t *>(im + r * (D / 2) + t * (D / 8) + 4 * i) = w;
+        }
+        *reinterpret_cast<uint16_t *>(im + 16 * D + 2 * (r * NG + i)) = sbits;
+      } else {
+        // V: the byte of (slot r, element d) pairs d and d+8 (low, high nibble)
+#pragma unroll
+        for (int e = 0; e < kGroup; ++e) {
+          if ((e % 16) >= 8) continue;
+          const int d = kGroup * i + e;
+          const int m = d / 16, g8 = d % 8, tt = (r % 8) / 2;
+          const int word = (m / 4) * 128 + (4 * g8 + tt) * 4 + (m % 4);
+          im[8 * D + 4 * word + 2 * (r % 2) + r / 8] = static_cast<uint8_t>(nib(c[e]) | nib(c[e + 8]) << 4);
+        }
+        *reinterpret_cast<uint16_t *>(im + 17 * D + 2 * (r * NG + i)) = sbits;
+      }
+    }
+    __syncwarp();
+    uint4 *dst = reinterpret_cast<uint4 *>(p.pool + (long long)page * p.page_bytes + (long long)h * p.head_bytes);
+    const uint4 *srci = reinterpret_cast<const uint4 *>(im);
+    for (int q = lane; q < 18 * D / 16; q += 32) dst[q] = srci[q];
+    __syncwarp();
+  }
+}
+
+// Quantise and store row (j, head h, K or V) of position pos of sequence b:
+// the INT4 slot (unless the page kernel owns the page) and the INT8 side rows.
+// One warp; lane l holds D/32 consecutive elements.
+template <int D>
+__device__ __forceinline__ void append_row(const AppendParams &p, long long j, int h, int kv, int b, int pos,
+                                           int L_new, int lane) {
+  constexpr int EPL = D / 32;              // elements per lane
+  constexpr int LPG = kGroup / EPL;        // lanes per INT4 group
+  const int S = p.sink, R = p.recent;
+  const int sink_row = pos < S ? pos : -1;
+  const int ring_row = (R > 0 && pos >= L_new - R) ? (S > 0 ? 16 : 0) + pos % R : -1;
+  // INT4 slots of pages this append fills completely belong to append_pages_kernel
+  const bool skip4 = p.page_kernel && in_full_page(pos, p.lens_old[b], L_new);
+  if (skip4 && sink_row < 0 && ring_row < 0) return;
   const int page = p.page_table[(long long)b * p.pt_stride + pos / kPageTokens];
   if (page < 0 || page >= p.num_pages) {
     if (lane == 0 && kv == 0) set_error(p.err, kErrBounds);
@@ -109,10 +263,6 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   uint8_t *blk = p.pool + (long long)page * p.page_bytes + (long long)h * p.head_bytes;
   const int d0 = lane * EPL;
   const int grp = d0 / kGroup;
-
-  const int S = p.sink, R = p.recent;
-  const int sink_row = pos < S ? pos : -1;
-  const int ring_row = (R > 0 && pos >= L_new - R) ? (S > 0 ? 16 : 0) + pos % R : -1;
   uint8_t *sblk = p.side + ((long long)b * p.Hkv + h) * p.side_stride;
   const long long spage = 32LL * D + 64;
 
@@ -133,8 +283,9 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
 
     // ---- INT4 copy, one scale per group of 32
     int c[EPL];
-    const uint16_t s4 = quant_lane<EPL>(x, LPG, 7.f, c, p.err);
-    if (kv == 0) {
+    const uint16_t s4 = skip4 ? 0 : quant_lane<EPL>(x, LPG, 7.f, c, p.err);
+    if (skip4) {
+    } else if (kv == 0) {
       // K: element d at row r, chunk (d%32)/8, word d/32, nibble d%8
       const int t = (d0 % kGroup) / 8, k0 = d0 % 8;
       uint8_t *dst = blk + r * (D / 2) + t * (D / 8) + 4 * grp + k0 / 2;
@@ -212,13 +363,74 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   }
 }
 
-cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream) {
+template <int D>
+__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+  const int lane = threadIdx.x & 31;
+  const long long task = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (task >= p.T * p.Hkv * 2) return;
+  const int kv = static_cast<int>(task & 1);   // 0: K, 1: V
+  const long long j = (task >> 1) / p.Hkv;
+  const int h = static_cast<int>((task >> 1) % p.Hkv);
+  int b, pos, L_new;
+  locate_row(p, j, b, pos, L_new);
+  if (pos < 0 || pos >= p.pt_stride * kPageTokens) {
+    if (lane == 0) set_error(p.err, kErrCapacity);
+    return;
+  }
+  append_row<D>(p, j, h, kv, b, pos, L_new, lane);
+}
+
+// Used with append_pages_kernel: one warp per new position, looping over the
+// KV heads and K / V, for the positions that have work outside the pages the
+// append fills completely (slots of partially filled pages, INT8 side rows).
+template <int D>
+__global__ void __launch_bounds__(256) append_tokens_kernel(AppendParams p) {
+  const int lane = threadIdx.x & 31;
+  const long long j = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (j >= p.T) return;
+  int b, pos, L_new;
+  locate_row(p, j, b, pos, L_new);
+  if (pos < 0 || pos >= p.pt_stride * kPageTokens) {
+    if (lane == 0) set_error(p.err, kErrCapacity);
+    return;
+  }
+  const bool int8_row = pos < p.sink || (p.recent > 0 && pos >= L_new - p.recent);
+  if (in_full_page(pos, p.lens_old[b], L_new) && !int8_row) return;
+  for (int hk = 0; hk < 2 * p.Hkv; ++hk) append_row<D>(p, j, hk >> 1, hk & 1, b, pos, L_new, lane);
+}
+
+cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream) {
+  AppendParams p = p_in;
   const long long tasks = p.T * p.Hkv * 2;
   if (tasks == 0) return cudaSuccess;
   const int warps_per_block = 8;
-  const unsigned blocks = static_cast<unsigned>((tasks + warps_per_block - 1) / warps_per_block);
-  if (D == 128) return launch_pdl(append_kernel<128>, dim3(blocks), dim3(32 * warps_per_block), 0, stream, p);
-  return launch_pdl(append_kernel<64>, dim3(blocks), dim3(32 * warps_per_block), 0, stream, p);
+  // Pages can only be filled completely by a multi-position append; the page
+  // kernel reads rows with 16-byte loads and keeps its plan in shared memory.
+  const bool aligned16 = ((reinterpret_cast<uintptr_t>(p.k) | reinterpret_cast<uintptr_t>(p.v)) & 15u) == 0;
+  // (the plan, 4 bytes per sequence, stays within the default 48 KB with the page images)
+  p.page_kernel = (p.offsets && p.T >= kPageTokens && aligned16 && p.B <= 7168) ? 1 : 0;
+  if (!p.page_kernel) {
+    const unsigned blocks = static_cast<unsigned>((tasks + warps_per_block - 1) / warps_per_block);
+    if (D == 128) return launch_pdl(append_kernel<128>, dim3(blocks), dim3(32 * warps_per_block), 0, stream, p);
+    return launch_pdl(append_kernel<64>, dim3(blocks), dim3(32 * warps_per_block), 0, stream, p);
+  }
+  const long long units = (p.T / kPageTokens) * p.Hkv;   // upper bound on (full page, head) units
+  const unsigned pblocks = static_cast<unsigned>(
+      std::max(1LL, std::min((units + warps_per_block - 1) / warps_per_block, 8192LL)));
+  const size_t plan_bytes = (size_t)(p.B + 1) * 4;
+  cudaError_t e = D == 128 ? launch_pdl(append_pages_kernel<128>, dim3(pblocks), dim3(32 * warps_per_block),
+                                        plan_bytes, stream, p)
+                           : launch_pdl(append_pages_kernel<64>, dim3(pblocks), dim3(32 * warps_per_block),
+                                        plan_bytes, stream, p);
+  if (e != cudaSuccess) return e;
+  const unsigned tblocks = static_cast<unsigned>((p.T + warps_per_block - 1) / warps_per_block);
+  if (D == 128)
+    return launch_pdl(append_tokens_kernel<128>, dim3(tblocks), dim3(32 * warps_per_block), 0, stream, p);
+  return launch_pdl(append_tokens_kernel<64>, dim3(tblocks), dim3(32 * warps_per_block), 0, stream, p);
 }
 
 }  // namespace kv4

@@ -19,6 +19,7 @@ struct AppendParams {
   uint8_t *side;
   long long page_bytes, head_bytes, side_stride;
   uint32_t *err;
+  int page_kernel;          // 1: pages filled completely by this append go through append_pages_kernel
 };
 
 struct DecodeParams {

@@ -45,6 +45,29 @@ def test_append_bytes_match_oracle(name, chunks):
     assert np.array_equal(gs, side), "side cache differs at %s" % np.flatnonzero(gs != side)[:10]
 
 
+def test_append_unaligned_rows_match_oracle():
+    """k_new / v_new 8- but not 16-byte aligned: whole pages go through the
+    per-position kernel instead of the page kernel; the bytes are the same."""
+    wl = small_wl([40, 64, 17, 200], Hq=8, Hkv=2)
+    c = Case(wl)
+    c.make_cache()
+    T = c.k.shape[0]
+    kbuf = torch.zeros(T * wl.Hkv * wl.D + 4, dtype=torch.bfloat16, device="cuda")
+    vbuf = torch.zeros_like(kbuf)
+    k = kbuf[4:].view(T, wl.Hkv, wl.D)
+    v = vbuf[4:].view(T, wl.Hkv, wl.D)
+    k.copy_(c.k.to("cuda"))
+    v.copy_(c.v.to("cuda"))
+    assert k.data_ptr() % 16 == 8
+    c.cache.append(k, v, torch.as_tensor(c.off.astype(np.int32), device="cuda"),
+                   torch.zeros(wl.B, dtype=torch.int32, device="cuda"), c.pt)
+    torch.cuda.synchronize()
+    pool, side, flags = c.oracle_cache()
+    assert flags == 0 and c.cache.get_error()[0] == K.KV4_OK
+    assert np.array_equal(c.cache.pool.cpu().numpy(), pool)
+    assert np.array_equal(c.cache.side.cpu().numpy(), side)
+
+
 def test_append_single_token_steps_ring():
     """Prefill, then one token per step: the ring keeps the last 128 positions
     exactly as the oracle's image of the final lengths."""
