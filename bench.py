@@ -664,7 +664,7 @@ def main():
         line = {"metric": "decode-attn KV positions/s and achieved HBM GB/s (% of B200 peak), 8B-like GQA",
                 "value": res["value"], "unit": "KV positions/s", "n_gpus": ws, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "int4+int8 codes, bf16 mma, f32 accumulate",
+                "scaling": "weak", "vs_baseline": None, "dtype": "int4/int8 codes; bf16+fp16 mma, f32 accumulate",
                 "data": "synthetic", "config": workload_config(wl), "roofline": res["roofline"],
                 "cpu_baseline": res.get("cpu_baseline"), "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
                 "clocks": res["clocks"], "step_hbm_gbs": res["step_gbs"], "worker_avg_us": res["worker_avg_us"],
