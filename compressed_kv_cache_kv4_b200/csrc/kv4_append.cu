@@ -113,14 +113,20 @@ __device__ __forceinline__ uint16_t quant_group32(const float (&x)[kGroup], int 
     return 0;
   }
   uint16_t bits = __half_as_ushort(__float2half_ru(__fdiv_rn(a, 7.f)));
-  if (bits == 0x7C00u) {           // a/7 > 65504: saturate and flag
+  const bool sat = bits == 0x7C00u;
+  if (sat) {                       // a/7 > 65504: saturate and flag
     bits = 0x7BFFu;
     set_error(err, kErrRange);
   }
   const float s = half_bits_to_f32(bits);
   const float r = __frcp_rn(s);
+  // s >= max|x| / 7 makes |x / s| <= 7, so the codes need a clamp only when
+  // the scale saturated
 #pragma unroll
-  for (int e = 0; e < kGroup; ++e) c[e] = static_cast<int>(fminf(fmaxf(round_code(x[e], s, r), -7.f), 7.f));
+  for (int e = 0; e < kGroup; ++e) {
+    const float v = round_code(x[e], s, r);
+    c[e] = static_cast<int>(sat ? fminf(fmaxf(v, -7.f), 7.f) : v);
+  }
   return bits;
 }
 
@@ -382,25 +388,81 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   append_row<D>(p, j, h, kv, b, pos, L_new, lane);
 }
 
-// Used with append_pages_kernel: one warp per new position, looping over the
-// KV heads and K / V, for the positions that have work outside the pages the
-// append fills completely (slots of partially filled pages, INT8 side rows).
+// Positions of sequence b that have work outside the pages the append fills
+// completely: the slots of partly filled pages and the INT8 sink and ring
+// rows. They form [L_old, a_end) and [b_start, L_new) (one range if these
+// meet); returns their number.
+__device__ __forceinline__ int token_work(const AppendParams &p, int b, int &L_old, int &a_end, int &b_start) {
+  L_old = p.lens_old[b];
+  const int L_new = L_old + (p.offsets[b + 1] - p.offsets[b]);
+  if (L_old < 0) {                 // invalid length: every position (the row kernel flags it)
+    a_end = b_start = L_new;
+    return L_new - L_old;
+  }
+  const int f0 = (L_old + kPageTokens - 1) / kPageTokens * kPageTokens;
+  const int f1 = L_new / kPageTokens * kPageTokens;
+  a_end = min(L_new, max(f0, min(p.sink, f1)));
+  b_start = max(L_old, min(f1, max(L_new - p.recent, f0)));
+  if (a_end >= b_start) {
+    a_end = b_start = L_new;
+    return L_new - L_old;
+  }
+  return (a_end - L_old) + (L_new - b_start);
+}
+
+// Used with append_pages_kernel: one warp per position that has work outside
+// the pages the append fills completely, looping over the KV heads and K / V.
+// Every CTA forms the prefix of those positions over sequences in shared memory.
 template <int D>
 __global__ void __launch_bounds__(256) append_tokens_kernel(AppendParams p) {
-  const int lane = threadIdx.x & 31;
-  const long long j = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  constexpr int WARPS = 8;
+  __shared__ int wtot[WARPS];
+  extern __shared__ int tplan[];   // [B + 1]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
   pdl_launch_dependents();
-  if (j >= p.T) return;
-  int b, pos, L_new;
-  locate_row(p, j, b, pos, L_new);
-  if (pos < 0 || pos >= p.pt_stride * kPageTokens) {
-    if (lane == 0) set_error(p.err, kErrCapacity);
-    return;
+  const int chunk = (p.B + WARPS * 32 - 1) / (WARPS * 32);
+  const int b0 = min(p.B, tid * chunk), b1 = min(p.B, b0 + chunk);
+  int mine = 0, lo_, ae_, bs_;
+  for (int b = b0; b < b1; ++b) mine += token_work(p, b, lo_, ae_, bs_);
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
-  const bool int8_row = pos < p.sink || (p.recent > 0 && pos >= L_new - p.recent);
-  if (in_full_page(pos, p.lens_old[b], L_new) && !int8_row) return;
-  for (int hk = 0; hk < 2 * p.Hkv; ++hk) append_row<D>(p, j, hk >> 1, hk & 1, b, pos, L_new, lane);
+  if (lane == 31) wtot[warp] = incl;
+  __syncthreads();
+  int run = incl - mine;
+  for (int w = 0; w < warp; ++w) run += wtot[w];
+  for (int b = b0; b < b1; ++b) {
+    tplan[b] = run;
+    run += token_work(p, b, lo_, ae_, bs_);
+  }
+  if (tid == WARPS * 32 - 1) tplan[p.B] = run;
+  __syncthreads();
+
+  const int total = tplan[p.B];
+  for (long long u = (long long)blockIdx.x * WARPS + warp; u < total; u += (long long)gridDim.x * WARPS) {
+    int lo = 0, hi = p.B - 1;   // sequence: largest b with tplan[b] <= u
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tplan[mid] <= u) lo = mid;
+      else hi = mid - 1;
+    }
+    const int b = lo;
+    int L_old, a_end, b_start;
+    token_work(p, b, L_old, a_end, b_start);
+    const int k = static_cast<int>(u - tplan[b]);
+    const int pos = k < a_end - L_old ? L_old + k : b_start + (k - (a_end - L_old));
+    const int L_new = L_old + (p.offsets[b + 1] - p.offsets[b]);
+    const long long j = p.offsets[b] + (pos - L_old);
+    if (pos < 0 || pos >= p.pt_stride * kPageTokens) {
+      if (lane == 0) set_error(p.err, kErrCapacity);
+      continue;
+    }
+    for (int hk = 0; hk < 2 * p.Hkv; ++hk) append_row<D>(p, j, hk >> 1, hk & 1, b, pos, L_new, lane);
+  }
 }
 
 cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream) {
@@ -427,10 +489,14 @@ cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream) 
                            : launch_pdl(append_pages_kernel<64>, dim3(pblocks), dim3(32 * warps_per_block),
                                         plan_bytes, stream, p);
   if (e != cudaSuccess) return e;
-  const unsigned tblocks = static_cast<unsigned>((p.T + warps_per_block - 1) / warps_per_block);
+  // upper bound on the positions with work left: all of them, or per sequence
+  // two partial pages plus the sink and ring rows
+  const long long tw = std::min<long long>(p.T, (long long)p.B * (2 * kPageTokens + p.sink + p.recent));
+  const unsigned tblocks = static_cast<unsigned>(
+      std::max(1LL, std::min((tw + warps_per_block - 1) / warps_per_block, 8192LL)));
   if (D == 128)
-    return launch_pdl(append_tokens_kernel<128>, dim3(tblocks), dim3(32 * warps_per_block), 0, stream, p);
-  return launch_pdl(append_tokens_kernel<64>, dim3(tblocks), dim3(32 * warps_per_block), 0, stream, p);
+    return launch_pdl(append_tokens_kernel<128>, dim3(tblocks), dim3(32 * warps_per_block), plan_bytes, stream, p);
+  return launch_pdl(append_tokens_kernel<64>, dim3(tblocks), dim3(32 * warps_per_block), plan_bytes, stream, p);
 }
 
 }  // namespace kv4
