@@ -8,14 +8,14 @@ here, so the two never share anything but their inputs.
 Workloads (the pages run RL rollouts of Qwen3-4B/8B-Base, which are not
 available; these synthetic shapes stand in for them):
 
-1. ``tiny``   B=2, L=(200, 37), 4 query / 2 KV heads, D=64, outlier K channels
+- ``tiny``   B=2, L=(200, 37), 4 query / 2 KV heads, D=64, outlier K channels
               3 and 17 scaled x8, softmax scale 1/8.
-2. ``qwen8b`` B=64, L ~ U{1024..8192}, 32/8 heads, D=128, per KV head 4 random
+- ``qwen8b`` B=64, L ~ U{1024..8192}, 32/8 heads, D=128, per KV head 4 random
               K channels scaled x10, pages randomly permuted.
-3. ``async``  B=256, L0 = clip(round(exp(N(ln 4096, 1))), 256, 32768), same
+- ``async``  B=256, L0 = clip(round(exp(N(ln 4096, 1))), 256, 32768), same
               heads; 64 decode steps of one appended token per sequence.
-4. ``long``   B=4, L=131072, same heads.
-5. ``evict``  B=64, L=16384, same heads; per-position scores are the summed
+- ``long``   B=4, L=131072, same heads.
+- ``evict``  B=64, L=16384, same heads; per-position scores are the summed
               softmax attention of 32 random N(0,1) queries at the 32 positions
               before the current one (H2O-style accumulated attention).
 
@@ -71,27 +71,27 @@ def _f32_inv_sqrt(D):
 
 def workload(name, **over):
     """Build one of the five workloads; keyword overrides shrink it for tests."""
-    if name in ("tiny", 1):
+    if name == "tiny":
         wl = Workload("tiny", 1001, 2, 4, 2, 64, np.array([200, 37], np.int32), 0.125,
                       outlier_channels=(3, 17), outlier_gain=8.0)
-    elif name in ("qwen8b", 2):
+    elif name == "qwen8b":
         B = over.pop("B", 64)
         lo, hi = over.pop("len_range", (1024, 8192))
         g = _gen(1002, 0)
         lens = torch.randint(lo, hi + 1, (B,), generator=g).numpy().astype(np.int32)
         wl = Workload("qwen8b", 1002, B, 32, 8, 128, lens, _f32_inv_sqrt(128))
-    elif name in ("async", 3):
+    elif name == "async":
         B = over.pop("B", 256)
         med, lo, hi = over.pop("len_dist", (4096, 256, 32768))
         g = _gen(1003, 0)
         z = torch.randn(B, generator=g, dtype=torch.float64).numpy()
         lens = np.clip(np.round(np.exp(math.log(med) + 1.0 * z)), lo, hi).astype(np.int32)
         wl = Workload("async", 1003, B, 32, 8, 128, lens, _f32_inv_sqrt(128), steps=64)
-    elif name in ("long", 4):
+    elif name == "long":
         B = over.pop("B", 4)
         L = over.pop("L", 131072)
         wl = Workload("long", 1004, B, 32, 8, 128, np.full(B, L, np.int32), _f32_inv_sqrt(128))
-    elif name in ("evict", 5):
+    elif name == "evict":
         B = over.pop("B", 64)
         L = over.pop("L", 16384)
         wl = Workload("evict", 1005, B, 32, 8, 128, np.full(B, L, np.int32), _f32_inv_sqrt(128),

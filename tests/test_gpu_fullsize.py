@@ -2,12 +2,12 @@
 times (default worker count, bf16 output, whole batch in one call), on sampled
 outputs the oracle computes sequence by sequence.
 
-- qwen8b (config 2): B = 64, L ~ U[1024, 8192].
-- async (config 3): B = 256, log-normal lengths up to 32768, 64 steps of
+- qwen8b: B = 64, L ~ U[1024, 8192].
+- async: B = 256, log-normal lengths up to 32768, 64 steps of
   one-token append + decode; checked at steps 0, 31 and 63.
-- long (config 4): B = 4, L = 131072; the split-K partials of each sequence
+- long: B = 4, L = 131072; the split-K partials of each sequence
   against the single-pass oracle.
-- evict (config 5): B = 64, L = 16384; top-k masks bit-exact at every budget,
+- evict: B = 64, L = 16384; top-k masks bit-exact at every budget,
   masked decode at 10% and 50% on sampled sequences, 100% = unmasked bitwise.
 """
 import gc
