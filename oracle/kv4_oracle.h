@@ -23,6 +23,23 @@
  * along head_dim with an fp16 scale; per-token INT8 with an fp16 scale;
  * scale rounded toward +inf; codes rounded to nearest-even) are this project's
  * stated readings.
+ *
+ * What pins each function to something other than itself (tests/test_oracle_*):
+ *  fp16 round-up, RNE, fp16/bf16 decoders: exact rational arithmetic over every
+ *    positive finite bf16 maximum (both divisors), numpy's fp16 decoder.
+ *  kv4o_quant_int4/int8: brute force over all codes with ties to even;
+ *    |x - c s| <= s/2; re-quantising c s returns c; overflow flag.
+ *  byte layout and kv4o_write_cache: hand-computed offsets, bijection of every
+ *    layout, the written image read back through the fragment view.
+ *  kv4o_attend_rows, kv4o_merge, kv4o_decode: closed forms (equal scores,
+ *    zero query, one dominant key, two keys), merge of random chunkings equal
+ *    to one softmax, decode equal to the merge of its INT4 and INT8 partials,
+ *    contexts of at most 144 positions independent of the INT4 codes, GQA
+ *    head mapping, full / empty / subset masks.
+ *  kv4o_topk: subset enumeration on short rows, nested budgets, the forced
+ *    set, budget counts from the floor rule, -0 equal to +0.
+ * Parity unpinned: the size of the error that INT8 protection removes relative
+ * to unquantised attention (reported, only its direction is checked).
  */
 #ifndef KV4_ORACLE_H
 #define KV4_ORACLE_H
