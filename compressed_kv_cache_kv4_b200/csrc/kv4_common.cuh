@@ -118,19 +118,11 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "r"(addr));
 }
 
-// Two signed 4-bit codes at bits 0-3 and 16-19 of w -> bf16x2 of the codes.
+// Two signed 4-bit codes at bits 0-3 and 16-19 of w -> bf16x2 of 136 + c.
 // LOP3 computes (w & 0x000F000F) ^ 0x43084308: flipping bit 3 turns the
 // two's-complement nibble c into c + 8, and 0x43 above it makes the bf16
-// value 128 + (c + 8). Subtracting 136 (bf16 0x4308) is exact.
-__device__ __forceinline__ uint32_t i4x2_to_bf16x2(uint32_t w) {
-  uint32_t t, d;
-  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x000F000Fu), "r"(0x43084308u));
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(t), "r"(0x43084308u));
-  return d;
-}
-
-// Same LOP3 without the subtraction: bf16x2 of 136 + c (the offset is removed
-// elsewhere, e.g. through the MMA accumulator's initial value).
+// value 128 + (c + 8). The offset 136 is removed elsewhere (through the MMA
+// accumulator's initial value).
 __device__ __forceinline__ uint32_t i4x2_biased(uint32_t w) {
   uint32_t t;
   asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(t) : "r"(w), "r"(0x000F000Fu), "r"(0x43084308u));
