@@ -75,6 +75,9 @@ def lib():
         L.kv4o_topk.restype = None
         L.kv4o_topk.argtypes = [P, C.c_int64, P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                 P, C.c_int, P]
+        L.kv4o_evict_pages.restype = None
+        L.kv4o_evict_pages.argtypes = [P, C.c_int64, P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                       C.c_int, P, C.c_int, P, P, P]
         _lib = L
     return _lib
 
@@ -252,3 +255,24 @@ def topk(scores, lens, permille, sink=16, recent=128):
     count = np.zeros((B, Hkv), np.int32)
     lib().kv4o_topk(_p(s), stride, _p(lens), B, Hkv, permille, sink, recent, _p(mask), mstride, _p(count))
     return mask, count
+
+
+# ---------------------------------------------------------------- page eviction
+def evict_pages(scores, lens, page_table, side, D, permille, sink=16, recent=128):
+    """Page-granular eviction and compaction on copies of the inputs.
+    scores: float32 [B][Hkv][stride]; lens int32 [B]; page_table int32 [B][pt_stride];
+    side: uint8 side-cache image (or None to skip the ring rotation check).
+    -> (lens, page_table, freed [B][pt_stride] (-1 past the count), freed_count, side)."""
+    s = _c(scores, np.float32)
+    B, Hkv, stride = s.shape
+    lens = np.array(lens, np.int32, copy=True)
+    pt = np.array(page_table, np.int32, copy=True)
+    freed = np.full(pt.shape, -1, np.int32)
+    cnt = np.zeros(B, np.int32)
+    if side is None:
+        side = np.zeros(B * Hkv * side_head_bytes(D, sink, recent), np.uint8)
+    side = np.array(side, np.uint8, copy=True)
+    assert np.all(lens <= stride) and np.all(lens <= 16 * pt.shape[1])
+    lib().kv4o_evict_pages(_p(s), stride, _p(lens), B, Hkv, D, permille, sink, recent, _p(pt),
+                           pt.shape[1], _p(freed), _p(cnt), _p(side))
+    return lens, pt, freed, cnt, side

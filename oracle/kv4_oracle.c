@@ -444,3 +444,85 @@ void kv4o_topk(const float *scores, int64_t score_stride, const int32_t *lens, i
     }
   }
 }
+
+/* ------------------------------------------------------------------ */
+/* Page-granular eviction and compaction.                              */
+/* [KVP] engineering-limitations section, third item (vLLM block       */
+/* granularity): a paged cache evicts whole 16-position blocks, ranked  */
+/* by the mean of their positions' scores. [KVS] method details (core   */
+/* idea): the compacted cache keeps streaming -- later appends go on    */
+/* into the surviving pages, nothing is flushed or re-prefilled.        */
+/* ------------------------------------------------------------------ */
+
+void kv4o_evict_pages(const float *scores, int64_t score_stride, int32_t *lens, int B, int Hkv, int D,
+                      int permille, int sink, int recent, int32_t *page_table, int pt_stride,
+                      int32_t *freed, int32_t *freed_count, uint8_t *side) {
+  const int64_t side_stride = kv4o_side_head_bytes(D, sink, recent);
+  const int64_t spb = kv4o_side_page_bytes(D);
+  const int ring_pages = recent / PAGE_TOKENS, ring0 = sink > 0 ? 1 : 0;
+  for (int b = 0; b < B; ++b) {
+    const int L = lens[b];
+    const int n = (L + PAGE_TOKENS - 1) / PAGE_TOKENS;
+    int32_t *row = page_table + (int64_t)b * pt_stride;
+    /* Candidates: full pages that hold no position of the INT8 set. */
+    cand_t *c = (cand_t *)malloc(sizeof(cand_t) * (size_t)(n > 0 ? n : 1));
+    char *evict = (char *)calloc((size_t)(n > 0 ? n : 1), 1);
+    int nc = 0;
+    for (int j = 0; j < n; ++j) {
+      int cand = (j + 1) * PAGE_TOKENS <= L;
+      for (int p = j * PAGE_TOKENS; cand && p < (j + 1) * PAGE_TOKENS; ++p)
+        if (is_protected(p, L, sink, recent)) cand = 0;
+      if (!cand) continue;
+      /* The page's score: its 16 * Hkv position scores added in fp64, head by
+       * head and slot by slot. Every candidate holds the same number of
+       * scores, so this sum orders pages as their mean does. */
+      double s = 0.0;
+      for (int h = 0; h < Hkv; ++h)
+        for (int r = 0; r < PAGE_TOKENS; ++r)
+          s += (double)scores[((int64_t)b * Hkv + h) * score_stride + (int64_t)j * PAGE_TOKENS + r];
+      c[nc].score = s;
+      c[nc].idx = j;
+      ++nc;
+    }
+    const int64_t kbud = (int64_t)n * permille / 1000;
+    int64_t take = kbud - (n - nc);
+    if (take < 0) take = 0;
+    if (take > nc) take = nc;
+    qsort(c, (size_t)nc, sizeof(cand_t), cand_cmp);
+    for (int i = (int)take; i < nc; ++i) evict[c[i].idx] = 1;
+    const int e = nc - (int)take;
+
+    /* Page table: surviving pages in order, then the entries past the last
+     * logical page (mapped ahead for later appends), then -1 for the freed
+     * tail. Evicted ids go to the free list in logical order. */
+    int32_t *old = (int32_t *)malloc(sizeof(int32_t) * (size_t)pt_stride);
+    memcpy(old, row, sizeof(int32_t) * (size_t)pt_stride);
+    int w = 0, f = 0;
+    for (int j = 0; j < pt_stride; ++j) {
+      if (j < n && evict[j]) freed[(int64_t)b * pt_stride + f++] = old[j];
+      else row[w++] = old[j];
+    }
+    while (w < pt_stride) row[w++] = -1;
+    freed_count[b] = e;
+    lens[b] = L - PAGE_TOKENS * e;
+
+    /* Positions after an evicted page move down by 16 each, so position p of
+     * the recent window becomes p - 16e and its ring slot (p - 16e) mod
+     * recent: ring page q moves to ring page (q - e) mod (recent / 16). */
+    if (ring_pages > 0 && e % ring_pages != 0) {
+      uint8_t *tmp = (uint8_t *)malloc((size_t)(ring_pages * spb));
+      for (int h = 0; h < Hkv; ++h) {
+        uint8_t *ring = side + ((int64_t)b * Hkv + h) * side_stride + ring0 * spb;
+        memcpy(tmp, ring, (size_t)(ring_pages * spb));
+        for (int q = 0; q < ring_pages; ++q) {
+          const int dst = ((q - e) % ring_pages + ring_pages) % ring_pages;
+          memcpy(ring + dst * spb, tmp + q * spb, (size_t)spb);
+        }
+      }
+      free(tmp);
+    }
+    free(old);
+    free(evict);
+    free(c);
+  }
+}

@@ -18,7 +18,12 @@
  *           index set is recorded as a binary mask and applied inside attention.
  *  [KVP]    promo of arXiv 2602.10238 ("learning to evict"), core-mechanism
  *           section: score every token, rank, truncate at a 10%..90% budget,
- *           one ranking per attention head.
+ *           one ranking per attention head; engineering-limitations section,
+ *           third item: in a paged (vLLM-style, 16-position block) cache the
+ *           ranking is taken per block, on the mean of its positions' scores.
+ *  [KVS]    "KV-streams for Efficient Compaction in Agentic Reinforcement
+ *           Learning" (summary page), method details, core idea: after a
+ *           compaction the cache keeps streaming instead of being flushed.
  * Quantiser details the pages leave open (symmetric INT4 per 32-element group
  * along head_dim with an fp16 scale; per-token INT8 with an fp16 scale;
  * scale rounded toward +inf; codes rounded to nearest-even) are this project's
@@ -38,6 +43,10 @@
  *    head mapping, full / empty / subset masks.
  *  kv4o_topk: subset enumeration on short rows, nested budgets, the forced
  *    set, budget counts from the floor rule, -0 equal to +0.
+ *  kv4o_evict_pages: pairwise order check of kept against evicted pages on
+ *    scores whose page sums are exact, hand-worked tables and free lists,
+ *    decode of the compacted cache equal to masked decode of the original,
+ *    the compacted side image equal to re-appending the surviving positions.
  * Parity unpinned: the size of the error that INT8 protection removes relative
  * to unquantised attention (reported, only its direction is checked).
  */
@@ -124,6 +133,23 @@ void kv4o_merge(int D, int C, const double *m, const double *l, const double *o,
  * best other positions by (score descending, index ascending). */
 void kv4o_topk(const float *scores, int64_t score_stride, const int32_t *lens, int B, int Hkv,
                int permille, int sink, int recent, uint32_t *mask, int mask_stride, int32_t *count);
+
+/* ---- page-granular eviction and compaction ([KVP], [KVS]) ----
+ * Per sequence b with L = lens[b] and n = ceil(L/16) logical pages.
+ * Candidates: full pages (16 positions < L) none of whose positions is in the
+ * INT8 set (p < sink or p >= L - recent); every other page is kept. Page score:
+ * the fp64 sum of its 16 * Hkv scores in (head, slot) order. k = floor(n *
+ * permille / 1000); the max(0, k - (n - candidates)) best candidates (score
+ * descending, index ascending) are kept, the other e are evicted. Then:
+ * lens[b] -= 16 e; page_table row b = surviving entries in order, then entries
+ * [n, pt_stride), then e times -1; freed[b][0..e) = evicted ids in logical
+ * order (freed is [B][pt_stride]); freed_count[b] = e; in the side cache ring
+ * page q of every (b, h) moves to ring page (q - e) mod (recent / 16).
+ * scores: [B][Hkv][score_stride]; requires lens[b] <= score_stride and
+ * lens[b] <= 16 * pt_stride. */
+void kv4o_evict_pages(const float *scores, int64_t score_stride, int32_t *lens, int B, int Hkv, int D,
+                      int permille, int sink, int recent, int32_t *page_table, int pt_stride,
+                      int32_t *freed, int32_t *freed_count, uint8_t *side);
 
 #ifdef __cplusplus
 }
