@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--workload", default="qwen8b", choices=["qwen8b", "async", "long", "evict", "tiny"])
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--page-evict-only", action="store_true",
+                    help="time only kv4_evict_pages on the eviction workload and print its figures")
     ap.add_argument("--sink", type=int, default=None, help="override the INT8 sink size (0 = pure INT4)")
     ap.add_argument("--recent", type=int, default=None, help="override the INT8 recent window")
     return ap.parse_args()
@@ -501,7 +503,7 @@ def secondary(wl, L0, cache, ptd, pt_np, npages, kpre, vpre, offpre, lens_pre, s
     return out
 
 
-def evict_secondary(steps=50):
+def evict_secondary(steps=50, page_only=False):
     import compressed_kv_cache_kv4_b200 as K
     from compressed_kv_cache_kv4_b200 import synth
     wl = synth.workload("evict")
@@ -512,6 +514,12 @@ def evict_secondary(steps=50):
     q = synth.gen_q(wl, device="cuda")
     lens = torch.as_tensor(wl.lens, device="cuda")
     L = int(wl.lens.max())
+    if page_only:
+        o = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
+        res = {"page_evict": page_evict_secondary(wl, cache, scores, lens, ptd, q, o, cache.workspace(wl.B, wl.Hq))}
+        res["device_error"] = cache.get_error()[1]
+        cache.close()
+        return res
     mstride = (ptd.shape[1] * 16 + 31) // 32
     mask = torch.zeros((wl.B, wl.Hkv, mstride), dtype=torch.int32, device="cuda")
     count = torch.zeros((wl.B, wl.Hkv), dtype=torch.int32, device="cuda")
@@ -529,10 +537,77 @@ def evict_secondary(steps=50):
     call, kern = time_calls(lambda: K.kv4_decode_attn(cache.handle, q, lens, ptd, wl.softmax_scale, wsb, o), steps,
                             kind=0)
     res["unmasked_decode_us"] = call * 1e3
+    res["page_evict"] = page_evict_secondary(wl, cache, scores, lens, ptd, q, o, wsb)
     st, bits = cache.get_error()
     res["device_error"] = bits
     cache.close()
     return res
+
+
+def page_evict_bytes(wl, lens, pt_stride, permille, nring):
+    """Algorithmic bytes of one kv4_evict_pages launch: the candidate pages'
+    scores, the page-table row read and written, the free list and lengths,
+    and the ring pages of every head read and written when they rotate."""
+    total = 0
+    for L in np.asarray(lens, np.int64):
+        n = (L + 15) // 16
+        jlo = 1 if wl.sink > 0 else 0
+        nc = max(0, max(jlo, (L - wl.recent) // 16) - jlo)
+        ksel = min(max(n * permille // 1000 - (n - nc), 0), nc)
+        e = nc - ksel
+        total += 8 + 4
+        if e == 0:
+            continue
+        n, nc, ksel, e = int(n), int(nc), int(ksel), int(e)
+        total += (nc * 16 * wl.Hkv * 4 if ksel > 0 else 0) + 2 * pt_stride * 4 + e * 4
+        if nring and e % nring:
+            total += 2 * wl.Hkv * nring * (32 * wl.D + 64)
+    return total
+
+
+def page_evict_secondary(wl, cache, scores, lens, ptd, q, o, wsb, reps=20):
+    """kv4_evict_pages on the eviction workload: each launch timed alone with
+    CUDA events, after the cache state is restored and L2 is flushed by a read
+    of 256 MB (the inputs fit in L2), with a spin on the stream ahead of the start event so
+    that host-side launch work is not timed; then decode on the compacted
+    cache."""
+    import compressed_kv_cache_kv4_b200 as K
+    peak, _ = peaks()
+    lens0, pt0, side0 = lens.clone(), ptd.clone(), cache.side.clone()
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device="cuda")
+    freed = torch.empty_like(ptd)
+    cnt = torch.empty_like(lens)
+    stream = torch.cuda.current_stream()
+    nring = wl.recent // 16
+    out = {}
+    for permille in (100, 500):
+        ms = []
+        for r in range(reps + 3):
+            lens.copy_(lens0)
+            ptd.copy_(pt0)
+            cache.side.copy_(side0)
+            flush.max()                  # reads 256 MB: L2 holds clean flush lines only
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(100000)   # keeps the GPU busy until the launch below is queued
+            e0.record(stream)
+            K.kv4_evict_pages(cache.handle, scores, permille, lens, ptd, freed, cnt)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if r >= 3:
+                ms.append(e0.elapsed_time(e1))
+        t = float(np.mean(ms))
+        nbytes = int(page_evict_bytes(wl, wl.lens, ptd.shape[1], permille, nring))
+        kept = int(lens.sum().item())
+        call, _ = time_calls(lambda: K.kv4_decode_attn(cache.handle, q, lens, ptd, wl.softmax_scale, wsb, o), 20)
+        out["%d" % permille] = {"us": t * 1e3, "gbs": nbytes / (t / 1e3) / 1e9,
+                                "frac_of_peak": nbytes / (t / 1e3) / 1e9 / peak,
+                                "algorithmic_bytes": nbytes, "pages_freed": int(cnt.sum().item()),
+                                "positions_after": kept, "decode_after_us": call * 1e3}
+    lens.copy_(lens0)
+    ptd.copy_(pt0)
+    cache.side.copy_(side0)
+    del flush
+    return out
 
 
 # ---------------------------------------------------------------------------- CPU oracle
@@ -658,6 +733,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, ws, rank)
+        return
+    if args.page_evict_only:
+        if rank == 0:
+            print(json.dumps(evict_secondary(page_only=True)), flush=True)
         return
     wl, res = run_kv4(args, ws, rank)
     if rank == 0:

@@ -7,8 +7,8 @@ been built, importing the compute entry points raises ImportError; there is no
 fallback implementation.
 
 Names mirror the C ABI (kv4_cache_bytes, kv4_cache_create, kv4_append,
-kv4_workspace_bytes, kv4_decode_attn, kv_topk_retain, bf16_paged_decode_attn,
-kv4_get_error); ``KV4Cache`` bundles the buffers and handle of one cache.
+kv4_workspace_bytes, kv4_decode_attn, kv_topk_retain, kv4_evict_pages,
+bf16_paged_decode_attn, kv4_get_error); ``KV4Cache`` bundles the buffers and handle of one cache.
 """
 import ctypes as C
 import os
@@ -62,6 +62,7 @@ def lib():
         "kv4_decode_attn_noalloc": (C.c_int, [_P, _P, _P, _I32, _P, _P, _I32, _P, _I32, C.c_float, _I32,
                                               _P, _I32, _I32]),
         "kv_topk_retain": (C.c_int, [_P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P, _I32, _P, _I32]),
+        "kv4_evict_pages": (C.c_int, [_P, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P, _I32]),
         "bf16_paged_workspace_bytes": (C.c_int, [_I32, _I32, _I32, _I32, _I32, C.POINTER(_SZ)]),
         "bf16_paged_decode_attn": (C.c_int, [_P, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _P, C.c_float,
                                              _I32, _P, _SZ, _P, _I32, _I32, _P]),
@@ -179,6 +180,17 @@ def kv_topk_retain(scores, seq_lens, budget_permille, mask_out, count_out=None, 
     _check(st, "kv_topk_retain")
 
 
+def kv4_evict_pages(handle, scores, budget_permille, seq_lens, page_table, freed_pages, freed_count,
+                    stream=None):
+    """Page-granular eviction and compaction: rewrites seq_lens, page_table and
+    the side cache's ring pages in place; freed_pages[b, :freed_count[b]] get the
+    evicted physical page ids."""
+    B, _, stride = scores.shape
+    st = lib().kv4_evict_pages(handle, _stream(stream), _ptr(scores), stride, budget_permille, _ptr(seq_lens),
+                               _ptr(page_table), page_table.shape[1], _ptr(freed_pages), _ptr(freed_count), B)
+    _check(st, "kv4_evict_pages")
+
+
 def bf16_paged_workspace_bytes(B, Hq, Hkv, D, num_workers=0):
     n = _SZ(0)
     _check(lib().bf16_paged_workspace_bytes(B, Hq, Hkv, D, num_workers, C.byref(n)), "bf16_paged_workspace_bytes")
@@ -275,6 +287,14 @@ class KV4Cache:
         kv4_decode_attn(self.handle, q, seq_lens, page_table, softmax_scale, ws, out, retain_mask,
                         num_workers, stream)
         return out
+
+    def evict_pages(self, scores, budget_permille, seq_lens, page_table, stream=None):
+        """Evict whole pages in place; returns (freed_pages [B][pt_stride], freed_count [B])."""
+        B = seq_lens.shape[0]
+        freed = torch.full((B, page_table.shape[1]), -1, dtype=torch.int32, device=page_table.device)
+        count = torch.zeros(B, dtype=torch.int32, device=page_table.device)
+        kv4_evict_pages(self.handle, scores, budget_permille, seq_lens, page_table, freed, count, stream)
+        return freed, count
 
     def get_error(self, stream=None):
         return kv4_get_error(self.handle, stream)

@@ -405,6 +405,38 @@ kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32
   return cuda_status(launch_decode(p, D, true, static_cast<cudaStream_t>(stream), e0, e1));
 }
 
+kv4_status kv4_evict_pages(kv4_cache *cache, void *stream, const float *scores, int64_t score_stride,
+                           int32_t budget_permille, int32_t *seq_lens, int32_t *page_table, int32_t pt_stride,
+                           int32_t *freed_pages, int32_t *freed_count, int32_t B) {
+  if (!cache) return KV4_ERR_INVALID;
+  if (B < 0 || pt_stride < 1 || score_stride < 0) return KV4_ERR_INVALID;
+  if (budget_permille < 0 || budget_permille > 1000) return KV4_ERR_INVALID;
+  if (B == 0) return KV4_OK;
+  if (B > cache->cfg.max_seqs) return KV4_ERR_CAPACITY;
+  if (!scores || !seq_lens || !page_table || !freed_pages || !freed_count) return KV4_ERR_INVALID;
+  if (!aligned(scores, 4)) return KV4_ERR_INVALID;
+  if (pt_stride > kEvictMaxPages) return KV4_ERR_UNSUPPORTED;
+  EvictParams p{};
+  p.scores = scores;
+  p.score_stride = score_stride;
+  p.seq_lens = seq_lens;
+  p.page_table = page_table;
+  p.freed = freed_pages;
+  p.freed_count = freed_count;
+  p.pt_stride = pt_stride;
+  p.B = B;
+  p.Hkv = cache->cfg.num_kv_heads;
+  p.permille = budget_permille;
+  p.sink = cache->cfg.sink;
+  p.recent = cache->cfg.recent;
+  p.side = cache->side;
+  p.side_stride = side_head_bytes(cache->cfg.head_dim, p.sink, p.recent);
+  p.side_page_bytes = 32LL * cache->cfg.head_dim + 64;
+  p.err = cache->err;
+  const bool vec = aligned(scores, 16) && score_stride % 4 == 0;
+  return cuda_status(launch_evict(p, vec, static_cast<cudaStream_t>(stream)));
+}
+
 kv4_status kv4_get_error(kv4_cache *cache, void *stream, uint32_t *bits) {
   if (!cache) return KV4_ERR_INVALID;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

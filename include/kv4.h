@@ -179,6 +179,42 @@ kv4_status kv_topk_retain(void *stream, const float *scores, int64_t score_strid
                           int32_t *count_out, int32_t max_len);
 
 /*
+ * kv4_evict_pages -- page-granular eviction and compaction of the cache.
+ * [KVP] engineering-limitations section, third item: in a paged cache of
+ * 16-position blocks the ranking applies per block, on the mean of the block's
+ * position scores, and whole blocks leave. "KV-streams for Efficient
+ * Compaction in Agentic Reinforcement Learning" (summary page), method
+ * details, core idea: the compacted cache keeps streaming; appends continue in
+ * the surviving pages.
+ *  scores: device fp32 [B][Hkv][score_stride] (4-byte aligned), one score per
+ *    position, as for kv_topk_retain; positions [0, L) of each row are read.
+ *  budget_permille: 0..1000.
+ *  seq_lens: device int32 [B], read and rewritten (L - 16 e).
+ *  page_table: device int32 [B][pt_stride], pt_stride <= 16384, read and
+ *    rewritten in place.
+ *  freed_pages: device int32 [B][pt_stride]; entries 0..e-1 of row b receive
+ *    the evicted physical page ids in logical order, later entries are not
+ *    touched. freed_count: device int32 [B], receives e.
+ * Per sequence with L positions in n = ceil(L/16) pages: the candidates are
+ * the full pages holding no position of the INT8 set (p < sink or p >= L -
+ * recent); all other pages stay. A candidate's score is the fp64 sum of its
+ * 16 * Hkv scores taken head by head, slot by slot (the same order as its
+ * mean). k = floor(n * budget_permille / 1000) pages stay: the non-candidates
+ * and the max(0, k - non-candidates) best candidates (score descending, then
+ * lower page index); the other e are evicted. The row becomes the surviving
+ * entries in order, then the entries past logical page n - 1 (mapped ahead for
+ * later appends), then e times -1. Positions after an evicted page move down
+ * 16 each; the recent window moves down 16 e, and the INT8 ring pages of each
+ * (sequence, head) in the side cache are rotated to match. The INT4 pages are
+ * not touched; the freed ids belong to the caller's allocator. A length below
+ * 0, above 16 * pt_stride or above score_stride sets KV4_ERR_CAPACITY and
+ * leaves that sequence unchanged (freed_count 0). Scores must not be NaN.
+ */
+kv4_status kv4_evict_pages(kv4_cache *cache, void *stream, const float *scores, int64_t score_stride,
+                           int32_t budget_permille, int32_t *seq_lens, int32_t *page_table, int32_t pt_stride,
+                           int32_t *freed_pages, int32_t *freed_count, int32_t B);
+
+/*
  * bf16_paged_workspace_bytes / bf16_paged_decode_attn -- the uncompressed
  * comparison ([KV4RL] sec. 3 compares against BF16 rollouts): the same decode
  * attention over bf16 pages. One page holds 16 positions of every KV head: per

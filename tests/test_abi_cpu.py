@@ -57,6 +57,7 @@ def test_host_validation_without_launch():
     n = C.c_size_t(0)
     assert L.bf16_paged_workspace_bytes(4, 12, 4, 128, 0, C.byref(n)) == K.KV4_ERR_UNSUPPORTED   # G = 3
     assert L.bf16_paged_workspace_bytes(4, 8, 4, 96, 0, C.byref(n)) == K.KV4_ERR_UNSUPPORTED     # D = 96
+    assert L.kv4_evict_pages(None, None, fake, 100, 500, fake, fake, 8, fake, fake, 1) == K.KV4_ERR_INVALID
     assert L.kv4_get_error(None, None, None) == K.KV4_ERR_INVALID
     assert L.kv4_debug_set_wait_limit(None, 0) == K.KV4_ERR_INVALID
 
