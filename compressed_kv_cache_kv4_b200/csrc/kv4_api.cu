@@ -13,6 +13,7 @@
 #include "../../include/kv4.h"
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
+#include "kv4_evict.h"
 
 using namespace kv4;
 

@@ -42,6 +42,7 @@
 
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
+#include "kv4_evict.h"
 
 namespace cg = cooperative_groups;
 

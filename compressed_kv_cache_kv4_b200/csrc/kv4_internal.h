@@ -52,25 +52,6 @@ struct TopkParams {
   int32_t *count;
 };
 
-struct EvictParams {
-  const float *scores;          // [B][Hkv][score_stride]
-  long long score_stride;
-  int32_t *seq_lens;            // [B], rewritten
-  int32_t *page_table;          // [B][pt_stride], rewritten
-  int32_t *freed;               // [B][pt_stride], evicted ids first
-  int32_t *freed_count;         // [B]
-  int pt_stride, B, Hkv, permille, sink, recent;
-  uint8_t *side;                // INT8 side blocks, ring pages rotated in place
-  long long side_stride, side_page_bytes;
-  uint32_t *err;
-};
-
-// Ring pages per (sequence, head) at most (recent <= 128).
-constexpr int kMaxRingPages = 8;
-// Longest page-table row kv4_evict_pages accepts (its keys and the staged row
-// live in shared memory).
-constexpr int kEvictMaxPages = 16384;
-
 // Largest batch kv4_decode_attn accepts (the per-CTA plan lives in shared memory).
 constexpr int kMaxBatch = 8192;
 
@@ -104,8 +85,6 @@ int decode_smem_bytes(int D, bool bf16, int B);
 cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t stream, cudaEvent_t ev0,
                           cudaEvent_t ev1);
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream);
-size_t evict_smem_bytes(int pt_stride);
-cudaError_t launch_evict(const EvictParams &p, bool vec, cudaStream_t stream);
 // Exact merge of the decode partials (np8 = INT8 side pages per (sequence, head)).
 cudaError_t launch_merge(const DecodeParams &p, int D, int np8, cudaStream_t stream);
 
