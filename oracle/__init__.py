@@ -78,6 +78,9 @@ def lib():
         L.kv4o_evict_pages.restype = None
         L.kv4o_evict_pages.argtypes = [P, C.c_int64, P, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                        C.c_int, P, C.c_int, P, P, P]
+        L.kv4o_masked_attn.restype = None
+        L.kv4o_masked_attn.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, P, P, P, P, P, C.c_int,
+                                       C.c_float, P]
         _lib = L
     return _lib
 
@@ -276,3 +279,21 @@ def evict_pages(scores, lens, page_table, side, D, permille, sink=16, recent=128
     lib().kv4o_evict_pages(_p(s), stride, _p(lens), B, Hkv, D, permille, sink, recent, _p(pt),
                            pt.shape[1], _p(freed), _p(cnt), _p(side))
     return lens, pt, freed, cnt, side
+
+
+# ---------------------------------------------------------------- learner-side masked attention
+def masked_attn(q_bits, k_bits, v_bits, softmax_scale, lens=None, mask=None):
+    """q_bits uint16 [B][T][Hq][D]; k_bits, v_bits uint16 [B][T][Hkv][D];
+    mask None or uint32 [B][Hkv][T][mask_stride]. -> float64 [B][T][Hq][D]."""
+    q = _c(q_bits, np.uint16)
+    k = _c(k_bits, np.uint16)
+    v = _c(v_bits, np.uint16)
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    ln = None if lens is None else _c(lens, np.int32)
+    m = None if mask is None else _c(mask, np.uint32)
+    ms = 0 if m is None else m.shape[-1]
+    out = np.zeros((B, T, Hq, D), np.float64)
+    lib().kv4o_masked_attn(B, T, Hq, Hkv, D, _p(q), _p(k), _p(v), _p(ln), _p(m), ms,
+                           C.c_float(softmax_scale), _p(out))
+    return out

@@ -526,3 +526,56 @@ void kv4o_evict_pages(const float *scores, int64_t score_stride, int32_t *lens, 
     free(c);
   }
 }
+
+/* ------------------------------------------------------------------ */
+/* Learner-side attention under the recorded shadow mask ([SMD] sec. 1 */
+/* and Figure 1): the rollout records, for the query at each position, */
+/* the set of positions its eviction kept; the learner's causal        */
+/* attention applies exactly that set, over the full-precision (bf16)  */
+/* K and V, so each row reproduces what the rollout attended to.       */
+/* ------------------------------------------------------------------ */
+
+void kv4o_masked_attn(int B, int T, int Hq, int Hkv, int D, const uint16_t *q, const uint16_t *k,
+                      const uint16_t *v, const int32_t *lens, const uint32_t *mask, int mask_stride,
+                      float softmax_scale, double *out) {
+  const int G = Hq / Hkv;
+  const double tau = (double)softmax_scale;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int b = 0; b < B; ++b) {
+    for (int hq = 0; hq < Hq; ++hq) {
+      const int h = hq / G;
+      const int L = lens ? lens[b] : T;
+      double *s = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+      double *qd = (double *)malloc(sizeof(double) * (size_t)D);
+      for (int t = 0; t < T; ++t) {
+        double *o = out + (((int64_t)b * T + t) * Hq + hq) * D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        if (t >= L) continue;
+        for (int d = 0; d < D; ++d) qd[d] = kv4o_bf16_to_double(q[(((int64_t)b * T + t) * Hq + hq) * D + d]);
+        const uint32_t *mrow = mask ? mask + (((int64_t)b * Hkv + h) * T + t) * mask_stride : NULL;
+        /* visible keys: p <= t (causal) whose bit is set in row t */
+        double m = -INFINITY;
+        for (int p = 0; p <= t; ++p) {
+          s[p] = -INFINITY;
+          if (mrow && !((mrow[p / 32] >> (p % 32)) & 1u)) continue;
+          const uint16_t *kr = k + (((int64_t)b * T + p) * Hkv + h) * D;
+          double dot = 0.0;
+          for (int d = 0; d < D; ++d) dot += qd[d] * kv4o_bf16_to_double(kr[d]);
+          s[p] = tau * dot;
+          if (s[p] > m) m = s[p];
+        }
+        double l = 0.0;
+        for (int p = 0; p <= t; ++p) {
+          if (s[p] == -INFINITY) continue;
+          const double w = exp(s[p] - m);
+          const uint16_t *vr = v + (((int64_t)b * T + p) * Hkv + h) * D;
+          l += w;
+          for (int d = 0; d < D; ++d) o[d] += w * kv4o_bf16_to_double(vr[d]);
+        }
+        for (int d = 0; d < D; ++d) o[d] = (l > 0.0) ? o[d] / l : 0.0;
+      }
+      free(s);
+      free(qd);
+    }
+  }
+}

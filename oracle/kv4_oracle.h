@@ -43,6 +43,10 @@
  *    head mapping, full / empty / subset masks.
  *  kv4o_topk: subset enumeration on short rows, nested budgets, the forced
  *    set, budget counts from the floor rule, -0 equal to +0.
+ *  kv4o_masked_attn: torch float64 softmax attention on small cases, closed
+ *    forms (a diagonal-only mask returns v_t, an empty row returns 0), and
+ *    row t equal to kv4o_decode over bf16 values at length t + 1 under mask
+ *    row t (the learner reproduces the rollout's attention).
  *  kv4o_evict_pages: pairwise order check of kept against evicted pages on
  *    scores whose page sums are exact, hand-worked tables and free lists,
  *    decode of the compacted cache equal to masked decode of the original,
@@ -150,6 +154,17 @@ void kv4o_topk(const float *scores, int64_t score_stride, const int32_t *lens, i
 void kv4o_evict_pages(const float *scores, int64_t score_stride, int32_t *lens, int B, int Hkv, int D,
                       int permille, int sink, int recent, int32_t *page_table, int pt_stride,
                       int32_t *freed, int32_t *freed_count, uint8_t *side);
+
+/* ---- learner-side attention under the shadow mask ([SMD] sec. 1, Figure 1) ----
+ * q: bf16 bits [B][T][Hq][D]; k, v: bf16 bits [B][T][Hkv][D]; lens: NULL or [B]
+ * (positions >= lens[b] give 0 and are never attended). mask: NULL (dense
+ * causal) or bits [B][Hkv][T][mask_stride]: row t of KV head h lists the
+ * positions the rollout kept for the query at position t. Query t of head hq
+ * (KV head hq / (Hq/Hkv)) attends to {p <= t : bit p of row t set} over the bf16
+ * values; an empty set gives 0. out: [B][T][Hq][D]. */
+void kv4o_masked_attn(int B, int T, int Hq, int Hkv, int D, const uint16_t *q, const uint16_t *k,
+                      const uint16_t *v, const int32_t *lens, const uint32_t *mask, int mask_stride,
+                      float softmax_scale, double *out);
 
 #ifdef __cplusplus
 }
