@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--page-evict-only", action="store_true",
                     help="time only kv4_evict_pages on the eviction workload and print its figures")
+    ap.add_argument("--learner-only", action="store_true",
+                    help="time only smd_masked_attn on the learner workload and print its figures")
     ap.add_argument("--sink", type=int, default=None, help="override the INT8 sink size (0 = pure INT4)")
     ap.add_argument("--recent", type=int, default=None, help="override the INT8 recent window")
     return ap.parse_args()
@@ -500,6 +502,8 @@ def secondary(wl, L0, cache, ptd, pt_np, npages, kpre, vpre, offpre, lens_pre, s
 
     # eviction workload: top-k (per KV head) + masked decode at 10/30/50/90/100%
     out["evict"] = evict_secondary()
+    # learner-side attention under the recorded shadow mask
+    out["smd_learner"] = learner_secondary()
     return out
 
 
@@ -608,6 +612,53 @@ def page_evict_secondary(wl, cache, scores, lens, ptd, q, o, wsb, reps=20):
     cache.side.copy_(side0)
     del flush
     return out
+
+
+def bf16_peak():
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+    except Exception:
+        return 1590.0, "fallback (1.59 PFLOP/s, earlier measurement on this pool)"
+
+
+def mask_popcount(mask):
+    """Set bits of an int32 mask tensor (on its device)."""
+    x = mask.to(torch.int64) & 0xFFFFFFFF
+    x = x - ((x >> 1) & 0x55555555)
+    x = (x & 0x33333333) + ((x >> 2) & 0x33333333)
+    x = (x + (x >> 4)) & 0x0F0F0F0F
+    return int((((x * 0x01010101) & 0xFFFFFFFF) >> 24).sum().item())
+
+
+def learner_secondary(steps=20):
+    """smd_masked_attn on the learner workload (4 sequences x 8192 positions,
+    32/8 heads, D = 128, the recorded-eviction mask, ~46% of keys kept).
+    Inputs (q 268 MB, K/V 134 MB, mask 134 MB) exceed L2."""
+    import compressed_kv_cache_kv4_b200 as K
+    from compressed_kv_cache_kv4_b200 import synth
+    wl = synth.workload("learner")
+    T = int(wl.lens.max())
+    q, k, v = synth.gen_learner_qkv(wl, T, device="cuda")
+    mask = synth.gen_shadow_mask(wl, T, device="cuda")
+    out = torch.empty((wl.B, T, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
+    peak, peak_src = bf16_peak()
+    res = {}
+    for name, m in (("shadow_mask", mask), ("dense_causal", None)):
+        call, _ = time_calls(lambda: K.smd_masked_attn(q, k, v, wl.softmax_scale, out, mask=m), steps)
+        pairs = mask_popcount(mask) if m is not None else wl.B * wl.Hkv * T * (T + 1) // 2
+        dense_pairs = wl.B * wl.Hkv * T * (T + 1) // 2
+        flops = 4.0 * wl.D * wl.G * pairs                 # q.k and p.v per visible (query, key) pair
+        dense_flops = 4.0 * wl.D * wl.G * dense_pairs     # what the kernel computes (no block is empty)
+        res[name] = {"ms": call, "visible_pairs": pairs, "tflops_algorithmic": flops / (call / 1e3) / 1e12,
+                     "tflops_dense_causal": dense_flops / (call / 1e3) / 1e12,
+                     "frac_of_bf16_peak": dense_flops / (call / 1e3) / 1e12 / peak,
+                     "tokens_per_s": wl.B * T / (call / 1e3)}
+    res["peak_tflops"] = peak
+    res["peak_source"] = peak_src
+    del q, k, v, mask, out
+    torch.cuda.empty_cache()
+    return res
 
 
 # ---------------------------------------------------------------------------- CPU oracle
@@ -737,6 +788,10 @@ def main():
     if args.page_evict_only:
         if rank == 0:
             print(json.dumps(evict_secondary(page_only=True)), flush=True)
+        return
+    if args.learner_only:
+        if rank == 0:
+            print(json.dumps(learner_secondary()), flush=True)
         return
     wl, res = run_kv4(args, ws, rank)
     if rank == 0:

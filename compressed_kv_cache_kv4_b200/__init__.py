@@ -8,7 +8,7 @@ fallback implementation.
 
 Names mirror the C ABI (kv4_cache_bytes, kv4_cache_create, kv4_append,
 kv4_workspace_bytes, kv4_decode_attn, kv_topk_retain, kv4_evict_pages,
-bf16_paged_decode_attn, kv4_get_error); ``KV4Cache`` bundles the buffers and handle of one cache.
+smd_masked_attn, bf16_paged_decode_attn, kv4_get_error); ``KV4Cache`` bundles the buffers and handle of one cache.
 """
 import ctypes as C
 import os
@@ -63,6 +63,8 @@ def lib():
                                               _P, _I32, _I32]),
         "kv_topk_retain": (C.c_int, [_P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P, _I32, _P, _I32]),
         "kv4_evict_pages": (C.c_int, [_P, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P, _I32]),
+        "smd_masked_attn": (C.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P, _I32, C.c_float,
+                                      _P, _I32, _P]),
         "bf16_paged_workspace_bytes": (C.c_int, [_I32, _I32, _I32, _I32, _I32, C.POINTER(_SZ)]),
         "bf16_paged_decode_attn": (C.c_int, [_P, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _P, C.c_float,
                                              _I32, _P, _SZ, _P, _I32, _I32, _P]),
@@ -189,6 +191,18 @@ def kv4_evict_pages(handle, scores, budget_permille, seq_lens, page_table, freed
     st = lib().kv4_evict_pages(handle, _stream(stream), _ptr(scores), stride, budget_permille, _ptr(seq_lens),
                                _ptr(page_table), page_table.shape[1], _ptr(freed_pages), _ptr(freed_count), B)
     _check(st, "kv4_evict_pages")
+
+
+def smd_masked_attn(q, k, v, softmax_scale, out, seq_lens=None, mask=None, error_word=None, stream=None):
+    """Learner-side causal attention under the shadow mask. q [B][T][Hq][D],
+    k/v [B][T][Hkv][D] bf16; mask None or int32/uint32 [B][Hkv][T][mask_stride];
+    out [B][T][Hq][D] bf16 or fp32."""
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    st = lib().smd_masked_attn(_stream(stream), _ptr(q), _ptr(k), _ptr(v), B, T, Hq, Hkv, D, _ptr(seq_lens),
+                               _ptr(mask), 0 if mask is None else mask.shape[-1], C.c_float(softmax_scale),
+                               _ptr(out), 1 if out.dtype == torch.float32 else 0, _ptr(error_word))
+    _check(st, "smd_masked_attn")
 
 
 def bf16_paged_workspace_bytes(B, Hq, Hkv, D, num_workers=0):

@@ -14,6 +14,7 @@
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
 #include "kv4_evict.h"
+#include "smd_attn.h"
 
 using namespace kv4;
 
@@ -436,6 +437,38 @@ kv4_status kv4_evict_pages(kv4_cache *cache, void *stream, const float *scores, 
   p.err = cache->err;
   const bool vec = aligned(scores, 16) && score_stride % 4 == 0;
   return cuda_status(launch_evict(p, vec, static_cast<cudaStream_t>(stream)));
+}
+
+kv4_status smd_masked_attn(void *stream, const void *q, const void *k, const void *v, int32_t B, int32_t T,
+                           int32_t Hq, int32_t Hkv, int32_t D, const int32_t *seq_lens, const uint32_t *mask,
+                           int32_t mask_stride, float softmax_scale, void *out, int32_t out_is_fp32,
+                           uint32_t *error_word) {
+  if (B < 0 || T < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv) return KV4_ERR_INVALID;
+  if (B == 0 || T == 0) return KV4_OK;
+  if (!q || !k || !v || !out) return KV4_ERR_INVALID;
+  const int G = Hq / Hkv;
+  if ((G != 1 && G != 2 && G != 4) || (D != 64 && D != 128)) return KV4_ERR_UNSUPPORTED;
+  if (T > kMaxSmdT || B > 65535 || Hkv > 65535) return KV4_ERR_UNSUPPORTED;
+  if (mask && (long long)mask_stride * 32 < T) return KV4_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return KV4_ERR_INVALID;
+  if (mask && !aligned(mask, 4)) return KV4_ERR_INVALID;
+  SmdParams p{};
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.k = static_cast<const __nv_bfloat16 *>(k);
+  p.v = static_cast<const __nv_bfloat16 *>(v);
+  p.lens = seq_lens;
+  p.mask = mask;
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.mask_stride = mask ? mask_stride : 0;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  p.out_fp32 = out_is_fp32 ? 1 : 0;
+  p.err = error_word;
+  return cuda_status(launch_smd(p, D, static_cast<cudaStream_t>(stream)));
 }
 
 kv4_status kv4_get_error(kv4_cache *cache, void *stream, uint32_t *bits) {

@@ -18,6 +18,10 @@ available; these synthetic shapes stand in for them):
 - ``evict``  B=64, L=16384, same heads; per-position scores are the summed
               softmax attention of 32 random N(0,1) queries at the 32 positions
               before the current one (H2O-style accumulated attention).
+- ``learner`` B=4 sequences of T=8192 positions, same heads, for the
+              learner-side attention under the shadow mask: q, K, V of every
+              position and the mask the rollout's eviction recorded per query
+              position (``gen_shadow_mask``).
 
 Random values depend on the device the generator runs on (torch's CPU and CUDA
 generators differ); every comparison hands the same tensors to both sides.
@@ -91,6 +95,10 @@ def workload(name, **over):
         B = over.pop("B", 4)
         L = over.pop("L", 131072)
         wl = Workload("long", 1004, B, 32, 8, 128, np.full(B, L, np.int32), _f32_inv_sqrt(128))
+    elif name == "learner":
+        B = over.pop("B", 4)
+        T = over.pop("T", 8192)
+        wl = Workload("learner", 1006, B, 32, 8, 128, np.full(B, T, np.int32), _f32_inv_sqrt(128))
     elif name == "evict":
         B = over.pop("B", 64)
         L = over.pop("L", 16384)
@@ -206,3 +214,52 @@ def pad_batch(x, off, seqs, Lmax=None):
 def bf16_bits(t):
     """bf16 tensor -> numpy uint16 bit patterns (CPU)."""
     return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def gen_learner_qkv(wl, T=None, device="cpu"):
+    """Learner inputs for B sequences of T positions: q [B][T][Hq][D], K and V
+    [B][T][Hkv][D] in bf16, N(0,1) with the outlier K channels scaled."""
+    T = int(wl.lens.max()) if T is None else T
+    g = _gen(wl.seed, 7, device)
+    q = torch.randn((wl.B, T, wl.Hq, wl.D), generator=g, device=device, dtype=torch.float32)
+    k = torch.randn((wl.B, T, wl.Hkv, wl.D), generator=g, device=device, dtype=torch.float32)
+    v = torch.randn((wl.B, T, wl.Hkv, wl.D), generator=g, device=device, dtype=torch.float32)
+    gain = torch.ones((wl.Hkv, wl.D), device=device, dtype=torch.float32)
+    for h, chans in enumerate(outlier_channels(wl)):
+        gain[h, torch.as_tensor(chans, device=device)] = wl.outlier_gain
+    k.mul_(gain)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def gen_shadow_mask(wl, T=None, device="cpu", sink=None, recent=None, rows=None):
+    """The mask a rollout's eviction records, int32 [B][Hkv][T][ceil(T/32)]
+    (bit p % 32 of word p / 32 of row t: position p kept at query position t).
+
+    Eviction is monotone: position p of (b, h) stays until step
+    e = p + 1 + floor(2 p u), u ~ U[0, 1), and never returns; the first `sink`
+    and the last `recent` positions are always kept. About 46% of the
+    positions <= t are kept in row t. Bits above t are clear. `rows` limits the
+    output to those query positions (then [B][Hkv][len(rows)][words])."""
+    T = int(wl.lens.max()) if T is None else T
+    sink = wl.sink if sink is None else sink
+    recent = wl.recent if recent is None else recent
+    g = _gen(wl.seed, 8, device)
+    u = torch.rand((wl.B, wl.Hkv, T), generator=g, device=device, dtype=torch.float64)
+    pos = torch.arange(T, device=device, dtype=torch.float64)
+    evict_at = (pos + 1 + torch.floor(2 * pos * u)).to(torch.int64)       # [B][Hkv][T]
+    W = (T + 31) // 32
+    trows = torch.arange(T, device=device) if rows is None else torch.as_tensor(rows, device=device)
+    out = torch.zeros((wl.B, wl.Hkv, len(trows), W), dtype=torch.int32, device=device)
+    shifts = torch.arange(32, device=device, dtype=torch.int64)
+    p = torch.arange(W * 32, device=device)
+    pe = torch.full((wl.B, wl.Hkv, W * 32), -1, dtype=torch.int64, device=device)
+    pe[..., :T] = evict_at
+    chunk = 256
+    for c0 in range(0, len(trows), chunk):
+        t = trows[c0: c0 + chunk].to(torch.int64)[:, None]                    # [c][1]
+        keep = (p[None, :] <= t) & ((p[None, :] < sink) | (p[None, :] >= t - recent + 1)
+                                    | (pe[:, :, None, :] > t))                  # [B][Hkv][c][W*32]
+        keep &= p[None, :] < T
+        words = (keep.view(wl.B, wl.Hkv, -1, W, 32).to(torch.int64) << shifts).sum(-1)
+        out[:, :, c0: c0 + chunk] = (words & 0xFFFFFFFF).to(torch.int32)
+    return out

@@ -215,6 +215,33 @@ kv4_status kv4_evict_pages(kv4_cache *cache, void *stream, const float *scores, 
                            int32_t *freed_pages, int32_t *freed_count, int32_t B);
 
 /*
+ * smd_masked_attn -- learner-side causal attention under the recorded shadow
+ * mask. "How to compress the KV cache in RL post-training? Shadow Mask
+ * Distillation" (arXiv 2605.06850), sec. 1 and Figure 1: the rollout records,
+ * for the query at every position, a binary mask of the positions its KV
+ * eviction kept; the learner applies that mask inside its causal attention so
+ * that each row reproduces what the rollout attended to.
+ *  q: device bf16 [B][T][Hq][D]; k, v: device bf16 [B][T][Hkv][D]; all 16-byte
+ *    aligned. D: 64 or 128; Hq / Hkv: 1, 2 or 4; T <= 65536.
+ *  seq_lens: NULL (every sequence has T positions) or device int32 [B]; rows at
+ *    or past the length are written as 0 and never attended to. A length
+ *    outside [0, T] is clamped and sets KV4_ERR_CAPACITY in *error_word.
+ *  mask: NULL (dense causal attention) or device uint32 [B][Hkv][T][mask_stride]
+ *    (mask_stride >= ceil(T / 32)): bit p % 32 of word p / 32 of row (b, h, t)
+ *    set = the rollout kept position p when it produced the query at position
+ *    t. Bits above t are ignored (causality).
+ *  Query t of head hq (KV head hq / (Hq/Hkv)) attends to {p <= t : bit p of its
+ *    row set} with scores softmax_scale * q.k over the bf16 values; an empty
+ *    set gives 0.
+ *  out: device [B][T][Hq][D], bf16 (out_is_fp32 = 0) or fp32 (1).
+ *  error_word: NULL or a device uint32 receiving status bits (1 << status).
+ */
+kv4_status smd_masked_attn(void *stream, const void *q, const void *k, const void *v, int32_t B, int32_t T,
+                           int32_t Hq, int32_t Hkv, int32_t D, const int32_t *seq_lens, const uint32_t *mask,
+                           int32_t mask_stride, float softmax_scale, void *out, int32_t out_is_fp32,
+                           uint32_t *error_word);
+
+/*
  * bf16_paged_workspace_bytes / bf16_paged_decode_attn -- the uncompressed
  * comparison ([KV4RL] sec. 3 compares against BF16 rollouts): the same decode
  * attention over bf16 pages. One page holds 16 positions of every KV head: per
