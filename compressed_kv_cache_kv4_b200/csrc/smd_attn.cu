@@ -15,7 +15,8 @@
 // per 64-key block; blocks with no retained key for any of its rows are never
 // loaded. Active blocks stream through a two-stage cp.async ring of K and V
 // tiles (rows padded to D + 8 elements so that fragment loads are free of bank
-// conflicts). Per block: S = Q K^T (Q fragments held in registers), masked
+// conflicts). Per block: S = Q K^T (Q fragments held in registers, K fragments
+// by ldmatrix), masked
 // keys and keys after the query set to -inf, online softmax in base 2, then
 // O += P V with P split into bf16 hi + lo parts (two MMAs) so that P keeps
 // 16 significant bits; V fragments come from ldmatrix.trans.
@@ -165,13 +166,17 @@ __global__ void __launch_bounds__(kSmdThreads) smd_attn_kernel(SmdParams p) {
     float s[8][4];
 #pragma unroll
     for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+    // K fragments by ldmatrix: matrices (keys 8n.., d 16st), (8n.., 16st + 8),
+    // (8n + 8.., 16st), (8n + 8.., 16st + 8) give b0, b1 of n-tiles n and n + 1
+    const int kmi = lane >> 3, kri = lane & 7;
 #pragma unroll
     for (int st = 0; st < KS; ++st) {
 #pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        const __nv_bfloat16 *kr = kt + (n * 8 + grp) * PITCH + st * 16 + 2 * tig;
-        mma_bf16(s[n], qa[st], *reinterpret_cast<const uint32_t *>(kr),
-                 *reinterpret_cast<const uint32_t *>(kr + 8));
+      for (int n = 0; n < 8; n += 2) {
+        uint32_t bk[4];
+        ldmatrix_x4(bk, smem_u32(kt + ((n + (kmi >> 1)) * 8 + kri) * PITCH + st * 16 + (kmi & 1) * 8));
+        mma_bf16(s[n], qa[st], bk[0], bk[1]);
+        mma_bf16(s[n + 1], qa[st], bk[2], bk[3]);
       }
     }
 
