@@ -58,6 +58,19 @@ def test_host_validation_without_launch():
     assert L.bf16_paged_workspace_bytes(4, 12, 4, 128, 0, C.byref(n)) == K.KV4_ERR_UNSUPPORTED   # G = 3
     assert L.bf16_paged_workspace_bytes(4, 8, 4, 96, 0, C.byref(n)) == K.KV4_ERR_UNSUPPORTED     # D = 96
     assert L.kv4_evict_pages(None, None, fake, 100, 500, fake, fake, 8, fake, fake, 1) == K.KV4_ERR_INVALID
+    # smd_masked_attn: argument checks before any launch
+    f = C.c_float(0.1)
+    a16 = C.c_void_p(0x10000)
+    args = lambda q=a16, Hq=8, Hkv=2, D=128, mask=None, ms=0, out=a16, T=100: (
+        None, q, a16, a16, 1, T, Hq, Hkv, D, None, mask, ms, f, out, 0, None)
+    assert L.smd_masked_attn(*args(q=None)) == K.KV4_ERR_INVALID            # null q
+    assert L.smd_masked_attn(*args(Hq=6, Hkv=4)) == K.KV4_ERR_INVALID       # Hq % Hkv != 0
+    assert L.smd_masked_attn(*args(Hq=24, Hkv=3)) == K.KV4_ERR_UNSUPPORTED  # G = 8
+    assert L.smd_masked_attn(*args(D=96)) == K.KV4_ERR_UNSUPPORTED          # head_dim
+    assert L.smd_masked_attn(*args(T=70000)) == K.KV4_ERR_UNSUPPORTED       # longer than 65536
+    assert L.smd_masked_attn(*args(mask=fake, ms=3)) == K.KV4_ERR_INVALID   # 3 words < ceil(100/32)
+    assert L.smd_masked_attn(*args(out=C.c_void_p(0x10008))) == K.KV4_ERR_INVALID   # misaligned out
+    assert L.smd_masked_attn(*args(T=0)) == K.KV4_OK                        # nothing to do
     assert L.kv4_get_error(None, None, None) == K.KV4_ERR_INVALID
     assert L.kv4_debug_set_wait_limit(None, 0) == K.KV4_ERR_INVALID
 
