@@ -8,18 +8,24 @@
 // attends to {p <= t : bit p of mask row (h, t)} over the bf16 K and V; an
 // empty set gives 0.
 //
-// Flash-attention style, on mma.sync m16n8k16 bf16 tiles. A CTA of four warps
-// takes one KV head and 16 * 4/G query positions; warp w owns query head
-// g = w % G for positions 16 (w / G) .. +15, so the G heads of a KV head share
-// every K/V tile and every mask row. Before the loop the CTA ORs its mask rows
-// per 64-key block; blocks with no retained key for any of its rows are never
-// loaded. Active blocks stream through a two-stage cp.async ring of K and V
-// tiles (rows padded to D + 8 elements so that fragment loads are free of bank
-// conflicts). Per block: S = Q K^T (Q fragments held in registers, K fragments
-// by ldmatrix), masked
-// keys and keys after the query set to -inf, online softmax in base 2, then
-// O += P V with P split into bf16 hi + lo parts (two MMAs) so that P keeps
-// 16 significant bits; V fragments come from ldmatrix.trans.
+// Flash-attention style on the 5th-generation tensor cores (tcgen05). A CTA
+// of one warpgroup (128 threads) takes one KV head and 128/G query positions:
+// tile row r = g (128/G) + position, so the G query heads of a KV head share
+// every K/V tile and mask row, and thread r owns row r (TMEM lane r) for the
+// whole softmax. Before the loop the CTA ORs its mask rows per 64-key block;
+// blocks with no kept key for any of its rows are never loaded. Per active
+// block: S = Q K^T by tcgen05.mma (Q, K in shared memory, S in 64 TMEM
+// columns); each thread reads its S row (tcgen05.ld), applies the mask bits,
+// causality and the length, and takes the exponentials against its running
+// maximum; P goes to shared memory as bf16 hi + lo parts (P keeps 16
+// significant bits) and O += P V accumulates in TMEM (two MMAs per 16 keys, V
+// as an MN-major operand). O is rescaled in TMEM only when a row's maximum
+// grows by more than 2^8 since it was last used (the exponentials stay below
+// 256, the result is the same softmax). MMAs are issued by one thread and
+// signal an mbarrier through tcgen05.commit; every wait is bounded. K tiles of
+// the next block load (cp.async) while the softmax runs, V tiles while the
+// next S is computed. Operands use the no-swizzle core-matrix layout: 8 rows
+// of 16 bytes per core matrix.
 #include <math.h>
 
 #include "kv4_common.cuh"
@@ -30,9 +36,9 @@ namespace kv4 {
 
 namespace {
 
-constexpr int kSmdWarps = 4;
-constexpr int kSmdThreads = kSmdWarps * 32;
-constexpr int kKeyBlock = 64;
+constexpr int kTcThreads = 128;   // one warpgroup: TMEM lanes 0..127
+constexpr int kTcRows = 128;      // tile rows (M of every MMA)
+constexpr int kKeyBlock = 64;     // keys per block (N of S, K of P V)
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -42,26 +48,92 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, no swizzle: start, leading and stride byte
+// offsets in 16-byte units, descriptor version 1.
+__device__ __forceinline__ uint64_t umma_desc(const void *p, uint32_t lbo, uint32_t sbo) {
+  const uint32_t a = smem_u32(p);
+  return (uint64_t)((a >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, A
+// K-major, B K-major or MN-major, shape M x N.
+__device__ __forceinline__ uint32_t umma_idesc(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// 32 consecutive 32-bit TMEM columns of this thread's lane
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t addr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(addr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+      "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+      "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// A bounded wait every thread takes; true on all threads only if it completed
+// on all of them.
+__device__ __forceinline__ bool cta_wait(uint64_t *bar, uint32_t parity, long long cap) {
+  const bool ok = mbar_wait_bounded(bar, parity, cap);
+  return !__syncthreads_or(!ok);
+}
 
 }  // namespace
 
 template <int D, int G>
-__global__ void __launch_bounds__(kSmdThreads) smd_attn_kernel(SmdParams p) {
-  constexpr int QP = 16 * (kSmdWarps / G);   // query positions per CTA
-  constexpr int PITCH = D + 8;               // smem row pitch in elements
-  constexpr int TILE = kKeyBlock * PITCH;    // elements per K or V tile
-  constexpr int CH = D / 8;                  // 16-byte chunks per row
-  constexpr int KS = D / 16;                 // k-steps of q.K
-  constexpr int ND = D / 8;                  // n-tiles of the output
-  extern __shared__ __align__(16) uint8_t smem[];
-  __nv_bfloat16 *ks = reinterpret_cast<__nv_bfloat16 *>(smem);     // [2][TILE]
-  __nv_bfloat16 *vs = ks + 2 * TILE;                                 // [2][TILE]
-  int *blist = reinterpret_cast<int *>(vs + 2 * TILE);               // [T/64 + 1]
+__global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
+  constexpr int QP = kTcRows / G;                          // query positions per CTA
+  constexpr int CH = D / 8;                                // 16-byte chunks of a row
+  constexpr int QBYTES = kTcRows * D * 2;
+  constexpr int KVBYTES = kKeyBlock * D * 2;
+  constexpr int PBYTES = kTcRows * kKeyBlock * 2;
+  constexpr uint32_t TCOLS = D == 128 ? 256u : 128u;       // S (64 columns) then O (D columns)
+  constexpr uint32_t OCOL = kKeyBlock;
+  constexpr long long kCap = 1ll << 31;                    // cycles per wait (about a second)
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // Q: element (row, d) at ((d/8)*16 + row/8)*128 + (row%8)*16 + (d%8)*2
+  // K, V: element (key, d) at ((d/8)*8 + key/8)*128 + (key%8)*16 + (d%8)*2
+  // P: element (row, key) at ((key/8)*16 + row/8)*128 + (row%8)*16 + (key%8)*2
+  uint8_t *sq = smem;
+  uint8_t *sk = sq + QBYTES;
+  uint8_t *sv = sk + KVBYTES;
+  uint8_t *sph = sv + KVBYTES;
+  uint8_t *spl = sph + PBYTES;
+  int *blist = reinterpret_cast<int *>(spl + PBYTES);      // [T/64 + 1]
   __shared__ uint32_t active[kMaxSmdBlocks / 32];
   __shared__ int nact;
+  __shared__ __align__(8) uint64_t bar_s, bar_o;
+  __shared__ uint32_t tslot;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int grp = lane >> 2, tig = lane & 3;
   const int b = blockIdx.z, h = blockIdx.y;
   const int ntile = (p.T + QP - 1) / QP;
   const int t0 = (ntile - 1 - static_cast<int>(blockIdx.x)) * QP;   // longest rows first
@@ -75,27 +147,27 @@ __global__ void __launch_bounds__(kSmdThreads) smd_attn_kernel(SmdParams p) {
       L = L < 0 ? 0 : p.T;
     }
   }
-  const int g = warp % G, pg = warp / G;
-  const int hq = h * G + g;
-  const int ta = t0 + 16 * pg + grp, tb = ta + 8;   // this lane's two query rows
+  const int r = tid;                                       // tile row = TMEM lane
+  const int g = r / QP, t = t0 + r % QP, hq = h * G + g;
+  const bool live = t < L;
 
   // ---- active key blocks of this CTA's rows
-  const int tlast = min(t0 + QP, L) - 1;            // last query row that exists
+  const int tlast = min(t0 + QP, L) - 1;
   const int nblk = tlast >= 0 ? tlast / kKeyBlock + 1 : 0;
-  for (int i = tid; i < (nblk + 31) / 32; i += kSmdThreads) active[i] = 0u;
+  for (int i = tid; i < (nblk + 31) / 32; i += kTcThreads) active[i] = 0u;
   __syncthreads();
   if (p.mask) {
-    const int nw = 2 * nblk;                        // mask words covering the blocks
+    const int nw = 2 * nblk;
     const int rows = tlast - t0 + 1;
-    for (int idx = tid; idx < rows * nw; idx += kSmdThreads) {
-      const int r = idx / nw, w = idx % nw;
+    for (int idx = tid; idx < rows * nw; idx += kTcThreads) {
+      const int rr = idx / nw, w = idx % nw;
       const uint32_t word = w < p.mask_stride
-                                ? __ldg(p.mask + (((long long)b * p.Hkv + h) * p.T + t0 + r) * p.mask_stride + w)
+                                ? __ldg(p.mask + (((long long)b * p.Hkv + h) * p.T + t0 + rr) * p.mask_stride + w)
                                 : 0u;
       if (word) atomicOr(&active[(w >> 1) >> 5], 1u << ((w >> 1) & 31));
     }
   } else {
-    for (int j = tid; j < nblk; j += kSmdThreads) atomicOr(&active[j >> 5], 1u << (j & 31));
+    for (int j = tid; j < nblk; j += kTcThreads) atomicOr(&active[j >> 5], 1u << (j & 31));
   }
   __syncthreads();
   if (warp == 0) {
@@ -111,199 +183,228 @@ __global__ void __launch_bounds__(kSmdThreads) smd_attn_kernel(SmdParams p) {
   }
   __syncthreads();
   const int na = nact;
+  const long long orow = (((long long)b * p.T + t) * p.Hq + hq) * D;
 
-  // ---- Q fragments (rows beyond the length are zero)
-  uint32_t qa[KS][4];
-  {
-    const __nv_bfloat16 *qra = p.q + (((long long)b * p.T + ta) * p.Hq + hq) * D;
-    const __nv_bfloat16 *qrb = p.q + (((long long)b * p.T + tb) * p.Hq + hq) * D;
-#pragma unroll
-    for (int s = 0; s < KS; ++s) {
-      const int d = s * 16 + 2 * tig;
-      qa[s][0] = ta < L ? *reinterpret_cast<const uint32_t *>(qra + d) : 0u;
-      qa[s][1] = tb < L ? *reinterpret_cast<const uint32_t *>(qrb + d) : 0u;
-      qa[s][2] = ta < L ? *reinterpret_cast<const uint32_t *>(qra + d + 8) : 0u;
-      qa[s][3] = tb < L ? *reinterpret_cast<const uint32_t *>(qrb + d + 8) : 0u;
+  if (na == 0) {   // nothing visible to any row of the CTA: the rows are 0
+    if (t < p.T) {
+      if (p.out_fp32) {
+        float4 *o = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + orow);
+        for (int c = 0; c < D / 4; ++c) o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        uint4 *o = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + orow);
+        for (int c = 0; c < D / 8; ++c) o[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
+    return;
   }
 
-  auto load_block = [&](int j, int stage) {
+  // ---- TMEM, barriers, Q tile, first K and V tiles
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tslot)),
+                 "n"(TCOLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    mbar_init(&bar_s, 1);
+    mbar_init(&bar_o, 1);
+    fence_mbar_init();
+  }
+  {
+    const __nv_bfloat16 *qrow = p.q + orow;
+#pragma unroll 4
+    for (int c = 0; c < CH; ++c) {
+      const uint4 v = live ? *reinterpret_cast<const uint4 *>(qrow + c * 8) : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4 *>(sq + (c * 16 + r / 8) * 128 + (r % 8) * 16) = v;
+    }
+  }
+  auto load_kv = [&](uint8_t *dst_tile, const __nv_bfloat16 *src_base, int j) {
     const int kb = j * kKeyBlock;
-    for (int c = tid; c < 2 * kKeyBlock * CH; c += kSmdThreads) {
-      const int which = c / (kKeyBlock * CH), rem = c % (kKeyBlock * CH);
-      const int row = rem / CH, ch = rem % CH;
-      const int pos = kb + row;
+    for (int e = tid; e < kKeyBlock * CH; e += kTcThreads) {
+      const int n = e / CH, c = e % CH;
+      const int pos = kb + n;
       const bool in = pos < L;
-      const __nv_bfloat16 *base = which ? p.v : p.k;
-      const __nv_bfloat16 *src = base + (((long long)b * p.T + (in ? pos : 0)) * p.Hkv + h) * D + ch * 8;
-      __nv_bfloat16 *dst = (which ? vs : ks) + stage * TILE + row * PITCH + ch * 8;
-      cp_async16(smem_u32(dst), src, in ? 16u : 0u);
+      const __nv_bfloat16 *src = src_base + (((long long)b * p.T + (in ? pos : 0)) * p.Hkv + h) * D + c * 8;
+      cp_async16(smem_u32(dst_tile + (c * 8 + n / 8) * 128 + (n % 8) * 16), src, in ? 16u : 0u);
     }
     cp_async_commit();
   };
+  load_kv(sk, p.k, blist[0]);
+  load_kv(sv, p.v, blist[0]);
+  tc_before_sync();
+  __syncthreads();
+  tc_after_sync();
+  const uint32_t tmem = tslot;
+  const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's lane quarter
+  const uint32_t idesc_s = umma_idesc(kTcRows, kKeyBlock, false);
+  const uint32_t idesc_o = umma_idesc(kTcRows, D, true);
+  const uint32_t *mrow = p.mask && live ? p.mask + (((long long)b * p.Hkv + h) * p.T + t) * p.mask_stride : nullptr;
 
-  float o[ND][4];
-#pragma unroll
-  for (int n = 0; n < ND; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
-  const uint32_t *mra = p.mask ? p.mask + (((long long)b * p.Hkv + h) * p.T + ta) * p.mask_stride : nullptr;
-  const uint32_t *mrb = p.mask ? p.mask + (((long long)b * p.Hkv + h) * p.T + tb) * p.mask_stride : nullptr;
-
-  if (na > 0) load_block(blist[0], 0);
-  for (int i = 0; i < na; ++i) {
-    if (i + 1 < na) {
-      load_block(blist[i + 1], (i + 1) & 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
+  float m_used = -INFINITY, l = 0.f;
+  uint32_t ph_s = 0, ph_o = 0;
+  bool ok = true;
+  for (int i = 0; i < na && ok; ++i) {
+    const int j = blist[i], kb = j * kKeyBlock;
+    // K(i) (and at i = 0 also V(0)) has landed: it is the only group in flight
+    cp_async_wait<0>();
+    fence_async_smem();
+    tc_before_sync();
     __syncthreads();
-    const int j = blist[i], kb = j * kKeyBlock, stage = i & 1;
-    const __nv_bfloat16 *kt = ks + stage * TILE;
-    const __nv_bfloat16 *vt = vs + stage * TILE;
-
-    // S = Q K^T over the 64 keys of the block
-    float s[8][4];
+    tc_after_sync();
+    if (tid == 0) {
 #pragma unroll
-    for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-    // K fragments by ldmatrix: matrices (keys 8n.., d 16st), (8n.., 16st + 8),
-    // (8n + 8.., 16st), (8n + 8.., 16st + 8) give b0, b1 of n-tiles n and n + 1
-    const int kmi = lane >> 3, kri = lane & 7;
-#pragma unroll
-    for (int st = 0; st < KS; ++st) {
-#pragma unroll
-      for (int n = 0; n < 8; n += 2) {
-        uint32_t bk[4];
-        ldmatrix_x4(bk, smem_u32(kt + ((n + (kmi >> 1)) * 8 + kri) * PITCH + st * 16 + (kmi & 1) * 8));
-        mma_bf16(s[n], qa[st], bk[0], bk[1]);
-        mma_bf16(s[n + 1], qa[st], bk[2], bk[3]);
-      }
+      for (int st = 0; st < D / 16; ++st)
+        umma_bf16(tmem, umma_desc(sq + st * 2 * 2048, 2048, 128), umma_desc(sk + st * 2 * 1024, 1024, 128), idesc_s,
+                  st > 0 ? 1u : 0u);
+      umma_commit(&bar_s);
     }
+    if (i > 0) {   // P V of the previous block: its P tiles, V tile and O are free/stable after this
+      ok = cta_wait(&bar_o, ph_o, kCap);
+      ph_o ^= 1u;
+      if (!ok) break;
+      tc_after_sync();
+      load_kv(sv, p.v, j);
+    }
+    ok = cta_wait(&bar_s, ph_s, kCap);
+    ph_s ^= 1u;
+    if (!ok) break;
+    tc_after_sync();
+    float x[kKeyBlock];
+    {
+      uint32_t sr[32];
+      tmem_ld32(trow, sr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(sr[k]);
+      tmem_ld32(trow + 32, sr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 32; ++k) x[32 + k] = __uint_as_float(sr[k]);
+    }
+    if (i + 1 < na) load_kv(sk, p.k, blist[i + 1]);   // S is read: the K tile is free
 
-    // visibility: query row < L, key <= query (so key < L), mask bit set
-    uint32_t wa0 = 0xffffffffu, wa1 = 0xffffffffu, wb0 = 0xffffffffu, wb1 = 0xffffffffu;
+    // visibility: live row, key <= query, mask bit set
+    uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
     if (p.mask) {
-      const int w0 = kb >> 5;
-      wa0 = ta < L && w0 < p.mask_stride ? __ldg(mra + w0) : 0u;
-      wa1 = ta < L && w0 + 1 < p.mask_stride ? __ldg(mra + w0 + 1) : 0u;
-      wb0 = tb < L && w0 < p.mask_stride ? __ldg(mrb + w0) : 0u;
-      wb1 = tb < L && w0 + 1 < p.mask_stride ? __ldg(mrb + w0 + 1) : 0u;
+      const int wi = kb >> 5;
+      w0 = mrow && wi < p.mask_stride ? __ldg(mrow + wi) : 0u;
+      w1 = mrow && wi + 1 < p.mask_stride ? __ldg(mrow + wi + 1) : 0u;
     }
-    float mxa = -INFINITY, mxb = -INFINITY;
+    float mloc = -INFINITY;
 #pragma unroll
-    for (int n = 0; n < 8; ++n) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int kk = n * 8 + 2 * tig + e;          // key offset in the block
-        const int key = kb + kk;
-        const uint32_t bit = 1u << (kk & 31);
-        const bool va = ta < L && key <= ta && ((kk < 32 ? wa0 : wa1) & bit);
-        const bool vb = tb < L && key <= tb && ((kk < 32 ? wb0 : wb1) & bit);
-        s[n][e] = va ? s[n][e] * p.scale_log2 : -INFINITY;
-        s[n][2 + e] = vb ? s[n][2 + e] * p.scale_log2 : -INFINITY;
-        mxa = fmaxf(mxa, s[n][e]);
-        mxb = fmaxf(mxb, s[n][2 + e]);
+    for (int k = 0; k < kKeyBlock; ++k) {
+      const bool vis = live && kb + k <= t && (((k < 32 ? w0 : w1) >> (k & 31)) & 1u);
+      x[k] = vis ? x[k] * p.scale_log2 : -INFINITY;
+      mloc = fmaxf(mloc, x[k]);
+    }
+    float corr = 1.f;
+    bool resc = false;
+    if (mloc > m_used + 8.f) {   // also true when the first visible key arrives
+      if (m_used != -INFINITY) {
+        resc = true;
+        corr = ex2(m_used - mloc);
       }
+      m_used = mloc;
     }
+    const float base = m_used == -INFINITY ? 0.f : m_used;
+    float lsum = 0.f;
 #pragma unroll
-    for (int x = 1; x < 4; x <<= 1) {
-      mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, x));
-      mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, x));
+    for (int k = 0; k < kKeyBlock; ++k) {
+      x[k] = ex2(x[k] - base);
+      lsum += x[k];
     }
-    const float mna = fmaxf(ma, mxa), mnb = fmaxf(mb, mxb);
-    // a row with nothing visible so far keeps m = -inf, weights 0, factor 1
-    const float ca = mna == -INFINITY ? 1.f : ex2(ma - mna);
-    const float cb = mnb == -INFINITY ? 1.f : ex2(mb - mnb);
-    const float ba = mna == -INFINITY ? 0.f : mna, bb = mnb == -INFINITY ? 0.f : mnb;
-    ma = mna;
-    mb = mnb;
-    la *= ca;
-    lb *= cb;
+    l = l * corr + lsum;
+    if (__any_sync(0xffffffffu, resc)) {   // this warp's O rows in TMEM (settled: P V of i - 1 is done)
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(trow + OCOL + c0, o);
+        tmem_wait_ld();
 #pragma unroll
-    for (int n = 0; n < ND; ++n) {
-      o[n][0] *= ca;
-      o[n][1] *= ca;
-      o[n][2] *= cb;
-      o[n][3] *= cb;
-    }
-#pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      s[n][0] = ex2(s[n][0] - ba);
-      s[n][1] = ex2(s[n][1] - ba);
-      s[n][2] = ex2(s[n][2] - bb);
-      s[n][3] = ex2(s[n][3] - bb);
-      la += s[n][0] + s[n][1];
-      lb += s[n][2] + s[n][3];
-    }
-
-    // O += P V, P as bf16 hi + lo
-#pragma unroll
-    for (int kc = 0; kc < 4; ++kc) {
-      uint32_t ph[4], pl[4];
-      const float *s0 = s[2 * kc], *s1 = s[2 * kc + 1];
-      const float f[8] = {s0[0], s0[1], s0[2], s0[3], s1[0], s1[1], s1[2], s1[3]};
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        // a0: row a keys 2tig..; a1: row b; a2: row a keys 8 + 2tig..; a3: row b
-        const float x0 = f[(r & 1) * 2 + (r >> 1) * 4], x1 = f[(r & 1) * 2 + (r >> 1) * 4 + 1];
-        ph[r] = pack_bf16x2(x0, x1);
-        pl[r] = pack_bf16x2(x0 - bf16lo_to_f32(ph[r]), x1 - bf16hi_to_f32(ph[r]));
+        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * corr);
+        tmem_st32(trow + OCOL + c0, o);
       }
-#pragma unroll
-      for (int n = 0; n < ND; n += 2) {
-        uint32_t bv[4];
-        const int mi = lane >> 3, ri = lane & 7;
-        const __nv_bfloat16 *vr = vt + (kc * 16 + (mi & 1) * 8 + ri) * PITCH + (n + (mi >> 1)) * 8;
-        ldmatrix_x4_trans(bv, smem_u32(vr));
-        mma_bf16(o[n], ph, bv[0], bv[1]);
-        mma_bf16(o[n], pl, bv[0], bv[1]);
-        mma_bf16(o[n + 1], ph, bv[2], bv[3]);
-        mma_bf16(o[n + 1], pl, bv[2], bv[3]);
-      }
+      tmem_wait_st();
     }
-    __syncthreads();   // the stage is refilled by the next iteration's prefetch
+    // P as bf16 hi + lo, row r
+#pragma unroll
+    for (int c = 0; c < kKeyBlock / 8; ++c) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = x[c * 8 + 2 * e], x1 = x[c * 8 + 2 * e + 1];
+        hw[e] = pack_bf16x2(x0, x1);
+        lw[e] = pack_bf16x2(x0 - bf16lo_to_f32(hw[e]), x1 - bf16hi_to_f32(hw[e]));
+      }
+      const int off = (c * 16 + r / 8) * 128 + (r % 8) * 16;
+      *reinterpret_cast<uint4 *>(sph + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4 *>(spl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    // V(i) has landed (K(i + 1) may still be in flight)
+    if (i + 1 < na) cp_async_wait<1>(); else cp_async_wait<0>();
+    fence_async_smem();
+    tc_before_sync();
+    __syncthreads();
+    tc_after_sync();
+    if (tid == 0) {
+#pragma unroll
+      for (int kk = 0; kk < kKeyBlock / 16; ++kk) {
+        const uint64_t dv = umma_desc(sv + kk * 2 * 128, 128, 1024);
+        umma_bf16(tmem + OCOL, umma_desc(sph + kk * 2 * 2048, 2048, 128), dv, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+        umma_bf16(tmem + OCOL, umma_desc(spl + kk * 2 * 2048, 2048, 128), dv, idesc_o, 1u);
+      }
+      umma_commit(&bar_o);
+    }
   }
-
-  // ---- normalise and store
+  if (ok) ok = cta_wait(&bar_o, ph_o, kCap);   // the last P V
+  if (!ok) {
+    if (tid == 0 && p.err) set_error(p.err, kErrTimeout);
+  } else {
+    tc_after_sync();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t o[32];
+      tmem_ld32(trow + OCOL + c0, o);
+      tmem_wait_ld();
+      if (t < p.T) {
+        if (p.out_fp32) {
+          float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(p.out) + orow + c0);
 #pragma unroll
-  for (int x = 1; x < 4; x <<= 1) {
-    la += __shfl_xor_sync(0xffffffffu, la, x);
-    lb += __shfl_xor_sync(0xffffffffu, lb, x);
-  }
-  const float ia = la > 0.f ? 1.f / la : 0.f, ib = lb > 0.f ? 1.f / lb : 0.f;
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
+                                 __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
+        } else {
+          uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + orow + c0);
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int t = half ? tb : ta;
-    if (t >= p.T) continue;
-    const float inv = half ? ib : ia;
-    const long long base = (((long long)b * p.T + t) * p.Hq + hq) * D + 2 * tig;
-#pragma unroll
-    for (int n = 0; n < ND; ++n) {
-      const float y0 = o[n][2 * half] * inv, y1 = o[n][2 * half + 1] * inv;
-      if (p.out_fp32) {
-        *reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + base + n * 8) = make_float2(y0, y1);
-      } else {
-        *reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + base + n * 8) =
-            pack_bf16x2(y0, y1);
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * k]) * inv, __uint_as_float(o[8 * k + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv));
+        }
       }
     }
   }
+  cp_async_wait<0>();
+  tc_before_sync();
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(TCOLS));
 }
 
 size_t smd_smem_bytes(int D, int T) {
-  const size_t tile = (size_t)64 * (D + 8) * 2;
-  return 4 * tile + ((size_t)(T + 63) / 64 + 1) * 4;
+  const size_t q = (size_t)128 * D * 2, kv = (size_t)64 * D * 2, pt = (size_t)128 * 64 * 2;
+  return q + 2 * kv + 2 * pt + ((size_t)(T + 63) / 64 + 1) * 4;
 }
 
 template <int D, int G>
 static cudaError_t launch_smd_dg(const SmdParams &p, cudaStream_t stream) {
-  constexpr int QP = 16 * (kSmdWarps / G);
+  constexpr int QP = kTcRows / G;
   const size_t smem = smd_smem_bytes(D, p.T);
   cudaError_t e = cudaFuncSetAttribute(smd_attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid((p.T + QP - 1) / QP, p.Hkv, p.B);
-  return launch_pdl(smd_attn_kernel<D, G>, grid, dim3(kSmdThreads), smem, stream, p);
+  return launch_pdl(smd_attn_kernel<D, G>, grid, dim3(kTcThreads), smem, stream, p);
 }
 
 template <int D>

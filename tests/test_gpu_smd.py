@@ -106,3 +106,24 @@ def test_learner_full_size_rows_equal_rollout_decode():
         assert_close(got[:, i], ref, what="row %d" % t)
     del q, k, v, mask, out
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("D,Hq,Hkv", [(64, 4, 2), (128, 8, 2)])
+@pytest.mark.parametrize("div", [16.0, 160.0])
+def test_growing_scores_rescale_the_accumulator(D, Hq, Hkv, div):
+    """K rows scaled up along the sequence: a row's running maximum grows by
+    about 60 (div 16) or 5-12 (div 160) base-2 units per 64-key block, so the
+    accumulator is rescaled in place, every block or only some; results still
+    match the oracle."""
+    T = 640
+    wl, q, k, v = _case(2, T, Hq, Hkv, D, seed=31 + D)
+    gain = (1.0 + torch.arange(T, dtype=torch.float32) / div)[None, :, None, None]
+    k = (k.float() * gain).to(torch.bfloat16)
+    q = (q.float().abs()).to(torch.bfloat16)          # positive queries ...
+    k = k.float().abs().to(torch.bfloat16)            # ... and keys: scores grow with the key position
+    mask = synth.gen_shadow_mask(wl, T)
+    for m in (None, mask):
+        ref = _oracle(q, k, v, wl.softmax_scale, mask=m)
+        out, err = _run(q, k, v, wl.softmax_scale, mask=m)
+        assert err == 0
+        assert_close(out.cpu().numpy(), ref, what="growing scores D=%d" % D)
