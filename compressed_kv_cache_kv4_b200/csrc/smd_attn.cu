@@ -99,11 +99,11 @@ __device__ __forceinline__ void tmem_st32(uint32_t addr, const uint32_t (&r)[32]
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// A bounded wait every thread takes; true on all threads only if it completed
-// on all of them.
-__device__ __forceinline__ bool cta_wait(uint64_t *bar, uint32_t parity, long long cap) {
-  const bool ok = mbar_wait_bounded(bar, parity, cap);
-  return !__syncthreads_or(!ok);
+// A bounded wait; once one has run out on this thread the later ones give up
+// at once, so control flow stays the same on every thread and the total wait
+// stays bounded. The CTA checks the outcome once, at the end.
+__device__ __forceinline__ void sticky_wait(uint64_t *bar, uint32_t parity, long long cap, bool &ok) {
+  ok = mbar_wait_bounded(bar, parity, ok ? cap : 0) && ok;
 }
 
 }  // namespace
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
   float m_used = -INFINITY, l = 0.f;
   uint32_t ph_s = 0, ph_o = 0;
   bool ok = true;
-  for (int i = 0; i < na && ok; ++i) {
+  for (int i = 0; i < na; ++i) {
     const int j = blist[i], kb = j * kKeyBlock;
     // K(i) (and at i = 0 also V(0)) has landed: it is the only group in flight
     cp_async_wait<0>();
@@ -257,16 +257,21 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
                   st > 0 ? 1u : 0u);
       umma_commit(&bar_s);
     }
+    // this row's mask words for the block, loaded while the MMAs run
+    uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
+    if (p.mask) {
+      const int wi = kb >> 5;
+      w0 = mrow && wi < p.mask_stride ? __ldg(mrow + wi) : 0u;
+      w1 = mrow && wi + 1 < p.mask_stride ? __ldg(mrow + wi + 1) : 0u;
+    }
     if (i > 0) {   // P V of the previous block: its P tiles, V tile and O are free/stable after this
-      ok = cta_wait(&bar_o, ph_o, kCap);
+      sticky_wait(&bar_o, ph_o, kCap, ok);
       ph_o ^= 1u;
-      if (!ok) break;
       tc_after_sync();
       load_kv(sv, p.v, j);
     }
-    ok = cta_wait(&bar_s, ph_s, kCap);
+    sticky_wait(&bar_s, ph_s, kCap, ok);
     ph_s ^= 1u;
-    if (!ok) break;
     tc_after_sync();
     float x[kKeyBlock];
     {
@@ -283,12 +288,6 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
     if (i + 1 < na) load_kv(sk, p.k, blist[i + 1]);   // S is read: the K tile is free
 
     // visibility: live row, key <= query, mask bit set
-    uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
-    if (p.mask) {
-      const int wi = kb >> 5;
-      w0 = mrow && wi < p.mask_stride ? __ldg(mrow + wi) : 0u;
-      w1 = mrow && wi + 1 < p.mask_stride ? __ldg(mrow + wi + 1) : 0u;
-    }
     float mloc = -INFINITY;
 #pragma unroll
     for (int k = 0; k < kKeyBlock; ++k) {
@@ -355,8 +354,8 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
       umma_commit(&bar_o);
     }
   }
-  if (ok) ok = cta_wait(&bar_o, ph_o, kCap);   // the last P V
-  if (!ok) {
+  sticky_wait(&bar_o, ph_o, kCap, ok);   // the last P V
+  if (__syncthreads_or(!ok)) {
     if (tid == 0 && p.err) set_error(p.err, kErrTimeout);
   } else {
     tc_after_sync();
