@@ -22,10 +22,11 @@
 // as an MN-major operand). O is rescaled in TMEM only when a row's maximum
 // grows by more than 2^8 since it was last used (the exponentials stay below
 // 256, the result is the same softmax). MMAs are issued by one thread and
-// signal an mbarrier through tcgen05.commit; every wait is bounded. K tiles of
-// the next block load (cp.async) while the softmax runs, V tiles while the
-// next S is computed. Operands use the no-swizzle core-matrix layout: 8 rows
-// of 16 bytes per core matrix.
+// signal an mbarrier through tcgen05.commit; every wait is bounded. One CTA
+// barrier per block: after it the issuing thread queues P V of this block and
+// then S of the next. K tiles of the next block load (cp.async) while the
+// softmax runs, V tiles while S is computed. Operands use the no-swizzle
+// core-matrix layout: 8 rows of 16 bytes per core matrix.
 #include <math.h>
 
 #include "kv4_common.cuh"
@@ -230,6 +231,8 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
   };
   load_kv(sk, p.k, blist[0]);
   load_kv(sv, p.v, blist[0]);
+  cp_async_wait<0>();
+  fence_async_smem();
   tc_before_sync();
   __syncthreads();
   tc_after_sync();
@@ -238,25 +241,20 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
   const uint32_t idesc_s = umma_idesc(kTcRows, kKeyBlock, false);
   const uint32_t idesc_o = umma_idesc(kTcRows, D, true);
   const uint32_t *mrow = p.mask && live ? p.mask + (((long long)b * p.Hkv + h) * p.T + t) * p.mask_stride : nullptr;
+  auto issue_qk = [&]() {
+#pragma unroll
+    for (int st = 0; st < D / 16; ++st)
+      umma_bf16(tmem, umma_desc(sq + st * 2 * 2048, 2048, 128), umma_desc(sk + st * 2 * 1024, 1024, 128), idesc_s,
+                st > 0 ? 1u : 0u);
+    umma_commit(&bar_s);
+  };
+  if (tid == 0) issue_qk();
 
   float m_used = -INFINITY, l = 0.f;
   uint32_t ph_s = 0, ph_o = 0;
   bool ok = true;
   for (int i = 0; i < na; ++i) {
     const int j = blist[i], kb = j * kKeyBlock;
-    // K(i) (and at i = 0 also V(0)) has landed: it is the only group in flight
-    cp_async_wait<0>();
-    fence_async_smem();
-    tc_before_sync();
-    __syncthreads();
-    tc_after_sync();
-    if (tid == 0) {
-#pragma unroll
-      for (int st = 0; st < D / 16; ++st)
-        umma_bf16(tmem, umma_desc(sq + st * 2 * 2048, 2048, 128), umma_desc(sk + st * 2 * 1024, 1024, 128), idesc_s,
-                  st > 0 ? 1u : 0u);
-      umma_commit(&bar_s);
-    }
     // this row's mask words for the block, loaded while the MMAs run
     uint32_t w0 = 0xffffffffu, w1 = 0xffffffffu;
     if (p.mask) {
@@ -270,7 +268,7 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
       tc_after_sync();
       load_kv(sv, p.v, j);
     }
-    sticky_wait(&bar_s, ph_s, kCap, ok);
+    sticky_wait(&bar_s, ph_s, kCap, ok);   // S = Q K^T of this block
     ph_s ^= 1u;
     tc_after_sync();
     float x[kKeyBlock];
@@ -338,8 +336,8 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
       *reinterpret_cast<uint4 *>(sph + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4 *>(spl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
-    // V(i) has landed (K(i + 1) may still be in flight)
-    if (i + 1 < na) cp_async_wait<1>(); else cp_async_wait<0>();
+    // V(i) and K(i + 1) have landed; P(i) is written; S(i) has been read
+    cp_async_wait<0>();
     fence_async_smem();
     tc_before_sync();
     __syncthreads();
@@ -352,6 +350,7 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
         umma_bf16(tmem + OCOL, umma_desc(spl + kk * 2 * 2048, 2048, 128), dv, idesc_o, 1u);
       }
       umma_commit(&bar_o);
+      if (i + 1 < na) issue_qk();   // S of the next block, queued behind this P V
     }
   }
   sticky_wait(&bar_o, ph_o, kCap, ok);   // the last P V
