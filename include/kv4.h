@@ -17,7 +17,12 @@
  *          attention instead of slicing tensors.
  *  [KVP]   promo of arXiv 2602.10238 ("learning to evict"), core-mechanism
  *          section, and the TTKV promo (arXiv 2604.19769), insight 1: score each
- *          position, rank, truncate at a budget, per attention head.
+ *          position, rank, truncate at a budget, per attention head; the KVP
+ *          promo's engineering-limitations section, third item: in a paged
+ *          cache of 16-position blocks the ranking is taken per block.
+ *  [KVS]   "KV-streams for Efficient Compaction in Agentic Reinforcement
+ *          Learning" (summary page), method details, core idea: a compacted
+ *          cache keeps streaming into its surviving pages.
  * Stated readings where the pages are silent: symmetric INT4 codes in [-7, 7]
  * per group of 32 consecutive head_dim elements with one fp16 scale; per-token
  * INT8 codes in [-127, 127] with one fp16 scale; scales are max|x|/qmax rounded
