@@ -349,6 +349,8 @@ def run_kv4(args, ws, rank):
                      min(args.steps, 512))
     if rank == 0 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline(wl, kpre, vpre, offpre, lens_pre)
+        if "secondary" in res:   # the oracle beside the other measured rows
+            res["cpu_baseline"]["rows"] = cpu_rows()
     cache.close()
     return wl, res
 
@@ -717,6 +719,43 @@ def cpu_baseline(wl, k, v, off, lens_pre, budget_s=20.0):
     return {"value": total_pos / total_t, "unit": "KV positions/s", "cores": oracle_threads(), "kind": "oracle",
             "sample": "%d of %d sequences of the %s workload (%d positions): oracle cache image + fp64 decode, "
                       "%.1f s" % (len(seqs_done), wl.B, wl.name, total_pos, total_t)}
+
+
+def cpu_rows():
+    """The oracle timed beside the eviction and learner rows, on the host cores:
+    page-granular eviction on the whole eviction workload (64 sequences of
+    16384 positions, 8 KV heads, 10% of pages kept; seeded uniform scores stand
+    in for the H2O-style ones, the oracle's work does not depend on the values),
+    and the learner attention under the shadow mask on one sequence of 1024
+    positions with the learner heads (32/8, D = 128)."""
+    import oracle as O
+    from compressed_kv_cache_kv4_b200 import synth
+    out = {}
+    wl = synth.workload("evict")
+    L = int(wl.lens.max())
+    rng = np.random.default_rng(1005)
+    scores = rng.random((wl.B, wl.Hkv, L), dtype=np.float32)
+    npg = L // 16
+    pt = np.arange(wl.B * npg, dtype=np.int32).reshape(wl.B, npg)
+    t0 = time.perf_counter()
+    _, _, _, cnt, _ = O.evict_pages(scores, wl.lens, pt, None, wl.D, 100, wl.sink, wl.recent)
+    dt = time.perf_counter() - t0
+    out["page_evict"] = {"us": dt * 1e6, "pages_freed": int(cnt.sum()),
+                         "sample": "all 64 sequences, 10% of pages kept, fp64 page sums and a full sort"}
+    wl = synth.workload("learner", B=1, T=1024)
+    T = 1024
+    q, k, v = synth.gen_learner_qkv(wl, T)
+    mask = synth.gen_shadow_mask(wl, T).numpy().view(np.uint32)
+    qb, kb, vb = synth.bf16_bits(q), synth.bf16_bits(k), synth.bf16_bits(v)
+    t0 = time.perf_counter()
+    O.masked_attn(qb, kb, vb, wl.softmax_scale, mask=mask)
+    dt = time.perf_counter() - t0
+    pairs = int(sum(bin(int(w)).count("1") for w in mask.reshape(-1)))
+    out["smd_learner"] = {"s": dt, "tflops_algorithmic": 4.0 * wl.D * wl.G * pairs / dt / 1e12,
+                          "sample": "1 sequence x 1024 positions, 32/8 heads, D = 128, shadow mask "
+                                    "(%d visible pairs), fp64" % pairs}
+    out["cores"] = oracle_threads()
+    return out
 
 
 def run_reference(args, ws, rank):
