@@ -19,6 +19,7 @@
 #include <mutex>
 
 #include "kv4.h"
+#include "kv4_internal.h"
 
 namespace {
 
@@ -34,7 +35,10 @@ std::atomic<void *> g_scratch_ptr[kMaxDevices];
 std::mutex g_setup_mutex;
 
 // Device address of g_noalloc_scratch on the current device; the first call
-// per device performs the lookup.
+// per device performs the lookup. The cached address assumes the device's
+// primary context lives as long as the process: after a cudaDeviceReset the
+// module is loaded again and the address may change, so a process that resets
+// a device must not call this entry point on it afterwards.
 kv4_status scratch_on_current_device(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -67,6 +71,14 @@ extern "C" kv4_status kv4_decode_attn_noalloc(kv4_cache *cache, void *stream, co
                                               void *out, int32_t out_is_fp32, int32_t B) {
   if (!cache || B < 0 || num_workers < 0) return KV4_ERR_INVALID;
   if (B == 0) return KV4_OK;
+  // The scratch handed to the kernels is the current device's copy of the
+  // array, so the current device must be the one the cache lives on.
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return KV4_ERR_CUDA;
+  }
+  if (dev != kv4::cache_device(cache)) return KV4_ERR_INVALID;
   // The scratch this call needs, from the same sizing rule as the workspace
   // of kv4_decode_attn; refuse before touching the device if it does not fit.
   size_t need = 0;
