@@ -52,6 +52,7 @@ def lib():
     L = C.CDLL(LIB_PATH)
     sig = {
         "kv4_status_string": (C.c_char_p, [C.c_int]),
+        "kv4_last_cuda_error": (C.c_char_p, []),
         "kv4_cache_bytes": (C.c_int, [C.POINTER(kv4_config), C.POINTER(_SZ), C.POINTER(_SZ)]),
         "kv4_cache_create": (C.c_int, [C.POINTER(kv4_config), _P, _SZ, _P, _SZ, C.POINTER(_P)]),
         "kv4_cache_destroy": (None, [_P]),
@@ -73,6 +74,7 @@ def lib():
         "kv4_device_info": (C.c_int, [C.POINTER(_I32), C.POINTER(_I32)]),
         "kv4_timing_enable": (C.c_int, [_I32, _I32]),
         "kv4_timing_read": (C.c_int, [_I32, C.POINTER(C.c_double), C.POINTER(_I32)]),
+        "kv4_timing_read_each": (C.c_int, [_I32, _P, _I32, C.POINTER(_I32)]),
         "kv4_timing_disable": (C.c_int, []),
     }
     for name, (res, args) in sig.items():
@@ -92,6 +94,8 @@ def header_symbols():
 
 def _check(st, what):
     if st != KV4_OK:
+        if st == KV4_ERR_CUDA:
+            what = "%s (%s)" % (what, lib().kv4_last_cuda_error().decode())
         raise Kv4Error(st, what)
 
 
@@ -247,6 +251,14 @@ def kv4_timing_read(kind):
     ms, n = C.c_double(0), _I32(0)
     _check(lib().kv4_timing_read(int(kind), C.byref(ms), C.byref(n)), "kv4_timing_read")
     return ms.value, n.value
+
+
+def kv4_timing_read_each(kind, cap=4096):
+    """Per-launch durations (ms, oldest first) of the recorded worker-kernel launches."""
+    buf = (C.c_float * max(int(cap), 1))()
+    n = _I32(0)
+    _check(lib().kv4_timing_read_each(int(kind), buf, int(cap), C.byref(n)), "kv4_timing_read_each")
+    return [float(buf[i]) for i in range(min(n.value, int(cap)))]
 
 
 def kv4_timing_disable():

@@ -7,7 +7,9 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <vector>
 
 #include "../../include/kv4.h"
@@ -30,9 +32,21 @@ struct kv4_cache {
   long long wait_cap;
 };
 
+int kv4::cache_device(const kv4_cache *cache) { return cache ? cache->device : -1; }
+
 namespace {
 
 constexpr size_t kAlign = 256;
+
+// Last CUDA runtime error seen by a libkv4 call of this thread (kv4_last_cuda_error).
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+// True (and recorded) if e is an error.
+bool bad(cudaError_t e) {
+  if (e == cudaSuccess) return false;
+  g_last_cuda = e;
+  return true;
+}
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -58,69 +72,147 @@ kv4_status check_config(const kv4_config *c) {
   return KV4_OK;
 }
 
-// Per (D, G, format) launch geometry, computed once per process.
-struct Geometry {
-  bool ready = false;
-  cudaError_t err = cudaSuccess;
-  DecodeLaunch l{};
+// ---------------------------------------------------------------- launch geometry, per device
+struct DeviceInfo {
+  int sms = 0, smem_sm = 0, smem_reserved = 0, smem_optin = 0;
 };
 
 std::mutex g_mu;
-Geometry g_geo[2][3][2];   // [D=64,128][G=1,2,4][int4, bf16]
-int g_num_sms = 0;
+std::map<int, DeviceInfo> g_dev;
+std::map<std::tuple<int, int, int>, cudaError_t> g_kv4_attr;             // (device, D, G)
+std::map<std::tuple<int, int, int, int, int>, int> g_kv4_occ;            // (device, D, G, HB, smem)
+std::map<std::tuple<int, int, int>, std::pair<cudaError_t, DecodeLaunch>> g_bf16_geo;   // (device, D, G)
 
-int gidx(int G) { return G == 1 ? 0 : (G == 2 ? 1 : 2); }
-
-cudaError_t geometry(int D, int G, bool bf16, DecodeLaunch *out, int *num_sms) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+// Attributes of the current device (looked up once per device).
+cudaError_t device_info(int *dev_out, DeviceInfo *out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  auto it = g_dev.find(dev);
+  if (it == g_dev.end()) {
+    DeviceInfo d;
+    e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
+    it = g_dev.emplace(dev, d).first;
   }
-  Geometry &g = g_geo[D == 128][gidx(G)][bf16];
-  if (!g.ready) {
-    g.err = decode_prepare(D, G, bf16, &g.l);
-    g.ready = true;
-  }
-  if (g.err != cudaSuccess) return g.err;
-  *out = g.l;
-  *num_sms = g_num_sms;
+  *dev_out = dev;
+  *out = it->second;
   return cudaSuccess;
 }
 
-int default_workers(const DecodeLaunch &l, int num_sms) { return num_sms * l.blocks_per_sm * kWarps; }
+// Heads per CTA of the KV4 kernel: the largest divisor of Hkv that is <= 8.
+int kv4_head_block(int Hkv) {
+  for (int hb = Hkv < 8 ? Hkv : 8; hb > 1; --hb)
+    if (Hkv % hb == 0) return hb;
+  return 1;
+}
 
-int resolve_workers(int requested, const DecodeLaunch &l, int num_sms) {
-  int nw = requested > 0 ? requested : default_workers(l, num_sms);
+struct Kv4Plan {
+  int HB, NVB, NS, smem, n_cta;
+};
+
+// Launch plan of the KV4 kernel for B sequences on the current device: as
+// many ring stages (up to 6) as let 16 warps (16 / HB CTAs) share an SM, and
+// by default as many CTAs as are resident at once (num_workers > 0: that many
+// warps, i.e. ceil(num_workers / HB) CTAs).
+kv4_status kv4_plan(int D, int G, int Hkv, int B, int num_workers, Kv4Plan *out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev = 0;
+  DeviceInfo di;
+  if (bad(device_info(&dev, &di))) return KV4_ERR_CUDA;
+  Kv4Plan pl{};
+  pl.HB = kv4_head_block(Hkv);
+  const long long nvb = (long long)B * (Hkv / pl.HB);
+  if (nvb > kMaxBatch) return KV4_ERR_UNSUPPORTED;
+  pl.NVB = static_cast<int>(nvb);
+  const int target = 16 / pl.HB > 0 ? 16 / pl.HB : 1;
+  const int budget = (di.smem_sm - target * di.smem_reserved) / target;
+  pl.NS = 6;
+  while (pl.NS > 2 && kv4_smem_bytes(D, pl.HB, pl.NS, pl.NVB) > budget) --pl.NS;
+  pl.smem = kv4_smem_bytes(D, pl.HB, pl.NS, pl.NVB);
+  if (pl.smem > di.smem_optin) return KV4_ERR_UNSUPPORTED;
+  const auto key = std::make_tuple(dev, D, G, pl.HB, pl.smem);
+  auto it = g_kv4_occ.find(key);
+  if (it == g_kv4_occ.end()) {
+    // the dynamic shared-memory limit is raised once per (device, D, G) to
+    // the device's opt-in maximum, which covers every plan
+    const auto akey = std::make_tuple(dev, D, G);
+    if (g_kv4_attr.find(akey) == g_kv4_attr.end())
+      g_kv4_attr.emplace(akey, kv4_decode_set_smem_limit(D, G, di.smem_optin));
+    if (bad(g_kv4_attr[akey])) return KV4_ERR_CUDA;
+    int nb = 0;
+    if (bad(kv4_decode_occupancy(D, G, pl.HB, pl.smem, &nb))) return KV4_ERR_CUDA;
+    it = g_kv4_occ.emplace(key, nb > 0 ? nb : 1).first;
+  }
+  const long long def = (long long)it->second * di.sms;
+  const long long want = num_workers > 0 ? ((long long)num_workers + pl.HB - 1) / pl.HB : def;
+  pl.n_cta = static_cast<int>(want < 1 ? 1 : (want > (1 << 20) ? (1 << 20) : want));
+  *out = pl;
+  return KV4_OK;
+}
+
+// bf16 comparison kernel geometry, per device.
+cudaError_t bf16_geometry(int D, int G, DecodeLaunch *out, int *num_sms) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev = 0;
+  DeviceInfo di;
+  cudaError_t e = device_info(&dev, &di);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_tuple(dev, D, G);
+  auto it = g_bf16_geo.find(key);
+  if (it == g_bf16_geo.end()) {
+    DecodeLaunch l{};
+    const cudaError_t pe = bf16_decode_prepare(D, G, &l);
+    it = g_bf16_geo.emplace(key, std::make_pair(pe, l)).first;
+  }
+  if (it->second.first != cudaSuccess) return it->second.first;
+  *out = it->second.second;
+  *num_sms = di.sms;
+  return cudaSuccess;
+}
+
+int bf16_workers(int requested, const DecodeLaunch &l, int num_sms) {
+  const int nw = requested > 0 ? requested : num_sms * l.blocks_per_sm * kWarps;
   return (nw + kWarps - 1) / kWarps * kWarps;
 }
 
-// Workspace: plan int32 [B+1] | first, last int32
-// [2*B*Hkv] each | partial slots [2*B*Hkv + nw][slot_floats] (INT8 ranges,
-// then INT4 ranges, each offset by the worker index). Everything is written
-// before it is read within a call, so the workspace needs no clearing.
-size_t decode_ws_bytes(int B, int Hkv, int G, int D, int nw) {
+// KV4 workspace: plan int32 [NVB+1] | first, last int32 [2*NVB] each |
+// partial slots [2*NVB + n_cta][HB][slot_floats] (INT8 ranges, then INT4
+// ranges, each offset by the CTA index).
+size_t kv4_ws_bytes(const Kv4Plan &pl, int G, int D) {
   const size_t slot = (size_t)slot_floats(G, D) * 4;
-  return round_up((size_t)(B + 1) * 4, kAlign) +
-         2 * round_up((size_t)2 * B * Hkv * 4, kAlign) +
+  return round_up((size_t)(pl.NVB + 1) * 4, kAlign) + 2 * round_up((size_t)2 * pl.NVB * 4, kAlign) +
+         round_up(((size_t)2 * pl.NVB + pl.n_cta) * pl.HB * slot, kAlign);
+}
+
+// bf16 workspace: plan int32 [B+1] | first, last int32 [2*B*Hkv] each |
+// partial slots [2*B*Hkv + nw][slot_floats].
+size_t bf16_ws_bytes(int B, int Hkv, int G, int D, int nw) {
+  const size_t slot = (size_t)slot_floats(G, D) * 4;
+  return round_up((size_t)(B + 1) * 4, kAlign) + 2 * round_up((size_t)2 * B * Hkv * 4, kAlign) +
          round_up(((size_t)2 * B * Hkv + nw) * slot, kAlign);
 }
 
-void carve_workspace(DecodeParams &p, void *ws) {
+// Carve a workspace with `nplan` plan entries and `nrange` ranges.
+void carve_workspace(DecodeParams &p, void *ws, size_t nplan, size_t nrange) {
   uint8_t *w = static_cast<uint8_t *>(ws);
   p.plan = reinterpret_cast<int *>(w);
-  w += round_up((size_t)(p.B + 1) * 4, kAlign);
+  w += round_up(nplan * 4, kAlign);
   p.first = reinterpret_cast<int *>(w);
-  w += round_up((size_t)2 * p.B * p.Hkv * 4, kAlign);
+  w += round_up(nrange * 4, kAlign);
   p.last = reinterpret_cast<int *>(w);
-  w += round_up((size_t)2 * p.B * p.Hkv * 4, kAlign);
+  w += round_up(nrange * 4, kAlign);
   p.slots = reinterpret_cast<float *>(w);
 }
 
-kv4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KV4_OK : KV4_ERR_CUDA; }
+kv4_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return KV4_OK;
+  g_last_cuda = e;
+  return KV4_ERR_CUDA;
+}
 
 // Timing hook state: per kind, a fixed pool of event pairs filled in call order.
 struct Timing {
@@ -158,6 +250,10 @@ void timing_free() {
 }  // namespace
 
 extern "C" {
+
+const char *kv4_last_cuda_error(void) {
+  return g_last_cuda == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda);
+}
 
 const char *kv4_status_string(kv4_status s) {
   switch (s) {
@@ -257,11 +353,14 @@ kv4_status kv4_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t num_q_
   if (num_q_heads < 1 || num_q_heads % Hkv) return KV4_ERR_INVALID;
   const int G = num_q_heads / Hkv;
   if (G != 1 && G != 2 && G != 4) return KV4_ERR_UNSUPPORTED;
-  DecodeLaunch l{};
-  int sms = 0;
-  if (geometry(cache->cfg.head_dim, G, false, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
-  const int nw = resolve_workers(num_workers, l, sms);
-  *bytes = decode_ws_bytes(B, Hkv, G, cache->cfg.head_dim, nw);
+  if (B == 0) {
+    *bytes = 0;
+    return KV4_OK;
+  }
+  Kv4Plan pl{};
+  const kv4_status st = kv4_plan(cache->cfg.head_dim, G, Hkv, B, num_workers, &pl);
+  if (st != KV4_OK) return st;
+  *bytes = kv4_ws_bytes(pl, G, cache->cfg.head_dim);
   return KV4_OK;
 }
 
@@ -281,12 +380,15 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 16)) return KV4_ERR_INVALID;
   if (retain_mask && (long long)mask_stride * 32 < (long long)pt_stride * kPageTokens) return KV4_ERR_INVALID;
   if (!isfinite(softmax_scale)) return KV4_ERR_INVALID;
-  DecodeLaunch l{};
-  int sms = 0;
-  if (geometry(D, G, false, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
-  const int nw = resolve_workers(num_workers, l, sms);
+  if (pt_stride > kMaxPtStride) return KV4_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (bad(cudaGetDevice(&dev))) return KV4_ERR_CUDA;
+  if (dev != cache->device) return KV4_ERR_INVALID;
+  Kv4Plan pl{};
+  const kv4_status ps = kv4_plan(D, G, Hkv, B, num_workers, &pl);
+  if (ps != KV4_OK) return ps;
   const bool has8 = cache->cfg.sink + cache->cfg.recent > 0;
-  if (ws_bytes < decode_ws_bytes(B, Hkv, G, D, nw)) return KV4_ERR_INVALID;
+  if (ws_bytes < kv4_ws_bytes(pl, G, D)) return KV4_ERR_INVALID;
 
   DecodeParams p{};
   p.B = B;
@@ -298,10 +400,15 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   p.num_pages = cache->cfg.num_pages;
   p.pt_stride = pt_stride;
   p.mask_stride = mask_stride;
-  p.num_workers = nw;
+  p.num_workers = pl.n_cta * pl.HB;
   p.slot_floats = slot_floats(G, D);
   p.slot_o_off = slot_o_off(G);
   p.int8_units = has8 ? 1 : 0;
+  p.HB = pl.HB;
+  p.NVB = pl.NVB;
+  p.NS = pl.NS;
+  p.np8 = side_pages(p.sink, p.recent);
+  p.n_cta = pl.n_cta;
   p.q = static_cast<const __nv_bfloat16 *>(q);
   p.seq_lens = seq_lens;
   p.page_table = page_table;
@@ -316,7 +423,7 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   p.out_fp32 = out_is_fp32 ? 1 : 0;
   p.err = cache->err;
   p.wait_cap = cache->wait_cap;
-  carve_workspace(p, workspace);
+  carve_workspace(p, workspace, (size_t)pl.NVB + 1, (size_t)2 * pl.NVB);
   cudaEvent_t e0, e1;
   timing_pair(0, &e0, &e1);
   return cuda_status(launch_decode(p, D, false, static_cast<cudaStream_t>(stream), e0, e1));
@@ -354,8 +461,8 @@ kv4_status bf16_paged_workspace_bytes(int32_t B, int32_t Hq, int32_t Hkv, int32_
   if ((G != 1 && G != 2 && G != 4) || (D != 64 && D != 128)) return KV4_ERR_UNSUPPORTED;
   DecodeLaunch l{};
   int sms = 0;
-  if (geometry(D, G, true, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
-  *bytes = decode_ws_bytes(B, Hkv, G, D, resolve_workers(num_workers, l, sms));
+  if (bad(bf16_geometry(D, G, &l, &sms))) return KV4_ERR_CUDA;
+  *bytes = bf16_ws_bytes(B, Hkv, G, D, bf16_workers(num_workers, l, sms));
   return KV4_OK;
 }
 
@@ -376,9 +483,9 @@ kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32
   if (!isfinite(softmax_scale)) return KV4_ERR_INVALID;
   DecodeLaunch l{};
   int sms = 0;
-  if (geometry(D, G, true, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
-  const int nw = resolve_workers(num_workers, l, sms);
-  if (ws_bytes < decode_ws_bytes(B, Hkv, G, D, nw)) return KV4_ERR_INVALID;
+  if (bad(bf16_geometry(D, G, &l, &sms))) return KV4_ERR_CUDA;
+  const int nw = bf16_workers(num_workers, l, sms);
+  if (ws_bytes < bf16_ws_bytes(B, Hkv, G, D, nw)) return KV4_ERR_INVALID;
   DecodeParams p{};
   p.B = B;
   p.Hq = Hq;
@@ -401,7 +508,7 @@ kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32
   p.out_fp32 = out_is_fp32 ? 1 : 0;
   p.err = error_word;
   p.wait_cap = kDefaultWaitCycles;
-  carve_workspace(p, workspace);
+  carve_workspace(p, workspace, (size_t)B + 1, (size_t)2 * B * Hkv);
   cudaEvent_t e0, e1;
   timing_pair(1, &e0, &e1);
   return cuda_status(launch_decode(p, D, true, static_cast<cudaStream_t>(stream), e0, e1));
@@ -478,7 +585,7 @@ kv4_status kv4_get_error(kv4_cache *cache, void *stream, uint32_t *bits) {
   cudaError_t e = cudaStreamSynchronize(s);
   if (e == cudaSuccess) e = cudaMemcpy(&w, cache->err, sizeof(w), cudaMemcpyDeviceToHost);
   if (e == cudaSuccess) e = cudaMemset(cache->err, 0, sizeof(uint32_t));
-  if (e != cudaSuccess) return KV4_ERR_CUDA;
+  if (bad(e)) return KV4_ERR_CUDA;
   if (bits) *bits = w;
   if (w & (1u << KV4_ERR_TIMEOUT)) return KV4_ERR_TIMEOUT;
   if (w & (1u << KV4_ERR_BOUNDS)) return KV4_ERR_BOUNDS;
@@ -494,11 +601,18 @@ kv4_status kv4_debug_set_wait_limit(kv4_cache *cache, int64_t cycles) {
 }
 
 kv4_status kv4_device_info(int32_t *num_sms, int32_t *default_workers_out) {
-  DecodeLaunch l{};
-  int sms = 0;
-  if (geometry(128, 4, false, &l, &sms) != cudaSuccess) return KV4_ERR_CUDA;
-  if (num_sms) *num_sms = sms;
-  if (default_workers_out) *default_workers_out = default_workers(l, sms);
+  // the decode kernel at D = 128, 32 query / 8 KV heads, 64 sequences
+  Kv4Plan pl{};
+  const kv4_status st = kv4_plan(128, 4, 8, 64, 0, &pl);
+  if (st != KV4_OK) return st;
+  int dev = 0;
+  DeviceInfo di;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (bad(device_info(&dev, &di))) return KV4_ERR_CUDA;
+  }
+  if (num_sms) *num_sms = di.sms;
+  if (default_workers_out) *default_workers_out = pl.n_cta * pl.HB;
   return KV4_OK;
 }
 
@@ -509,7 +623,7 @@ kv4_status kv4_timing_enable(int32_t max_records, int32_t every) {
   for (int k = 0; k < 2; ++k) {
     g_timing.ev[k].resize(2 * (size_t)max_records, nullptr);
     for (auto &e : g_timing.ev[k]) {
-      if (cudaEventCreate(&e) != cudaSuccess) {
+      if (bad(cudaEventCreate(&e))) {
         timing_free();
         return KV4_ERR_CUDA;
       }
@@ -528,13 +642,29 @@ kv4_status kv4_timing_read(int32_t kind, double *total_ms, int32_t *count) {
   const int n = g_timing.used[kind];
   for (int i = 0; i < n; ++i) {
     float ms = 0.f;
-    if (cudaEventSynchronize(g_timing.ev[kind][2 * i + 1]) != cudaSuccess) return KV4_ERR_CUDA;
-    if (cudaEventElapsedTime(&ms, g_timing.ev[kind][2 * i], g_timing.ev[kind][2 * i + 1]) != cudaSuccess)
+    if (bad(cudaEventSynchronize(g_timing.ev[kind][2 * i + 1]))) return KV4_ERR_CUDA;
+    if (bad(cudaEventElapsedTime(&ms, g_timing.ev[kind][2 * i], g_timing.ev[kind][2 * i + 1])))
       return KV4_ERR_CUDA;
     sum += ms;
   }
   g_timing.used[kind] = 0;
   *total_ms = sum;
+  *count = n;
+  return KV4_OK;
+}
+
+kv4_status kv4_timing_read_each(int32_t kind, float *ms_out, int32_t cap, int32_t *count) {
+  if (kind < 0 || kind > 1 || !count || cap < 0 || (cap > 0 && !ms_out)) return KV4_ERR_INVALID;
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  const int n = g_timing.used[kind];
+  for (int i = 0; i < n; ++i) {
+    float ms = 0.f;
+    if (bad(cudaEventSynchronize(g_timing.ev[kind][2 * i + 1]))) return KV4_ERR_CUDA;
+    if (bad(cudaEventElapsedTime(&ms, g_timing.ev[kind][2 * i], g_timing.ev[kind][2 * i + 1])))
+      return KV4_ERR_CUDA;
+    if (i < cap) ms_out[i] = ms;
+  }
+  g_timing.used[kind] = 0;
   *count = n;
   return KV4_OK;
 }

@@ -7,21 +7,18 @@
 // a retained-position mask is applied inside attention.
 //
 // Two launches on the caller's stream:
-//   decode_kernel  persistent warp workers over one flat, weighted item space:
-//                  first every (sequence, KV head)'s INT8 side pages (16 rows
-//                  each; a sink page and recent/16 ring pages), then every
-//                  (sequence, KV head)'s INT4 pages. Each worker owns one
-//                  contiguous segment. Pages stream through a per-warp ring of
-//                  shared-memory stages filled by 1-D bulk copies (TMA engine,
-//                  mbarrier completion, bounded waits). Per page, q.K and P.V
-//                  are small tensor-core tiles (mma.sync m16n8k16, fp32
-//                  accumulate): q.K of INT4 pages on bf16 tiles (codes
-//                  unpacked in registers), P.V of INT4 pages and all of the
-//                  INT8 pages on fp16 tiles (the codes are exact in fp16).
-//                  Each worker writes one (m, l, o) partial per
-//                  (region, sequence, KV head) piece of its segment.
-//   merge_kernel   (kv4_merge.cu) one warp per (sequence, query head) merges
-//                  its partials exactly.
+//   kv4_decode_kernel  page-major workers: a CTA with one warp per KV head
+//                      streams whole pages (every head of a page in one bulk
+//                      copy, the TMA engine, mbarrier completion, bounded
+//                      waits) and side pages through a ring of shared-memory
+//                      stages shared by its warps. Per page and head, q.K and
+//                      P.V are small tensor-core tiles (mma.sync m16n8k16,
+//                      fp32 accumulate). Each warp writes one (m, l, o)
+//                      partial per (region, sequence) range its CTA touches.
+//   merge_kernel       (kv4_merge.cu) one warp per (sequence, query head)
+//                      merges the partials exactly.
+// The uncompressed comparison (bf16 pages) keeps per-warp workers over
+// (sequence, head) page ranges (bf16_decode_kernel).
 //
 // Softmax bookkeeping runs in the log2 domain (scores scaled by tau*log2 e).
 // P.V takes P*scale_V as two fp16 terms (hi + lo), which carries 22
@@ -34,25 +31,14 @@
 
 namespace kv4 {
 
-#ifndef KV4_INT4_STAGES
-#define KV4_INT4_STAGES 4
-#endif
-#ifndef KV4_MIN_BLOCKS
-#define KV4_MIN_BLOCKS 4
-#endif
-
-template <int D, bool kBF16>
-struct Cfg {
-  static constexpr int NS = kBF16 ? 3 : KV4_INT4_STAGES;    // stages per warp
+// Per-warp ring of the bf16 comparison kernel.
+template <int D>
+struct Bf16Cfg {
+  static constexpr int NS = 3;                              // stages per warp
   static constexpr int ROWB = 2 * D + 16;                   // padded bf16 row in shared memory
-  static constexpr int STAGE = kBF16 ? 2 * kPageTokens * ROWB : 18 * D;
+  static constexpr int STAGE = 2 * kPageTokens * ROWB;
   static constexpr int WARP_SMEM = NS * STAGE;
-  // per-warp query operands: [chunk][lane][16 bytes]; INT4 pieces use D/32
-  // chunks of q fragments and (D/32 + 1)/2 chunks of accumulator starts,
-  // INT8 pieces D/32 chunks of fp16 q fragments
-  static constexpr int QCHUNKS = kBF16 ? 0 : D / 32 + (D / 32 + 1) / 2;
-  static constexpr int QBYTES = QCHUNKS * 512;
-  static constexpr int RINGS = kWarps * (WARP_SMEM + NS * 8 + QBYTES);
+  static constexpr int RINGS = kWarps * (WARP_SMEM + NS * 8);
 };
 
 
@@ -293,365 +279,625 @@ __device__ __forceinline__ int next_page(PageCursor &c, int &pid, const int32_t 
   return -1;
 }
 
-// ---------------------------------------------------------------------------
-// INT4 pages of one piece (sequence b, KV head h, pages [pg0, pg1)).
-// Returns false if a bounded wait ran out (the worker must stop).
+// ===========================================================================
+// KV4 decode kernel: INT4 pages and INT8 side pages, page-major.
 //
-// q.K: A = K codes (rows = slots g, g+8), B = q. Per group two MMAs: a bf16
-// one over elements 32i+8t+{0, 4} (k-slots 2t, 2t+1) and {2, 6} (2t+8, 2t+9),
-// whose codes enter as 136 + c, and an fp16 one over {1, 5} and {3, 7}, whose
-// codes enter as 72 + c -- the nibble order of the K words; one shift by 8
-// serves both. The accumulator starts at -(136 * sum of q over the even
-// elements + 72 * sum over the odd ones), which removes the offsets.
-// P.V: A = V^T codes (rows = head_dim, k = slots), B = P * scale_V (hi + lo).
-// ---------------------------------------------------------------------------
-template <int D, int G>
-__device__ bool int4_piece(const DecodeParams &p, int b, int h, int L, int pg0, int pg1, uint8_t *wsm,
-                           uint64_t *bars, uint8_t *qsm, uint32_t &phase, float *slot, int lane) {
-  using C = Cfg<D, false>;
-  constexpr int NS = C::NS, NG = D / 32, NMT = D / 16, NSW = (NG + 1) / 2;
-  const int g = lane >> 2, t = lane & 3;
+// A CTA has one warp per KV head of a head block (HB heads, HB <= 8; with
+// more KV heads each block of HB heads is a "virtual sequence" vb = hb * B + b
+// of its own). Work items form one flat, ordered space, virtual sequence by
+// virtual sequence: first its INT8 side pages (2 * np8 items, the K half then
+// the V half of each side page), then its INT4 pages in page order. CTA c
+// takes items [c T / nc, (c+1) T / nc), a bound that would part the two
+// halves of a side page moved down by one, so every CTA holds its share of
+// side-page work and both halves of a side page stay in one CTA. An item
+// always covers every head of the block: one bulk copy of the page's HB head
+// blocks (INT4; they are contiguous in a page) or HB copies of one side-page
+// half, into a stage of an NS-stage ring shared by the CTA. Warp hh computes
+// head hh's slice. The warp that releases a stage last (a counter per stage,
+// acquire-release shared atomics) refills it with the item NS places ahead,
+// so nobody waits for a producer and no warp keeps ring or cursor state
+// beyond the stage index. Ranges: (virtual sequence vb, region) has range id
+// 2 * vb (INT8) or 2 * vb + 1 (INT4), increasing along the item space.
+//
+// Item descriptors (kind | vb | page or side page, page id) are prepared per
+// chunk of up to kChunk items by the whole CTA: classification, page-table
+// reads, bounds checks and the skip of pages without an attended position
+// all happen there, in parallel, and the kept items are compacted.
+// ===========================================================================
+constexpr int kChunk = 256;
+constexpr int kItemInt4 = 0, kItemInt8K = 1, kItemInt8V = 2;
 
-  // q as the B operand, and -136 * (sum of q over group i) for columns 2t and
-  // 2t+1, parked in the warp's shared-memory q area for the whole piece
-  {
-    const int head = g & 3;
-    const bool hv = head < G;
-    const uint4 *qh = reinterpret_cast<const uint4 *>(p.q + ((long long)b * p.Hq + h * G + (hv ? head : 0)) * D);
-    float qinit[NG][2];
+// Per-warp query area: D/32 chunks of 512 bytes (the B fragments of the q.K
+// tiles, one 16-byte piece per lane) and, for INT4 ranges, the accumulator
+// start of every (group, query head): D/32 x 4 floats.
+__host__ __device__ constexpr int kv4_q_bytes(int D) { return (D / 32) * 512 + (D / 32) * 16; }
+
+// Shared-memory layout of the KV4 kernel (bytes), for HB heads, NS stages and
+// NVB virtual sequences.
+struct Kv4Layout {
+  int bars, cnt, iss, flag, desc, q, plan, wtot, total;
+};
+
+__host__ __device__ inline Kv4Layout kv4_layout(int D, int HB, int NS, int NVB) {
+  Kv4Layout l;
+  int o = NS * HB * 18 * D;
+  l.bars = o;
+  o += NS * 8;
+  l.cnt = o;   // "empty" mbarriers: every warp arrives when it is done with a stage
+  o += NS * 8;
+  l.iss = o;
+  o += NS * 4;
+  l.flag = o;
+  o += 4;
+  o = (o + 15) & ~15;
+  l.desc = o;
+  o += kChunk * 8;
+  l.q = o;
+  o += HB * kv4_q_bytes(D);
+  l.plan = o;
+  o += (NVB + 1) * 4;
+  l.wtot = o;
+  o += 8 * 4;
+  l.total = o;
+  return l;
+}
+
+// Largest i in [0, n) with a[i] <= y (a non-decreasing, a[0] <= y).
+__device__ __forceinline__ int upper_index(const int *a, int n, long long y) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a[mid] <= y) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Side page j of a sequence of length L holds at least one attended row:
+// the sink page (j < js) when L > 0, a ring page when its 16 slots meet the
+// slots {p mod R : p in [max(S, L - R), L)}, a cyclic run of min(L - S, R).
+__device__ __forceinline__ bool side_page_attended(int j, int L, int S, int R) {
+  const int js = S > 0 ? 1 : 0;
+  if (L <= 0) return false;
+  if (j < js) return true;
+  const int r0 = max(S, L - R), nv = L - r0;
+  if (nv <= 0) return false;
+  if (nv >= R) return true;
+  const int lo = 16 * (j - js), a = r0 % R;
+  return ((lo - a + R) % R) < nv || ((a - lo + R) % R) < 16;
+}
+
+// Descriptor of flat item x, or false if the item has nothing to attend
+// (or names a page outside the pool, which is reported). n8 = INT8 items per
+// virtual sequence (0 without side pages).
+template <int D>
+__device__ bool classify_item(const DecodeParams &p, const int *plan, int n8, long long x, int2 &d) {
+  const int NVB = p.NVB, HB = p.HB, cap = p.pt_stride * kPageTokens;
+  const int vb = upper_index(plan, NVB, x);
+  const int off = static_cast<int>(x - plan[vb]);
+  const int hb = vb / p.B, b = vb - hb * p.B;
+  if (off < n8) {
+    const int j = off >> 1;
+    const int L = eff_len(p.seq_lens[b], cap);
+    if (!side_page_attended(j, L, p.sink, p.recent)) return false;
+    d.x = ((off & 1) ? kItemInt8V : kItemInt8K) | (vb << 2) | (j << 15);
+    d.y = 0;
+    return true;
+  }
+  const int pg = int4_first_page(p.sink) + off - n8;
+  if (p.mask) {
+    const int L = eff_len(p.seq_lens[b], cap);
+    const int lo_tok = p.sink, hi_tok = L - p.recent;
+    const int t0 = max(pg * kPageTokens, lo_tok) - pg * kPageTokens;
+    const int t1 = min(pg * kPageTokens + kPageTokens, hi_tok) - pg * kPageTokens;
+    const uint32_t win = ((t1 >= 16 ? 0xFFFFFFFFu : (1u << t1) - 1u)) & ~((1u << t0) - 1u);
+    uint32_t any = 0;
+    for (int hh = 0; hh < HB; ++hh) {
+      const uint32_t *mrow = p.mask + ((long long)b * p.Hkv + hb * HB + hh) * p.mask_stride;
+      any |= (mrow[pg >> 1] >> ((pg & 1) * 16)) & win;
+    }
+    if (!(any & 0xFFFFu)) return false;
+  }
+  const int pid = p.page_table[(long long)b * p.pt_stride + pg];
+  if (pid < 0 || pid >= p.num_pages) {
+    set_error(p.err, kErrBounds);
+    return false;
+  }
+  d.x = kItemInt4 | (vb << 2) | (pg << 15);
+  d.y = pid;
+  return true;
+}
+
+// Prepare the descriptors of flat items [cx, cx + n): classified in parallel
+// and compacted in order. Returns the number kept (the same in every thread).
+template <int D>
+__device__ int prepare_chunk(const DecodeParams &p, const int *plan, int n8, long long cx, int n, int2 *desc,
+                             int *wtot, int tid, int nthr) {
+  const int warp = tid >> 5, lane = tid & 31, nwarps = nthr >> 5;
+  int base = 0;
+  for (int r = 0; r < n; r += nthr) {
+    const int k = r + tid;
+    int2 d = make_int2(0, 0);
+    const bool keep = k < n && classify_item<D>(p, plan, n8, cx + k, d);
+    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) wtot[warp] = __popc(bal);
+    __syncthreads();
+    int off = base, tot = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const int c = wtot[w];
+      off += w < warp ? c : 0;
+      tot += c;
+    }
+    if (keep) desc[off + __popc(bal & ((1u << lane) - 1u))] = d;
+    __syncthreads();
+    base += tot;
+  }
+  return base;
+}
+
+// Issue the copies of item d into a stage (one thread). INT4: the HB head
+// blocks of the page, contiguous in the pool; INT8: one half of side page j
+// for each of the HB heads.
+template <int D>
+__device__ __forceinline__ void issue_item(const DecodeParams &p, int2 d, uint8_t *stage, uint64_t *bar) {
+  const int kind = d.x & 3, vb = (d.x >> 2) & 0x1FFF, pj = static_cast<int>(static_cast<uint32_t>(d.x) >> 15);
+  const int HB = p.HB, hb = vb / p.B, b = vb - hb * p.B;
+  if (kind == kItemInt4) {
+    const uint32_t bytes = static_cast<uint32_t>(HB * 18 * D);
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_g2s(stage, p.pool + (long long)d.y * p.page_bytes + (long long)hb * HB * p.head_bytes, bytes, bar);
+  } else {
+    constexpr uint32_t KHALF = 16 * D + 64, VHALF = 16 * D;
+    const uint32_t bytes = kind == kItemInt8K ? KHALF : VHALF;
+    const long long off = (long long)pj * (32 * D + 64) + (kind == kItemInt8K ? 0 : KHALF);
+    const uint8_t *src = p.side + ((long long)b * p.Hkv + (long long)hb * HB) * p.side_stride + off;
+    mbar_arrive_expect_tx(bar, bytes * HB);
+    for (int hh = 0; hh < HB; ++hh) bulk_g2s(stage + hh * 18 * D, src + hh * p.side_stride, bytes, bar);
+  }
+}
+
+// First/last CTA of every range met by [x0, x1), and an empty partial
+// (m = -inf, l = 0) for each of its heads, overwritten by the real one when a
+// warp closes the range.
+template <int G>
+__device__ void mark_ranges(const DecodeParams &p, const int *plan, int n8, long long x0, long long x1, int c,
+                            int tid, int nthr) {
+  const int NVB = p.NVB, HB = p.HB;
+  const int va = upper_index(plan, NVB, x0), vz = upper_index(plan, NVB, x1 - 1);
+  const int nr = 2 * (vz - va + 1);
+  for (int i = tid; i < nr * HB * G; i += nthr) {
+    const int ri = i / (HB * G), hh = (i / G) % HB, g = i % G;
+    const int vb = va + (ri >> 1), region = ri & 1;
+    const long long s = (long long)plan[vb] + (region ? n8 : 0);
+    const long long e = region ? (long long)plan[vb + 1] : (long long)plan[vb] + n8;
+    if (s == e || e <= x0 || s >= x1) continue;
+    const int rid = 2 * vb + region;
+    if (hh == 0 && g == 0) {
+      if (s >= x0) p.first[rid] = c;
+      if (e <= x1) p.last[rid] = c;
+    }
+    float *slot = p.slots + ((long long)(rid + c) * HB + hh) * p.slot_floats;
+    slot[g] = -INFINITY;
+    slot[G + g] = 0.f;
+  }
+}
+
+// Query fragments of one (virtual sequence, head) into the warp's q area.
+// INT4 format (per group i, 512 bytes): q as the B operand of the two q.K
+// tiles -- bf16 pairs of the even elements, fp16 pairs of the odd ones --
+// then, after the NG group chunks, a table [group][query head] of the
+// accumulator starts -(136 * sum of even q + 72 * sum of odd q).
+// INT8 format: fp16 fragments of the D/16 tiles of the side-page q.K.
+// Every query element must lie in the fp16 range (it enters fp16 tiles);
+// one that does not is reported as KV4_ERR_RANGE.
+template <int D, int G>
+__device__ __forceinline__ void load_q(const DecodeParams &p, int b, int h, bool int4, uint8_t *qsm, int lane) {
+  constexpr int NG = D / 32;
+  const int g = lane >> 2, t = lane & 3;
+  const int head = g & 3;
+  const bool hv = head < G;
+  const __nv_bfloat16 *qrow = p.q + ((long long)b * p.Hq + h * G + (hv ? head : 0)) * D;
+  bool big = false;
+  if (int4) {
+    const uint4 *qh = reinterpret_cast<const uint4 *>(qrow);
 #pragma unroll
     for (int i = 0; i < NG; ++i) {
       const uint4 e = hv ? qh[4 * i + t] : make_uint4(0, 0, 0, 0);
-      // e.x = (e0, e1), e.y = (e2, e3), e.z = (e4, e5), e.w = (e6, e7)
-      // e.x = (e0, e1), e.y = (e2, e3), e.z = (e4, e5), e.w = (e6, e7). Codes of
-      // even elements enter a bf16 MMA as 136 + c, codes of odd elements an
-      // fp16 MMA as 72 + c (see the q.K below), so the bf16 pairs (e0, e4),
-      // (e2, e6) and the fp16 pairs (e1, e5), (e3, e7) are stored.
       const float e0 = bf16lo_to_f32(e.x), e1 = bf16hi_to_f32(e.x), e2 = bf16lo_to_f32(e.y), e3 = bf16hi_to_f32(e.y);
       const float e4 = bf16lo_to_f32(e.z), e5 = bf16hi_to_f32(e.z), e6 = bf16lo_to_f32(e.w), e7 = bf16hi_to_f32(e.w);
+      const float mx = fmaxf(fmaxf(fmaxf(fabsf(e0), fabsf(e1)), fmaxf(fabsf(e2), fabsf(e3))),
+                             fmaxf(fmaxf(fabsf(e4), fabsf(e5)), fmaxf(fabsf(e6), fabsf(e7))));
+      big |= !(mx <= 65504.f);
       *reinterpret_cast<uint4 *>(qsm + i * 512 + lane * 16) =
           make_uint4(__byte_perm(e.x, e.z, 0x5410), __byte_perm(e.y, e.w, 0x5410), pack_f16x2(e1, e5),
                      pack_f16x2(e3, e7));
       float part = -136.f * ((e0 + e2) + (e4 + e6)) - 72.f * ((e1 + e3) + (e5 + e7));
       part += __shfl_xor_sync(0xffffffffu, part, 1);
       part += __shfl_xor_sync(0xffffffffu, part, 2);
-      // lanes 4c..4c+3 hold the group offset of column c; this lane needs columns 2t, 2t+1
-      qinit[i][0] = __shfl_sync(0xffffffffu, part, 8 * t);
-      qinit[i][1] = __shfl_sync(0xffffffffu, part, 8 * t + 4);
+      // lanes 4c..4c+3 now hold the offset of column c, i.e. of query head c & 3
+      if (t == 0 && g < 4) reinterpret_cast<float *>(qsm + NG * 512)[4 * i + g] = part;
     }
-#pragma unroll
-    for (int c = 0; c < (NG + 1) / 2; ++c) {
-      const float a0 = qinit[2 * c][0], a1 = qinit[2 * c][1];
-      const float a2 = 2 * c + 1 < NG ? qinit[(2 * c + 1) % NG][0] : 0.f;
-      const float a3 = 2 * c + 1 < NG ? qinit[(2 * c + 1) % NG][1] : 0.f;
-      *reinterpret_cast<float4 *>(qsm + (NG + c) * 512 + lane * 16) = make_float4(a0, a1, a2, a3);
-    }
-    __syncwarp();
-  }
-
-  const int lo_tok = p.sink, hi_tok = L - p.recent;
-  const uint32_t *mrow = p.mask ? p.mask + ((long long)b * p.Hkv + h) * p.mask_stride : nullptr;
-  const int32_t *ptrow = p.page_table + (long long)b * p.pt_stride;
-  const uint8_t *hbase = p.pool + (long long)h * p.head_bytes;
-  const float2 neg_sel = t >= 2 ? make_float2(-1.f, -1.f) : make_float2(0.f, 0.f);
-
-  SoftmaxState<NMT> st;
-  st.reset();
-  PageCursor cur;
-  cur.pg1 = pg1;
-  cur.cursor = pg0;
-  load_batch(cur, pg0, ptrow, lo_tok, hi_tok, mrow, p, lane);
-
-  Ring<NS> ring;
-  ring.s = 0;
-#pragma unroll
-  for (int k = 0; k < NS; ++k) {
-    int pid = -1;
-    ring.item[k] = next_page(cur, pid, ptrow, lo_tok, hi_tok, mrow, p, lane);
-    if (ring.item[k] >= 0 && lane == 0) {
-      mbar_arrive_expect_tx(&bars[k], C::STAGE);
-      bulk_g2s(wsm + k * C::STAGE, hbase + (long long)pid * p.page_bytes, C::STAGE, &bars[k]);
-    }
-  }
-
-  while (ring.item[0] >= 0) {
-    if (!ring_wait<NS>(ring, bars, phase, p.wait_cap, p.err, lane)) return false;
-    const uint8_t *stg = wsm + ring.s * C::STAGE;
-    const int pg = ring.item[0];
-
-    // ---- q.K
-    uint32_t kw0[NG], kw1[NG], ksw0[NSW], ksw1[NSW], vsw0[NSW], vsw1[NSW];
-    if constexpr (NG == 4) {
-      const uint4 a0 = *reinterpret_cast<const uint4 *>(stg + g * (D / 2) + t * (D / 8));
-      const uint4 a1 = *reinterpret_cast<const uint4 *>(stg + (g + 8) * (D / 2) + t * (D / 8));
-      kw0[0] = a0.x; kw0[1] = a0.y; kw0[2] = a0.z; kw0[3] = a0.w;
-      kw1[0] = a1.x; kw1[1] = a1.y; kw1[2] = a1.z; kw1[3] = a1.w;
-      const uint2 s0 = *reinterpret_cast<const uint2 *>(stg + 16 * D + g * 8);
-      const uint2 s1 = *reinterpret_cast<const uint2 *>(stg + 16 * D + (g + 8) * 8);
-      const uint2 u0 = *reinterpret_cast<const uint2 *>(stg + 17 * D + g * 8);
-      const uint2 u1 = *reinterpret_cast<const uint2 *>(stg + 17 * D + (g + 8) * 8);
-      ksw0[0] = s0.x; ksw0[1] = s0.y; ksw1[0] = s1.x; ksw1[1] = s1.y;
-      vsw0[0] = u0.x; vsw0[1] = u0.y; vsw1[0] = u1.x; vsw1[1] = u1.y;
-    } else {
-      const uint2 a0 = *reinterpret_cast<const uint2 *>(stg + g * (D / 2) + t * (D / 8));
-      const uint2 a1 = *reinterpret_cast<const uint2 *>(stg + (g + 8) * (D / 2) + t * (D / 8));
-      kw0[0] = a0.x; kw0[1] = a0.y;
-      kw1[0] = a1.x; kw1[1] = a1.y;
-      ksw0[0] = *reinterpret_cast<const uint32_t *>(stg + 16 * D + g * 4);
-      ksw1[0] = *reinterpret_cast<const uint32_t *>(stg + 16 * D + (g + 8) * 4);
-      vsw0[0] = *reinterpret_cast<const uint32_t *>(stg + 17 * D + g * 4);
-      vsw1[0] = *reinterpret_cast<const uint32_t *>(stg + 17 * D + (g + 8) * 4);
-    }
-    float ks0[NG], ks1[NG], vs0a[NG], vs1a[NG];
-#pragma unroll
-    for (int c = 0; c < NSW; ++c) {
-      const float2 a0 = f16x2_to_f32x2(ksw0[c]), a1 = f16x2_to_f32x2(ksw1[c]);
-      const float2 b0 = f16x2_to_f32x2(vsw0[c]), b1 = f16x2_to_f32x2(vsw1[c]);
-      ks0[2 * c] = a0.x; ks1[2 * c] = a1.x; vs0a[2 * c] = b0.x; vs1a[2 * c] = b1.x;
-      if (2 * c + 1 < NG) {
-        ks0[2 * c + 1] = a0.y; ks1[2 * c + 1] = a1.y; vs0a[2 * c + 1] = b0.y; vs1a[2 * c + 1] = b1.y;
-      }
-    }
-    float2 sc01 = make_float2(0.f, 0.f), sc23 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < NG; ++i) {
-      const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + i * 512 + lane * 16);
-      const float2 qi = *reinterpret_cast<const float2 *>(qsm + (NG + i / 2) * 512 + lane * 16 + (i & 1) * 8);
-      float acc[4] = {qi.x, qi.y, qi.x, qi.y};
-      const uint32_t k80 = kw0[i] >> 8, k81 = kw1[i] >> 8;
-      {   // elements 0, 4 (k-slots 2t, 2t+1) and 2, 6 (2t+8, 2t+9): bf16, 136 + c
-        const uint32_t a[4] = {i4x2_biased(kw0[i]), i4x2_biased(kw1[i]), i4x2_biased(k80), i4x2_biased(k81)};
-        mma_bf16(acc, a, qv.x, qv.y);
-      }
-      {   // elements 1, 5 and 3, 7: fp16, 72 + c (bits 4-7 convert in place)
-        const uint32_t a[4] = {i4x2_hi_biased_f16(kw0[i]), i4x2_hi_biased_f16(kw1[i]), i4x2_hi_biased_f16(k80),
-                               i4x2_hi_biased_f16(k81)};
-        mma_f16(acc, a, qv.z, qv.w);
-      }
-      const float k0 = ks0[i], k1 = ks1[i];
-      sc01 = __ffma2_rn(make_float2(k0, k0), make_float2(acc[0], acc[1]), sc01);
-      sc23 = __ffma2_rn(make_float2(k1, k1), make_float2(acc[2], acc[3]), sc23);
-    }
-    // ---- which of the page's slots are attended (all of them on interior pages)
-    const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
-    sc01 = __fmul2_rn(sc01, sl2);
-    sc23 = __fmul2_rn(sc23, sl2);
-    float sl[4] = {sc01.x, sc01.y, sc23.x, sc23.y};
-    if (mrow || pg * kPageTokens < lo_tok || pg * kPageTokens + kPageTokens > hi_tok) {
-      const int tok0 = pg * kPageTokens + g, tok1 = tok0 + 8;
-      bool v0 = tok0 >= lo_tok && tok0 < hi_tok;
-      bool v1 = tok1 >= lo_tok && tok1 < hi_tok;
-      if (mrow) {
-        const uint32_t mw = mrow[pg >> 1] >> ((pg & 1) * 16);
-        v0 = v0 && ((mw >> g) & 1u);
-        v1 = v1 && ((mw >> (g + 8)) & 1u);
-      }
-      if (!v0) sl[0] = sl[1] = -INFINITY;
-      if (!v1) sl[2] = sl[3] = -INFINITY;
-    }
-    // exact running max: probabilities <= 1, so P * scale_V fits fp16
-    float pr[4];
-    softmax_update<NMT, 0>(st, sl, pr);
-
-    // ---- P.V
-    uint32_t wb[NG][2];
-#pragma unroll
-    for (int i = 0; i < NG; ++i) {
-      const float vs0 = vs0a[i], vs1 = vs1a[i];
-      weights_f16x2(__fmul2_rn(make_float2(pr[0], pr[1]), make_float2(vs0, vs0)),
-                    __fmul2_rn(make_float2(pr[2], pr[3]), make_float2(vs1, vs1)), neg_sel, wb[i][0], wb[i][1]);
-    }
-    uint32_t vw[NMT];
-#pragma unroll
-    for (int q4 = 0; q4 < NMT / 4; ++q4) {
-      const uint4 w = *reinterpret_cast<const uint4 *>(stg + 8 * D + q4 * 512 + lane * 16);
-      vw[4 * q4 + 0] = w.x;
-      vw[4 * q4 + 1] = w.y;
-      vw[4 * q4 + 2] = w.z;
-      vw[4 * q4 + 3] = w.w;
-    }
-#pragma unroll
-    for (int mt = 0; mt < NMT; ++mt) {
-      const uint32_t v8 = vw[mt] >> 8;
-      const uint32_t a[4] = {i4x2_lo_to_f16x2(vw[mt]), i4x2_hi_to_f16x2(vw[mt]), i4x2_lo_to_f16x2(v8),
-                             i4x2_hi_to_f16x2(v8)};
-      mma_f16(st.o[mt], a, wb[mt >> 1][0], wb[mt >> 1][1]);
-    }
-
-    // ---- refill this stage
-    __syncwarp();
-    int pid = -1;
-    const int nxt = next_page(cur, pid, ptrow, lo_tok, hi_tok, mrow, p, lane);
-    if (nxt >= 0 && lane == 0) {
-      fence_proxy_async();
-      mbar_arrive_expect_tx(&bars[ring.s], C::STAGE);
-      bulk_g2s(wsm + ring.s * C::STAGE, hbase + (long long)pid * p.page_bytes, C::STAGE, &bars[ring.s]);
-    }
-    ring.push_rotate(nxt);
-  }
-  write_partial<D, NMT>(p, st, slot, lane);
-  return true;
-}
-
-// ---------------------------------------------------------------------------
-// INT8 side pages [j0, j1) of one (sequence b, KV head h): fp16 tensor-core
-// tiles. Each page streams as two items: the K half (codes + both scale
-// arrays) and the V half (codes).
-//
-// q.K: A = int8 K codes (exact in fp16; LOP3 gives 1152 + c, one HSUB2
-// removes 1152), B = q in fp16. With one scale per row, any element order is
-// allowed: MMA j covers elements tD/4 + 4j + {0, 2} (k-slots 2t, 2t+1) and
-// tD/4 + 4j + {1, 3} (k-slots 2t+8, 2t+9).
-// P.V: A = V^T codes (fp16), B = P * scale_V (fp16 hi + lo). The running max
-// is exact (P <= 1), so P * scale_V never exceeds the fp16 range.
-// ---------------------------------------------------------------------------
-template <int D, int G>
-__device__ bool int8_piece(const DecodeParams &p, int b, int h, int L, int j0, int j1, uint8_t *wsm,
-                           uint64_t *bars, uint8_t *qsm, uint32_t &phase, float *slot, int lane) {
-  using C = Cfg<D, false>;
-  constexpr int NS = C::NS, NJ = D / 16, NMT = D / 16, NW = D / 8;   // MMAs, M-tiles, words per lane
-  constexpr int KHALF = 16 * D + 64, VHALF = 16 * D;
-  const int g = lane >> 2, t = lane & 3;
-  const int S = p.sink, R = p.recent;
-  const int js = S > 0 ? 1 : 0;
-  const int r0 = max(S, L - R);
-
-  // fp16 q fragments of MMA j at q area chunk j/2, words 2*(j%2) + {0, 1}
-  {
-    const int head = g & 3;
-    const bool hv = head < G;
-    const uint32_t *qh =
-        reinterpret_cast<const uint32_t *>(p.q + ((long long)b * p.Hq + h * G + (hv ? head : 0)) * D);
+  } else {
+    constexpr int NJ = D / 16;
+    const uint32_t *qh = reinterpret_cast<const uint32_t *>(qrow);
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       const int d = t * (D / 4) + 4 * j;
       const uint32_t e01 = hv ? qh[d / 2] : 0u, e23 = hv ? qh[d / 2 + 1] : 0u;
+      const float x0 = bf16lo_to_f32(e01), x1 = bf16hi_to_f32(e01), x2 = bf16lo_to_f32(e23), x3 = bf16hi_to_f32(e23);
+      big |= !(fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3))) <= 65504.f);
       *reinterpret_cast<uint2 *>(qsm + (j / 2) * 512 + lane * 16 + (j % 2) * 8) =
-          make_uint2(pack_f16x2(bf16lo_to_f32(e01), bf16lo_to_f32(e23)),    // (q[d], q[d+2])
-                     pack_f16x2(bf16hi_to_f32(e01), bf16hi_to_f32(e23)));   // (q[d+1], q[d+3])
+          make_uint2(pack_f16x2(x0, x2), pack_f16x2(x1, x3));
     }
-    __syncwarp();
   }
-  const uint32_t *mrow = p.mask ? p.mask + ((long long)b * p.Hkv + h) * p.mask_stride : nullptr;
-  const uint8_t *blk = p.side + ((long long)b * p.Hkv + h) * p.side_stride;
-  const long long page_bytes8 = 32LL * D + 64;
-  const float lo_sel = t >= 2 ? 1.f : 0.f;
-  (void)G;
+  if (__any_sync(0xffffffffu, big) && lane == 0) set_error(p.err, kErrRange);
+  __syncwarp();
+}
 
-  // position held by row r of page j, or -1 when the row is not attended
-  auto row_pos = [&](int j, int r) -> int {
-    int pos;
-    if (j < js) {
-      pos = r < min(S, L) ? r : -1;
-    } else {
-      const int slotr = 16 * (j - js) + r;
-      const int off = ((slotr - r0) % R + R) % R;
-      pos = r0 + off < L ? r0 + off : -1;
+// Per-range context of a warp.
+struct RangeCtx {
+  int b, h, L, lo_tok, hi_tok, r0;
+  const uint32_t *mrow;
+};
+
+// One INT4 page of head h: q.K on bf16/fp16 tiles with offset codes (the
+// accumulator start removes the offsets), exact running-max softmax, P.V on
+// fp16 tiles with V^T codes and P * scale_V as hi + lo fp16 columns.
+template <int D, int G>
+__device__ __forceinline__ void int4_item(const DecodeParams &p, const uint8_t *stg, const uint8_t *qsm, int pg,
+                                          const RangeCtx &rc, SoftmaxState<D / 16> &st, int lane) {
+  constexpr int NG = D / 32, NMT = D / 16, NSW = (NG + 1) / 2;
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t kw0[NG], kw1[NG], ksw0[NSW], ksw1[NSW], vsw0[NSW], vsw1[NSW];
+  if constexpr (NG == 4) {
+    const uint4 a0 = *reinterpret_cast<const uint4 *>(stg + g * (D / 2) + t * (D / 8));
+    const uint4 a1 = *reinterpret_cast<const uint4 *>(stg + (g + 8) * (D / 2) + t * (D / 8));
+    kw0[0] = a0.x; kw0[1] = a0.y; kw0[2] = a0.z; kw0[3] = a0.w;
+    kw1[0] = a1.x; kw1[1] = a1.y; kw1[2] = a1.z; kw1[3] = a1.w;
+    const uint2 s0 = *reinterpret_cast<const uint2 *>(stg + 16 * D + g * 8);
+    const uint2 s1 = *reinterpret_cast<const uint2 *>(stg + 16 * D + (g + 8) * 8);
+    const uint2 u0 = *reinterpret_cast<const uint2 *>(stg + 17 * D + g * 8);
+    const uint2 u1 = *reinterpret_cast<const uint2 *>(stg + 17 * D + (g + 8) * 8);
+    ksw0[0] = s0.x; ksw0[1] = s0.y; ksw1[0] = s1.x; ksw1[1] = s1.y;
+    vsw0[0] = u0.x; vsw0[1] = u0.y; vsw1[0] = u1.x; vsw1[1] = u1.y;
+  } else {
+    const uint2 a0 = *reinterpret_cast<const uint2 *>(stg + g * (D / 2) + t * (D / 8));
+    const uint2 a1 = *reinterpret_cast<const uint2 *>(stg + (g + 8) * (D / 2) + t * (D / 8));
+    kw0[0] = a0.x; kw0[1] = a0.y;
+    kw1[0] = a1.x; kw1[1] = a1.y;
+    ksw0[0] = *reinterpret_cast<const uint32_t *>(stg + 16 * D + g * 4);
+    ksw1[0] = *reinterpret_cast<const uint32_t *>(stg + 16 * D + (g + 8) * 4);
+    vsw0[0] = *reinterpret_cast<const uint32_t *>(stg + 17 * D + g * 4);
+    vsw1[0] = *reinterpret_cast<const uint32_t *>(stg + 17 * D + (g + 8) * 4);
+  }
+  float ks0[NG], ks1[NG], vs0a[NG], vs1a[NG];
+#pragma unroll
+  for (int c = 0; c < NSW; ++c) {
+    const float2 a0 = f16x2_to_f32x2(ksw0[c]), a1 = f16x2_to_f32x2(ksw1[c]);
+    const float2 b0 = f16x2_to_f32x2(vsw0[c]), b1 = f16x2_to_f32x2(vsw1[c]);
+    ks0[2 * c] = a0.x; ks1[2 * c] = a1.x; vs0a[2 * c] = b0.x; vs1a[2 * c] = b1.x;
+    if (2 * c + 1 < NG) {
+      ks0[2 * c + 1] = a0.y; ks1[2 * c + 1] = a1.y; vs0a[2 * c + 1] = b0.y; vs1a[2 * c + 1] = b1.y;
     }
-    if (pos >= 0 && mrow && !((mrow[pos >> 5] >> (pos & 31)) & 1u)) pos = -1;
-    return pos;
+  }
+  float2 sc01 = make_float2(0.f, 0.f), sc23 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < NG; ++i) {
+    const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + i * 512 + lane * 16);
+    // accumulator start of columns 2t, 2t+1 (query heads 2t & 3, (2t & 3) + 1)
+    const float2 qi = *reinterpret_cast<const float2 *>(qsm + NG * 512 + 16 * i + 8 * (t & 1));
+    float acc[4];
+    const uint32_t k80 = kw0[i] >> 8, k81 = kw1[i] >> 8;
+    {   // elements 0, 4 (k-slots 2t, 2t+1) and 2, 6 (2t+8, 2t+9): bf16, 136 + c
+      const uint32_t a[4] = {i4x2_biased(kw0[i]), i4x2_biased(kw1[i]), i4x2_biased(k80), i4x2_biased(k81)};
+      mma_bf16_c(acc, a, qv.x, qv.y, qi.x, qi.y);
+    }
+    {   // elements 1, 5 and 3, 7: fp16, 72 + c (bits 4-7 convert in place)
+      const uint32_t a[4] = {i4x2_hi_biased_f16(kw0[i]), i4x2_hi_biased_f16(kw1[i]), i4x2_hi_biased_f16(k80),
+                             i4x2_hi_biased_f16(k81)};
+      mma_f16(acc, a, qv.z, qv.w);
+    }
+    const float k0 = ks0[i], k1 = ks1[i];
+    sc01 = __ffma2_rn(make_float2(k0, k0), make_float2(acc[0], acc[1]), sc01);
+    sc23 = __ffma2_rn(make_float2(k1, k1), make_float2(acc[2], acc[3]), sc23);
+  }
+  const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+  sc01 = __fmul2_rn(sc01, sl2);
+  sc23 = __fmul2_rn(sc23, sl2);
+  float sl[4] = {sc01.x, sc01.y, sc23.x, sc23.y};
+  // which of the page's slots are attended (all of them on interior pages)
+  if (rc.mrow || pg * kPageTokens < rc.lo_tok || pg * kPageTokens + kPageTokens > rc.hi_tok) {
+    const int tok0 = pg * kPageTokens + g, tok1 = tok0 + 8;
+    bool v0 = tok0 >= rc.lo_tok && tok0 < rc.hi_tok;
+    bool v1 = tok1 >= rc.lo_tok && tok1 < rc.hi_tok;
+    if (rc.mrow) {
+      const uint32_t mw = rc.mrow[pg >> 1] >> ((pg & 1) * 16);
+      v0 = v0 && ((mw >> g) & 1u);
+      v1 = v1 && ((mw >> (g + 8)) & 1u);
+    }
+    if (!v0) sl[0] = sl[1] = -INFINITY;
+    if (!v1) sl[2] = sl[3] = -INFINITY;
+  }
+  float pr[4];
+  softmax_update<NMT, 0>(st, sl, pr);
+
+  const float2 neg_sel = t >= 2 ? make_float2(-1.f, -1.f) : make_float2(0.f, 0.f);
+  uint32_t wb[NG][2];
+#pragma unroll
+  for (int i = 0; i < NG; ++i) {
+    const float vs0 = vs0a[i], vs1 = vs1a[i];
+    weights_f16x2(__fmul2_rn(make_float2(pr[0], pr[1]), make_float2(vs0, vs0)),
+                  __fmul2_rn(make_float2(pr[2], pr[3]), make_float2(vs1, vs1)), neg_sel, wb[i][0], wb[i][1]);
+  }
+  uint32_t vw[NMT];
+#pragma unroll
+  for (int q4 = 0; q4 < NMT / 4; ++q4) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(stg + 8 * D + q4 * 512 + lane * 16);
+    vw[4 * q4 + 0] = w.x;
+    vw[4 * q4 + 1] = w.y;
+    vw[4 * q4 + 2] = w.z;
+    vw[4 * q4 + 3] = w.w;
+  }
+#pragma unroll
+  for (int mt = 0; mt < NMT; ++mt) {
+    const uint32_t v8 = vw[mt] >> 8;
+    const uint32_t a[4] = {i4x2_lo_to_f16x2(vw[mt]), i4x2_hi_to_f16x2(vw[mt]), i4x2_lo_to_f16x2(v8),
+                           i4x2_hi_to_f16x2(v8)};
+    mma_f16(st.o[mt], a, wb[mt >> 1][0], wb[mt >> 1][1]);
+  }
+}
+
+// Position held by row r of side page j for the range, or -1 when the row is
+// not attended (unused slot, or not retained by the mask).
+__device__ __forceinline__ int side_row_pos(const DecodeParams &p, const RangeCtx &rc, int j, int r) {
+  const int S = p.sink, R = p.recent, js = S > 0 ? 1 : 0;
+  int pos;
+  if (j < js) {
+    pos = r < min(S, rc.L) ? r : -1;
+  } else {
+    const int slotr = 16 * (j - js) + r;
+    const int off = ((slotr - rc.r0) % R + R) % R;
+    pos = rc.r0 + off < rc.L ? rc.r0 + off : -1;
+  }
+  if (pos >= 0 && rc.mrow && !((rc.mrow[pos >> 5] >> (pos & 31)) & 1u)) pos = -1;
+  return pos;
+}
+
+// K half of INT8 side page j: q.K on fp16 tiles (codes exact in fp16), softmax,
+// and the P * scale_V weights (hi + lo) kept for the V half that follows.
+template <int D>
+__device__ __forceinline__ void int8k_item(const DecodeParams &p, const uint8_t *stg, const uint8_t *qsm, int j,
+                                           const RangeCtx &rc, SoftmaxState<D / 16> &st, uint32_t &wb0,
+                                           uint32_t &wb1, int lane) {
+  constexpr int NJ = D / 16, NMT = D / 16, NW = D / 8;
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t kw[NW];
+#pragma unroll
+  for (int c = 0; c < NW / 4; ++c) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(stg + c * 512 + lane * 16);
+    kw[4 * c + 0] = w.x;
+    kw[4 * c + 1] = w.y;
+    kw[4 * c + 2] = w.z;
+    kw[4 * c + 3] = w.w;
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int jj = 0; jj < NJ; jj += 2) {
+    const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + (jj / 2) * 512 + lane * 16);
+    const uint32_t a0[4] = {i8x2_to_f16x2(kw[jj]), i8x2_to_f16x2(kw[NJ + jj]), i8x2_to_f16x2(kw[jj] >> 8),
+                            i8x2_to_f16x2(kw[NJ + jj] >> 8)};
+    mma_f16(acc, a0, qv.x, qv.y);
+    const uint32_t a1[4] = {i8x2_to_f16x2(kw[jj + 1]), i8x2_to_f16x2(kw[NJ + jj + 1]),
+                            i8x2_to_f16x2(kw[jj + 1] >> 8), i8x2_to_f16x2(kw[NJ + jj + 1] >> 8)};
+    mma_f16(acc, a1, qv.z, qv.w);
+  }
+  const __half *ks = reinterpret_cast<const __half *>(stg + 16 * D);
+  const __half *vs = reinterpret_cast<const __half *>(stg + 16 * D + 32);
+  const float k0 = __half2float(ks[g]) * p.scale_log2, k1 = __half2float(ks[g + 8]) * p.scale_log2;
+  const bool v0 = side_row_pos(p, rc, j, g) >= 0, v1 = side_row_pos(p, rc, j, g + 8) >= 0;
+  float sl[4];
+  sl[0] = v0 ? acc[0] * k0 : -INFINITY;
+  sl[1] = v0 ? acc[1] * k0 : -INFINITY;
+  sl[2] = v1 ? acc[2] * k1 : -INFINITY;
+  sl[3] = v1 ? acc[3] * k1 : -INFINITY;
+  float pr[4];
+  softmax_update<NMT, 0>(st, sl, pr);
+  const float s0 = __half2float(vs[g]), s1 = __half2float(vs[g + 8]);
+  weights_f16(pr[0] * s0, pr[1] * s0, pr[2] * s1, pr[3] * s1, t >= 2 ? 1.f : 0.f, wb0, wb1);
+}
+
+// V half of an INT8 side page: P.V on fp16 tiles with the weights of the K half.
+template <int D>
+__device__ __forceinline__ void int8v_item(const uint8_t *stg, SoftmaxState<D / 16> &st, uint32_t wb0, uint32_t wb1,
+                                           int lane) {
+  constexpr int NMT = D / 16, NW = D / 8;
+  uint32_t vw[NW];
+#pragma unroll
+  for (int c = 0; c < NW / 4; ++c) {
+    const uint4 w = *reinterpret_cast<const uint4 *>(stg + c * 512 + lane * 16);
+    vw[4 * c + 0] = w.x;
+    vw[4 * c + 1] = w.y;
+    vw[4 * c + 2] = w.z;
+    vw[4 * c + 3] = w.w;
+  }
+#pragma unroll
+  for (int mt = 0; mt < NMT; ++mt) {
+    const uint32_t a[4] = {i8x2_to_f16x2(vw[2 * mt]), i8x2_to_f16x2(vw[2 * mt] >> 8),
+                           i8x2_to_f16x2(vw[2 * mt + 1]), i8x2_to_f16x2(vw[2 * mt + 1] >> 8)};
+    mma_f16(st.o[mt], a, wb0, wb1);
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
+  constexpr int NMT = D / 16, QB = kv4_q_bytes(D);
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nthr = blockDim.x, HB = p.HB, NS = p.NS, NVB = p.NVB;
+  const Kv4Layout lay = kv4_layout(D, HB, NS, NVB);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + lay.bars);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(smem + lay.cnt);
+  uint32_t *iss = reinterpret_cast<uint32_t *>(smem + lay.iss);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + lay.flag);
+  int2 *desc = reinterpret_cast<int2 *>(smem + lay.desc);
+  uint8_t *qsm = smem + lay.q + warp * QB;
+  int *plan = reinterpret_cast<int *>(smem + lay.plan);   // [NVB + 1]
+  int *wtot = reinterpret_cast<int *>(smem + lay.wtot);   // [8]
+  const int stage_bytes = HB * 18 * D;
+
+  if (tid < NS) {
+    mbar_init(&full[tid], 1);
+    mbar_init(&empty[tid], HB);
+    fence_mbar_init();
+    iss[tid] = 0;
+  }
+  if (tid == 0) *abort_flag = 0;
+  pdl_wait();                 // inputs and cache writes of earlier grids are visible from here
+  pdl_launch_dependents();    // the merge grid may queue behind the workers
+
+  // plan[vb] = first item of virtual sequence vb: n8 INT8 items and its INT4
+  // pages per virtual sequence before it
+  const int cap = p.pt_stride * kPageTokens;
+  const int n8 = p.int8_units ? 2 * p.np8 : 0;
+  {
+    const int chunk = (NVB + nthr - 1) / nthr;
+    const int v0 = min(NVB, tid * chunk), v1 = min(NVB, v0 + chunk);
+    int mine = 0;
+    for (int vb = v0; vb < v1; ++vb)
+      mine += n8 + int4_num_pages(eff_len(p.seq_lens[vb % p.B], cap), p.sink, p.recent);
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wtot[warp] = incl;
+    __syncthreads();
+    int run = incl - mine;
+    for (int w = 0; w < warp; ++w) run += wtot[w];
+    for (int vb = v0; vb < v1; ++vb) {
+      plan[vb] = run;
+      run += n8 + int4_num_pages(eff_len(p.seq_lens[vb % p.B], cap), p.sink, p.recent);
+    }
+    if (tid == nthr - 1) plan[NVB] = run;
+    __syncthreads();
+  }
+  if (blockIdx.x == 0) {
+    for (int vb = tid; vb <= NVB; vb += nthr) p.plan[vb] = plan[vb];
+    for (int b = tid; b < p.B; b += nthr)
+      if (p.seq_lens[b] < 0 || p.seq_lens[b] > cap) set_error(p.err, kErrCapacity);
+  }
+  const long long T = plan[NVB];
+  if (T == 0) return;
+  // at most T/2 CTAs, so that every segment keeps >= 1 item after a bound
+  // inside a side page moves down by one
+  const long long nc = min((long long)gridDim.x, max(1LL, T >> 1));
+  if ((long long)blockIdx.x >= nc) return;
+  const int c = blockIdx.x;
+  auto bound = [&](long long x) -> long long {
+    if (x >= T) return T;
+    const int vb = upper_index(plan, NVB, x);
+    const long long off = x - plan[vb];
+    return (off < n8 && (off & 1)) ? x - 1 : x;
   };
+  const long long x0 = bound((long long)c * T / nc), x1 = bound((long long)(c + 1) * T / nc);
 
   SoftmaxState<NMT> st;
   st.reset();
-  // item = 2*j + half; pages without an attended row are skipped
-  int cursor = 2 * j0;
-  auto next_item = [&]() -> int {
-    while (cursor < 2 * j1) {
-      const int it = cursor++;
-      if (it & 1) return it;
-      const bool any = __any_sync(0xffffffffu, lane < 16 && row_pos(it >> 1, lane) >= 0);
-      if (any) return it;
-      ++cursor;   // skip this page's V half too
+  RangeCtx rc{};
+  int cur = -1;              // open range: region * NVB + vb
+  uint32_t wb0 = 0, wb1 = 0;  // INT8 weights, K half -> V half
+  int s = 0, rnd = 0;        // ring stage of the next item, and how often the ring went round
+  uint32_t phase = 0;
+  for (long long cx = x0; cx < x1; cx += kChunk) {
+    __syncthreads();         // previous chunk consumed; empty partials written
+    if (*abort_flag) break;
+    const int n = static_cast<int>(min((long long)kChunk, x1 - cx));
+    const int m = prepare_chunk<D>(p, plan, n8, cx, n, desc, wtot, tid, nthr);
+    if (warp == 0 && lane < min(NS, m)) {
+      const int sl = (s + lane) % NS;
+      iss[sl] += 1;
+      fence_proxy_async();
+      issue_item<D>(p, desc[lane], smem + sl * stage_bytes, &full[sl]);
     }
-    return -1;
-  };
-  auto issue = [&](int stage, int it) {
-    if (lane == 0) {
-      const uint8_t *src = blk + (long long)(it >> 1) * page_bytes8 + ((it & 1) ? KHALF : 0);
-      const uint32_t bytes = (it & 1) ? VHALF : KHALF;
-      mbar_arrive_expect_tx(&bars[stage], bytes);
-      bulk_g2s(wsm + stage * C::STAGE, src, bytes, &bars[stage]);
+    if (cx == x0) {
+      // with the first copies in flight: first/last CTA and empty partials of
+      // every range of the segment, before any warp writes a partial
+      mark_ranges<G>(p, plan, n8, x0, x1, c, tid, nthr);
+      __syncthreads();
     }
-  };
-
-  Ring<NS> ring;
-  ring.s = 0;
-#pragma unroll
-  for (int k = 0; k < NS; ++k) {
-    ring.item[k] = next_item();
-    if (ring.item[k] >= 0) issue(k, ring.item[k]);
+    int2 dnext = desc[0];
+    int duty = HB - 1;       // warp that refills after the current item: (k - 1) mod HB
+    for (int k = 0; k < m; ++k) {
+      const int2 d = dnext;
+      if (k + 1 < m) dnext = desc[k + 1];
+      const int kind = d.x & 3, vb = (d.x >> 2) & 0x1FFF;
+      const int pj = static_cast<int>(static_cast<uint32_t>(d.x) >> 15);
+      const int rid = 2 * vb + (kind == kItemInt4 ? 1 : 0);
+      if (rid != cur) {
+        if (cur >= 0) write_partial<D, NMT>(p, st, p.slots + ((long long)(cur + c) * HB + warp) * p.slot_floats, lane);
+        st.reset();
+        cur = rid;
+        const int hb = vb / p.B;
+        rc.b = vb - hb * p.B;
+        rc.h = hb * HB + warp;
+        rc.L = eff_len(p.seq_lens[rc.b], cap);
+        rc.lo_tok = p.sink;
+        rc.hi_tok = rc.L - p.recent;
+        rc.r0 = max(p.sink, rc.L - p.recent);
+        rc.mrow = p.mask ? p.mask + ((long long)rc.b * p.Hkv + rc.h) * p.mask_stride : nullptr;
+        load_q<D, G>(p, rc.b, rc.h, kind == kItemInt4, qsm, lane);
+      }
+      const bool ok = p.wait_cap != 0 && mbar_wait_bounded(&full[s], (phase >> s) & 1u, p.wait_cap);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) {
+          set_error(p.err, kErrTimeout);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      phase ^= 1u << s;
+      const uint8_t *stg = smem + s * stage_bytes + warp * 18 * D;
+      if (kind == kItemInt4) int4_item<D, G>(p, stg, qsm, pj, rc, st, lane);
+      else if (kind == kItemInt8K) int8k_item<D>(p, stg, qsm, pj, rc, st, wb0, wb1, lane);
+      else int8v_item<D>(stg, st, wb0, wb1, lane);
+      // release the stage (no result to wait for); one warp per item, in
+      // turn, refills the stage of the item before this one once every warp
+      // has released it -- normally long done by then
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (k > 0 && k - 1 + NS < m && duty == warp) {
+        const int sp = s == 0 ? NS - 1 : s - 1;
+        const int up = s == 0 ? rnd - 1 : rnd;   // how often stage sp was used before that item
+        const bool freed = mbar_wait_bounded(&empty[sp], static_cast<uint32_t>(up) & 1u, p.wait_cap);
+        if (!__all_sync(0xffffffffu, freed)) {
+          if (lane == 0) {
+            set_error(p.err, kErrTimeout);
+            *abort_flag = 1;
+          }
+          break;
+        }
+        if (lane == 0) {
+          fence_proxy_async();
+          iss[sp] += 1;
+          issue_item<D>(p, desc[k - 1 + NS], smem + sp * stage_bytes, &full[sp]);
+        }
+      }
+      if (++s == NS) {
+        s = 0;
+        ++rnd;
+      }
+      if (++duty == HB) duty = 0;
+    }
   }
-
-  uint32_t wb0 = 0, wb1 = 0;
-  while (ring.item[0] >= 0) {
-    if (!ring_wait<NS>(ring, bars, phase, p.wait_cap, p.err, lane)) return false;
-    const uint8_t *stg = wsm + ring.s * C::STAGE;
-    const int it = ring.item[0];
-    if ((it & 1) == 0) {
-      // ---- K half: scores, softmax, weights
-      const int j = it >> 1;
-      uint32_t kw[NW];
-#pragma unroll
-      for (int c = 0; c < NW / 4; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(stg + c * 512 + lane * 16);
-        kw[4 * c + 0] = w.x;
-        kw[4 * c + 1] = w.y;
-        kw[4 * c + 2] = w.z;
-        kw[4 * c + 3] = w.w;
-      }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int jj = 0; jj < NJ; jj += 2) {
-        const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + (jj / 2) * 512 + lane * 16);
-        const uint32_t a0[4] = {i8x2_to_f16x2(kw[jj]), i8x2_to_f16x2(kw[NJ + jj]), i8x2_to_f16x2(kw[jj] >> 8),
-                                i8x2_to_f16x2(kw[NJ + jj] >> 8)};
-        mma_f16(acc, a0, qv.x, qv.y);
-        const uint32_t a1[4] = {i8x2_to_f16x2(kw[jj + 1]), i8x2_to_f16x2(kw[NJ + jj + 1]),
-                                i8x2_to_f16x2(kw[jj + 1] >> 8), i8x2_to_f16x2(kw[NJ + jj + 1] >> 8)};
-        mma_f16(acc, a1, qv.z, qv.w);
-      }
-      const __half *ks = reinterpret_cast<const __half *>(stg + 16 * D);
-      const __half *vs = reinterpret_cast<const __half *>(stg + 16 * D + 32);
-      const float k0 = __half2float(ks[g]) * p.scale_log2, k1 = __half2float(ks[g + 8]) * p.scale_log2;
-      const bool v0 = row_pos(j, g) >= 0, v1 = row_pos(j, g + 8) >= 0;
-      float sl[4];
-      sl[0] = v0 ? acc[0] * k0 : -INFINITY;
-      sl[1] = v0 ? acc[1] * k0 : -INFINITY;
-      sl[2] = v1 ? acc[2] * k1 : -INFINITY;
-      sl[3] = v1 ? acc[3] * k1 : -INFINITY;
-      float pr[4];
-      softmax_update<NMT, 0>(st, sl, pr);
-      const float s0 = __half2float(vs[g]), s1 = __half2float(vs[g + 8]);
-      weights_f16(pr[0] * s0, pr[1] * s0, pr[2] * s1, pr[3] * s1, lo_sel, wb0, wb1);
-    } else {
-      // ---- V half: P.V
-      uint32_t vw[NW];
-#pragma unroll
-      for (int c = 0; c < NW / 4; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(stg + c * 512 + lane * 16);
-        vw[4 * c + 0] = w.x;
-        vw[4 * c + 1] = w.y;
-        vw[4 * c + 2] = w.z;
-        vw[4 * c + 3] = w.w;
-      }
-#pragma unroll
-      for (int mt = 0; mt < NMT; ++mt) {
-        const uint32_t a[4] = {i8x2_to_f16x2(vw[2 * mt]), i8x2_to_f16x2(vw[2 * mt] >> 8),
-                               i8x2_to_f16x2(vw[2 * mt + 1]), i8x2_to_f16x2(vw[2 * mt + 1] >> 8)};
-        mma_f16(st.o[mt], a, wb0, wb1);
-      }
-    }
-    __syncwarp();
-    const int nxt = next_item();
-    if (nxt >= 0) {
-      if (lane == 0) fence_proxy_async();
-      issue(ring.s, nxt);
-    }
-    ring.push_rotate(nxt);
+  __syncthreads();
+  if (*abort_flag) {
+    // a copy never landed: wait (bounded) for every copy still in flight, then
+    // leave; this CTA's ranges keep their empty partials
+    if (tid < NS && iss[tid] > 0) mbar_wait_bounded(&full[tid], (iss[tid] - 1) & 1u, kDefaultWaitCycles);
+    return;
   }
-  write_partial<D, NMT>(p, st, slot, lane);
-  return true;
+  if (cur >= 0) write_partial<D, NMT>(p, st, p.slots + ((long long)(cur + c) * HB + warp) * p.slot_floats, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -662,7 +908,7 @@ __device__ bool int8_piece(const DecodeParams &p, int b, int h, int L, int j0, i
 template <int D, int G>
 __device__ bool bf16_piece(const DecodeParams &p, int b, int h, int L, int pg0, int pg1, uint8_t *wsm,
                            uint64_t *bars, uint32_t &phase, float *slot, int lane) {
-  using C = Cfg<D, true>;
+  using C = Bf16Cfg<D>;
   constexpr int NS = C::NS, NK = D / 16, NMT = D / 16, ROWB = C::ROWB;
   const int g = lane >> 2, t = lane & 3;
 
@@ -751,16 +997,16 @@ __device__ bool bf16_piece(const DecodeParams &p, int b, int h, int L, int pg0, 
 }
 
 // ---------------------------------------------------------------------------
-// Persistent worker kernel.
+// bf16 comparison kernel: persistent warp workers over the flat space of
+// (sequence, KV head) page ranges, weighted equally per page.
 // ---------------------------------------------------------------------------
-template <int D, int G, bool kBF16>
-__global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) decode_kernel(DecodeParams p) {
-  using C = Cfg<D, kBF16>;
+template <int D, int G>
+__global__ void __launch_bounds__(kWarps * 32, 4) bf16_decode_kernel(DecodeParams p) {
+  using C = Bf16Cfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t *wsm = smem + warp * C::WARP_SMEM;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kWarps * C::WARP_SMEM) + warp * C::NS;
-  uint8_t *qsm = smem + kWarps * (C::WARP_SMEM + C::NS * 8) + warp * C::QBYTES;
   int *plan = reinterpret_cast<int *>(smem + C::RINGS);   // [B + 1]
   __shared__ int wtot[kWarps];
 
@@ -769,18 +1015,15 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) decode_kernel(Dec
     for (int s = 0; s < C::NS; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
-  pdl_wait();                 // inputs and cache writes of earlier grids are visible from here
-  pdl_launch_dependents();    // the merge grid may queue behind the workers
+  pdl_wait();
+  pdl_launch_dependents();
 
-  // plan[b] = sum over b' < b of (attended pages of b') * Hkv, computed by the CTA
+  // plan[b] = sum over b' < b of (pages of b') * Hkv, computed by the CTA
   const int cap = p.pt_stride * kPageTokens;
   const int chunk = (p.B + kWarps * 32 - 1) / (kWarps * 32);
   const int b0 = min(p.B, tid * chunk), b1 = min(p.B, b0 + chunk);
   int mine = 0;
-  for (int b = b0; b < b1; ++b) {
-    const int L = eff_len(p.seq_lens[b], cap);
-    mine += kBF16 ? (L + kPageTokens - 1) / kPageTokens : int4_num_pages(L, p.sink, p.recent);
-  }
+  for (int b = b0; b < b1; ++b) mine += (eff_len(p.seq_lens[b], cap) + kPageTokens - 1) / kPageTokens;
   mine *= p.Hkv;
   int incl = mine;
 #pragma unroll
@@ -794,8 +1037,7 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) decode_kernel(Dec
   for (int w = 0; w < warp; ++w) run += wtot[w];
   for (int b = b0; b < b1; ++b) {
     plan[b] = run;
-    const int L = eff_len(p.seq_lens[b], cap);
-    run += (kBF16 ? (L + kPageTokens - 1) / kPageTokens : int4_num_pages(L, p.sink, p.recent)) * p.Hkv;
+    run += (eff_len(p.seq_lens[b], cap) + kPageTokens - 1) / kPageTokens * p.Hkv;
   }
   if (tid == kWarps * 32 - 1) plan[p.B] = run;
   __syncthreads();
@@ -807,125 +1049,136 @@ __global__ void __launch_bounds__(kWarps * 32, KV4_MIN_BLOCKS) decode_kernel(Dec
   }
 
   const long long wid = (long long)blockIdx.x * kWarps + warp;
-  const int np8 = (!kBF16 && p.int8_units) ? side_pages(p.sink, p.recent) : 0;
-  const long long T8 = (long long)p.B * p.Hkv * np8;
   const long long T4 = plan[p.B];
-  const long long NWk = active_workers(p.num_workers, T8, T4);
+  const long long NWk = active_workers(p.num_workers, 0, T4);
   if (wid >= NWk) return;
-  long long x = worker_first_item(wid, NWk, T8, T4);
-  const long long z = worker_first_item(wid + 1, NWk, T8, T4);
+  long long x = worker_first_item(wid, NWk, 0, T4);
+  const long long z = worker_first_item(wid + 1, NWk, 0, T4);
   const long long nbh = (long long)p.B * p.Hkv;
   if (x >= z) return;
 
   uint32_t phase = 0;
-  const int first_page = kBF16 ? 0 : int4_first_page(p.sink);
   int b = 0;
   bool located = false;
   while (x < z) {
-    bool ok;
-    bool int8_item = false;
-    if constexpr (!kBF16) int8_item = x < T8;
-    if (int8_item) {
-      if constexpr (!kBF16) {
-        const int r8 = static_cast<int>(x / np8);
-        const int j0 = static_cast<int>(x % np8);
-        const long long e = min(z, (long long)(r8 + 1) * np8);
-        const int L = eff_len(p.seq_lens[r8 / p.Hkv], cap);
-        float *slot = p.slots + ((long long)r8 + wid) * p.slot_floats;
-        if (lane == 0) {
-          if (j0 == 0) p.first[r8] = static_cast<int>(wid);
-          if (e == (long long)(r8 + 1) * np8) p.last[r8] = static_cast<int>(wid);
-        }
-        ok = int8_piece<D, G>(p, r8 / p.Hkv, r8 % p.Hkv, L, j0, j0 + static_cast<int>(e - x), wsm, bars, qsm,
-                              phase, slot, lane);
-        x = e;
+    const int y = static_cast<int>(x);
+    if (!located) {   // sequence holding y: largest b with plan[b] <= y
+      int lo = 0, hi = p.B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (plan[mid] <= y) lo = mid;
+        else hi = mid - 1;
       }
-    } else {
-      const int y = static_cast<int>(x - T8);
-      if (!located) {   // sequence holding y: largest b with plan[b] <= y
-        int lo = 0, hi = p.B - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (plan[mid] <= y) lo = mid;
-          else hi = mid - 1;
-        }
-        b = lo;
-        located = true;
-      }
-      while (plan[b + 1] <= y) ++b;
-      const int per = (plan[b + 1] - plan[b]) / p.Hkv;
-      const int h = (y - plan[b]) / per;
-      const int off = (y - plan[b]) % per;
-      const long long e = min(z, T8 + plan[b] + (long long)(h + 1) * per);
-      const int L = eff_len(p.seq_lens[b], cap);
-      float *slot = p.slots + (nbh + (long long)b * p.Hkv + h + wid) * p.slot_floats;
-      const int pg0 = first_page + off;
-      const int pg1 = pg0 + static_cast<int>(e - x);
-      if (lane == 0) {
-        if (off == 0) p.first[nbh + (long long)b * p.Hkv + h] = static_cast<int>(wid);
-        if (e == T8 + plan[b] + (long long)(h + 1) * per) p.last[nbh + (long long)b * p.Hkv + h] = static_cast<int>(wid);
-      }
-      if constexpr (kBF16) ok = bf16_piece<D, G>(p, b, h, L, pg0, pg1, wsm, bars, phase, slot, lane);
-      else ok = int4_piece<D, G>(p, b, h, L, pg0, pg1, wsm, bars, qsm, phase, slot, lane);
-      x = e;
+      b = lo;
+      located = true;
     }
-    if (!ok) return;
+    while (plan[b + 1] <= y) ++b;
+    const int per = (plan[b + 1] - plan[b]) / p.Hkv;
+    const int h = (y - plan[b]) / per;
+    const int off = (y - plan[b]) % per;
+    const long long e = min(z, (long long)plan[b] + (long long)(h + 1) * per);
+    const int L = eff_len(p.seq_lens[b], cap);
+    float *slot = p.slots + (nbh + (long long)b * p.Hkv + h + wid) * p.slot_floats;
+    if (lane == 0) {
+      if (off == 0) p.first[nbh + (long long)b * p.Hkv + h] = static_cast<int>(wid);
+      if (e == (long long)plan[b] + (long long)(h + 1) * per) p.last[nbh + (long long)b * p.Hkv + h] = static_cast<int>(wid);
+    }
+    if (!bf16_piece<D, G>(p, b, h, L, off, off + static_cast<int>(e - x), wsm, bars, phase, slot, lane)) return;
+    x = e;
   }
 }
 
 // ---------------------------------------------------------------------------
 // Host side launchers.
 // ---------------------------------------------------------------------------
-int decode_smem_bytes(int D, bool bf16, int B) {
-  const int rings = D == 128 ? (bf16 ? Cfg<128, true>::RINGS : Cfg<128, false>::RINGS)
-                             : (bf16 ? Cfg<64, true>::RINGS : Cfg<64, false>::RINGS);
-  return rings + 4 * (B + 1);
+int kv4_smem_bytes(int D, int HB, int NS, int NVB) { return kv4_layout(D, HB, NS, NVB).total; }
+
+int bf16_smem_bytes(int D, int B) {
+  return (D == 128 ? Bf16Cfg<128>::RINGS : Bf16Cfg<64>::RINGS) + 4 * (B + 1);
 }
 
-template <int D, int G, bool kBF16>
-static cudaError_t prepare_one(DecodeLaunch *out) {
-  const int smem_max = decode_smem_bytes(D, kBF16, kMaxBatch);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G, kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int D, int G>
+static cudaError_t kv4_prepare_one(int HB, int smem, int *blocks_per_sm) {
+  if (blocks_per_sm == nullptr)
+    return cudaFuncSetAttribute(kv4_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, kv4_decode_kernel<D, G>, HB * 32, smem);
+}
+
+static cudaError_t kv4_prepare(int D, int G, int HB, int smem, int *blocks_per_sm) {
+  if (D == 128) {
+    switch (G) {
+      case 1: return kv4_prepare_one<128, 1>(HB, smem, blocks_per_sm);
+      case 2: return kv4_prepare_one<128, 2>(HB, smem, blocks_per_sm);
+      case 4: return kv4_prepare_one<128, 4>(HB, smem, blocks_per_sm);
+    }
+  } else if (D == 64) {
+    switch (G) {
+      case 1: return kv4_prepare_one<64, 1>(HB, smem, blocks_per_sm);
+      case 2: return kv4_prepare_one<64, 2>(HB, smem, blocks_per_sm);
+      case 4: return kv4_prepare_one<64, 4>(HB, smem, blocks_per_sm);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t kv4_decode_set_smem_limit(int D, int G, int smem) { return kv4_prepare(D, G, 1, smem, nullptr); }
+
+cudaError_t kv4_decode_occupancy(int D, int G, int HB, int smem, int *blocks_per_sm) {
+  return kv4_prepare(D, G, HB, smem, blocks_per_sm);
+}
+
+template <int D, int G>
+static cudaError_t bf16_prepare_one(DecodeLaunch *out) {
+  const int smem_max = bf16_smem_bytes(D, kMaxBatch);
+  cudaError_t e = cudaFuncSetAttribute(bf16_decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        smem_max);
   if (e != cudaSuccess) return e;
   int nb = 0;
   // occupancy at batches up to 1024 sequences; larger batches only add plan bytes
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, decode_kernel<D, G, kBF16>, kWarps * 32,
-                                                    decode_smem_bytes(D, kBF16, 1024));
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, bf16_decode_kernel<D, G>, kWarps * 32,
+                                                    bf16_smem_bytes(D, 1024));
   if (e != cudaSuccess) return e;
-  out->smem_bytes = decode_smem_bytes(D, kBF16, 1024);
+  out->smem_bytes = bf16_smem_bytes(D, 1024);
   out->blocks_per_sm = nb > 0 ? nb : 1;
   return cudaSuccess;
 }
 
-template <int D, bool kBF16>
-static cudaError_t prepare_d(int G, DecodeLaunch *out) {
-  switch (G) {
-    case 1: return prepare_one<D, 1, kBF16>(out);
-    case 2: return prepare_one<D, 2, kBF16>(out);
-    case 4: return prepare_one<D, 4, kBF16>(out);
-    default: return cudaErrorInvalidValue;
+cudaError_t bf16_decode_prepare(int D, int G, DecodeLaunch *out) {
+  if (D == 128) {
+    switch (G) {
+      case 1: return bf16_prepare_one<128, 1>(out);
+      case 2: return bf16_prepare_one<128, 2>(out);
+      case 4: return bf16_prepare_one<128, 4>(out);
+    }
+  } else if (D == 64) {
+    switch (G) {
+      case 1: return bf16_prepare_one<64, 1>(out);
+      case 2: return bf16_prepare_one<64, 2>(out);
+      case 4: return bf16_prepare_one<64, 4>(out);
+    }
   }
-}
-
-cudaError_t decode_prepare(int D, int G, bool bf16, DecodeLaunch *out) {
-  if (D == 128) return bf16 ? prepare_d<128, true>(G, out) : prepare_d<128, false>(G, out);
-  if (D == 64) return bf16 ? prepare_d<64, true>(G, out) : prepare_d<64, false>(G, out);
   return cudaErrorInvalidValue;
 }
 
-template <int D, int G, bool kBF16>
-static cudaError_t launch_main(const DecodeParams &p, cudaStream_t stream) {
-  return launch_pdl(decode_kernel<D, G, kBF16>, dim3(p.num_workers / kWarps), dim3(kWarps * 32),
-                    decode_smem_bytes(D, kBF16, p.B), stream, p);
+template <int D>
+static cudaError_t launch_kv4_d(const DecodeParams &p, cudaStream_t stream) {
+  const dim3 grid(p.n_cta), block(p.HB * 32);
+  const int smem = kv4_smem_bytes(D, p.HB, p.NS, p.NVB);
+  switch (p.G) {
+    case 1: return launch_pdl(kv4_decode_kernel<D, 1>, grid, block, smem, stream, p);
+    case 2: return launch_pdl(kv4_decode_kernel<D, 2>, grid, block, smem, stream, p);
+    default: return launch_pdl(kv4_decode_kernel<D, 4>, grid, block, smem, stream, p);
+  }
 }
 
-template <int D, bool kBF16>
-static cudaError_t launch_main_d(const DecodeParams &p, cudaStream_t stream) {
+template <int D>
+static cudaError_t launch_bf16_d(const DecodeParams &p, cudaStream_t stream) {
+  const dim3 grid(p.num_workers / kWarps), block(kWarps * 32);
+  const int smem = bf16_smem_bytes(D, p.B);
   switch (p.G) {
-    case 1: return launch_main<D, 1, kBF16>(p, stream);
-    case 2: return launch_main<D, 2, kBF16>(p, stream);
-    default: return launch_main<D, 4, kBF16>(p, stream);
+    case 1: return launch_pdl(bf16_decode_kernel<D, 1>, grid, block, smem, stream, p);
+    case 2: return launch_pdl(bf16_decode_kernel<D, 2>, grid, block, smem, stream, p);
+    default: return launch_pdl(bf16_decode_kernel<D, 4>, grid, block, smem, stream, p);
   }
 }
 
@@ -933,12 +1186,11 @@ cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t 
                           cudaEvent_t ev1) {
   if (ev0) cudaEventRecord(ev0, stream);
   cudaError_t e;
-  if (D == 128) e = bf16 ? launch_main_d<128, true>(p, stream) : launch_main_d<128, false>(p, stream);
-  else e = bf16 ? launch_main_d<64, true>(p, stream) : launch_main_d<64, false>(p, stream);
+  if (bf16) e = D == 128 ? launch_bf16_d<128>(p, stream) : launch_bf16_d<64>(p, stream);
+  else e = D == 128 ? launch_kv4_d<128>(p, stream) : launch_kv4_d<64>(p, stream);
   if (e != cudaSuccess) return e;
   if (ev1) cudaEventRecord(ev1, stream);
-  const int np8 = (!bf16 && p.int8_units) ? side_pages(p.sink, p.recent) : 0;
-  return launch_merge(p, D, np8, stream);
+  return launch_merge(p, D, bf16, stream);
 }
 
 }  // namespace kv4

@@ -5,7 +5,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+struct kv4_cache;
+
 namespace kv4 {
+
+// Device a kv4_cache was created on (-1 for NULL).
+int cache_device(const kv4_cache *cache);
 
 struct AppendParams {
   const __nv_bfloat16 *k;   // [T][Hkv][D]
@@ -25,6 +30,9 @@ struct AppendParams {
 struct DecodeParams {
   int B, Hq, Hkv, G, sink, recent, num_pages, pt_stride, mask_stride;
   int num_workers, slot_floats, slot_o_off, int8_units;
+  // KV4 kernel: HB warps (KV heads) per CTA, NVB = B * Hkv / HB virtual
+  // sequences, NS ring stages, np8 side pages per (sequence, head), n_cta CTAs
+  int HB, NVB, NS, np8, n_cta;
   const __nv_bfloat16 *q;       // [B][Hq][D]
   const int32_t *seq_lens;      // [B]
   const int32_t *page_table;    // [B][pt_stride]
@@ -33,10 +41,15 @@ struct DecodeParams {
   const uint8_t *side;          // INT8 side blocks
   long long page_bytes, head_bytes, side_stride;
   float scale_log2;             // softmax_scale * log2(e)
-  int *plan;                    // [B+1] prefix of attended INT4/bf16 page-heads
-  int *first;                   // [2*B*Hkv] worker owning the first item of each range
-  int *last;                    // [2*B*Hkv] worker owning the last item of each range
-  float *slots;                 // [2*B*Hkv + num_workers][slot_floats] partials
+  // KV4: plan [NVB+1] (INT4 pages before each virtual sequence), first/last
+  // CTA of each (region, virtual sequence) range [2*NVB], partial slots
+  // [2*NVB + n_cta][HB][slot_floats]. bf16: plan [B+1] (page-heads before
+  // each sequence), first/last warp of each (sequence, head) range [2*B*Hkv],
+  // slots [2*B*Hkv + num_workers][slot_floats].
+  int *plan;
+  int *first;
+  int *last;
+  float *slots;
   void *out;
   int out_fp32;
   uint32_t *err;
@@ -52,8 +65,11 @@ struct TopkParams {
   int32_t *count;
 };
 
-// Largest batch kv4_decode_attn accepts (the per-CTA plan lives in shared memory).
+// Largest batch kv4_decode_attn accepts (the per-CTA plan lives in shared
+// memory; item descriptors hold a virtual sequence in 13 bits).
 constexpr int kMaxBatch = 8192;
+// Largest page-table row of the KV4 kernel (page index in 17 bits).
+constexpr int kMaxPtStride = 1 << 17;
 
 struct DecodeLaunch {
   int smem_bytes;
@@ -80,12 +96,17 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 cudaError_t launch_append(const AppendParams &p, int D, cudaStream_t stream);
-cudaError_t decode_prepare(int D, int G, bool bf16, DecodeLaunch *out);
-int decode_smem_bytes(int D, bool bf16, int B);
+// KV4 kernel: raise its dynamic shared-memory limit on the current device;
+// resident CTAs per SM at HB warps and `smem` bytes per CTA.
+cudaError_t kv4_decode_set_smem_limit(int D, int G, int smem);
+cudaError_t kv4_decode_occupancy(int D, int G, int HB, int smem, int *blocks_per_sm);
+int kv4_smem_bytes(int D, int HB, int NS, int NVB);
+cudaError_t bf16_decode_prepare(int D, int G, DecodeLaunch *out);
+int bf16_smem_bytes(int D, int B);
 cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t stream, cudaEvent_t ev0,
                           cudaEvent_t ev1);
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream);
-// Exact merge of the decode partials (np8 = INT8 side pages per (sequence, head)).
-cudaError_t launch_merge(const DecodeParams &p, int D, int np8, cudaStream_t stream);
+// Exact merge of the decode partials of kv4_decode_kernel or bf16_decode_kernel.
+cudaError_t launch_merge(const DecodeParams &p, int D, bool bf16, cudaStream_t stream);
 
 }  // namespace kv4

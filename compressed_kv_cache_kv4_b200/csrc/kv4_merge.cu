@@ -8,9 +8,12 @@
 // and out = 0 when every partial is empty (l_c = 0).
 //
 // One warp per (sequence b, query head hq); lane k owns output elements
-// [k D/32, (k+1) D/32). The decode kernel records, per (region, sequence, KV
-// head) range, the first and last worker whose segment touched it; partial c
-// of worker w sits in slot (range index + w). Every lane loads (m, l) and its
+// [k D/32, (k+1) D/32). The decode kernels record, per range of the work
+// space (KV4: a region of a virtual sequence, all heads of its block; bf16: a
+// (sequence, KV head)), the first and last worker whose segment touched it;
+// the partial of worker w sits in slot (range index + w) * (heads per range)
+// + head. Workers between the first and the last wrote a partial for the
+// range (an empty one, l = 0, if nothing of it was attended). Every lane loads (m, l) and its
 // slice of o for a batch of up to kBatch partials at once, so a batch costs a
 // single round trip to L2 (the partials were written moments ago by other SMs;
 // all loads bypass L1).
@@ -48,8 +51,8 @@ struct Vec<2> {
 
 }  // namespace
 
-template <int D, int G>
-__global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
+template <int D, int G, bool kKv4>
+__global__ void __launch_bounds__(128) merge_kernel(DecodeParams p) {
   constexpr int DPL = D / 32;
   const long long task = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -58,22 +61,48 @@ __global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
   if (task >= (long long)p.B * p.Hq) return;
   const int b = static_cast<int>(task / p.Hq), hq = static_cast<int>(task % p.Hq);
   const int h = hq / G, g = hq % G;
-  const long long nbh = (long long)p.B * p.Hkv, r = (long long)b * p.Hkv + h;
-
-  // Range bounds and the plan entries, all independent loads.
-  const int pb0 = __ldcg(&p.plan[b]), pb1 = __ldcg(&p.plan[b + 1]);
-  const long long T4 = __ldcg(&p.plan[p.B]);
-  const int f8 = __ldcg(&p.first[r]), l8 = __ldcg(&p.last[r]);
-  const int f4 = __ldcg(&p.first[nbh + r]), l4 = __ldcg(&p.last[nbh + r]);
-  const long long T8 = nbh * np8;
-  // the decode kernel's worker count; every one of them owns at least one item
-  const long long nw = active_workers(p.num_workers, T8, T4);
+  // Ranges of this query head and their slots; the partial of worker w for
+  // range r sits in slot (r + w) * HB + hh.
+  //   KV4: v = virtual sequence hb * B + b (hh = head within the block), its
+  //        INT8 range 2v and INT4 range 2v + 1; plan[v] = first item of v
+  //        (n8 INT8 items, then its INT4 pages); workers = CTAs.
+  //   bf16: v = b * Hkv + h, HB = 1; one range B * Hkv + v; plan[b] = first
+  //        page-head of sequence b; workers = warps.
+  int HB, hh;
+  long long r8, r4, nw;
+  bool has8, has4;
+  if constexpr (kKv4) {
+    HB = p.HB;
+    const int hb = h / HB;
+    hh = h - hb * HB;
+    const int v = hb * p.B + b;
+    const int n8 = p.int8_units ? 2 * p.np8 : 0;
+    const long long T = __ldcg(&p.plan[p.NVB]);
+    const int pb0 = __ldcg(&p.plan[v]), pb1 = __ldcg(&p.plan[v + 1]);
+    nw = T > 0 ? min((long long)p.n_cta, max(1LL, T >> 1)) : 0;   // CTAs that took part
+    r8 = 2LL * v;
+    r4 = 2LL * v + 1;
+    has8 = n8 > 0;
+    has4 = pb1 - pb0 > n8;
+  } else {
+    HB = 1;
+    hh = 0;
+    const long long T4 = __ldcg(&p.plan[p.B]);
+    const int pb0 = __ldcg(&p.plan[b]), pb1 = __ldcg(&p.plan[b + 1]);
+    nw = active_workers(p.num_workers, 0, T4);
+    r8 = 0;
+    r4 = (long long)p.B * p.Hkv + (long long)b * p.Hkv + h;
+    has8 = false;
+    has4 = pb1 > pb0;
+  }
+  const int f8 = has8 ? __ldcg(&p.first[r8]) : -1, l8 = has8 ? __ldcg(&p.last[r8]) : -1;
+  const int f4 = has4 ? __ldcg(&p.first[r4]) : -1, l4 = has4 ? __ldcg(&p.last[r4]) : -1;
   // A range is used only if it has items; bounds outside [0, nw) (possible only
   // after a worker stopped on an error) drop the range instead of being read.
-  const bool ok8 = np8 > 0 && f8 >= 0 && f8 <= l8 && l8 < nw;
-  const bool ok4 = pb1 > pb0 && f4 >= 0 && f4 <= l4 && l4 < nw;
-  const int n8 = ok8 ? l8 - f8 + 1 : 0;
-  const int n = n8 + (ok4 ? l4 - f4 + 1 : 0);
+  const bool ok8 = has8 && f8 >= 0 && f8 <= l8 && l8 < nw;
+  const bool ok4 = has4 && f4 >= 0 && f4 <= l4 && l4 < nw;
+  const int n8r = ok8 ? l8 - f8 + 1 : 0;
+  const int n = n8r + (ok4 ? l4 - f4 + 1 : 0);
 
   float M = -INFINITY, den = 0.f, acc[DPL];
 #pragma unroll
@@ -88,8 +117,8 @@ __global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
 #pragma unroll
       for (int e = 0; e < DPL; ++e) ok[k][e] = 0.f;
       if (i < n) {
-        const long long w = i < n8 ? f8 + i : f4 + (i - n8);
-        const float *slot = p.slots + ((i < n8 ? r : nbh + r) + w) * p.slot_floats;
+        const long long w = i < n8r ? f8 + i : f4 + (i - n8r);
+        const float *slot = p.slots + (((i < n8r ? r8 : r4) + w) * HB + hh) * p.slot_floats;
         mk[k] = __ldcg(slot + g);
         lk[k] = __ldcg(slot + G + g);
         Vec<DPL>::load(slot + p.slot_o_off + g * D + lane * DPL, ok[k]);
@@ -135,20 +164,21 @@ __global__ void __launch_bounds__(128) merge_kernel(DecodeParams p, int np8) {
   }
 }
 
-template <int D>
-static cudaError_t launch_merge_d(const DecodeParams &p, int np8, cudaStream_t stream) {
+template <int D, bool kKv4>
+static cudaError_t launch_merge_d(const DecodeParams &p, cudaStream_t stream) {
   const long long warps = (long long)p.B * p.Hq;
   if (warps == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((warps + 3) / 4);
   switch (p.G) {
-    case 1: return launch_pdl(merge_kernel<D, 1>, dim3(blocks), dim3(128), 0, stream, p, np8);
-    case 2: return launch_pdl(merge_kernel<D, 2>, dim3(blocks), dim3(128), 0, stream, p, np8);
-    default: return launch_pdl(merge_kernel<D, 4>, dim3(blocks), dim3(128), 0, stream, p, np8);
+    case 1: return launch_pdl(merge_kernel<D, 1, kKv4>, dim3(blocks), dim3(128), 0, stream, p);
+    case 2: return launch_pdl(merge_kernel<D, 2, kKv4>, dim3(blocks), dim3(128), 0, stream, p);
+    default: return launch_pdl(merge_kernel<D, 4, kKv4>, dim3(blocks), dim3(128), 0, stream, p);
   }
 }
 
-cudaError_t launch_merge(const DecodeParams &p, int D, int np8, cudaStream_t stream) {
-  return D == 128 ? launch_merge_d<128>(p, np8, stream) : launch_merge_d<64>(p, np8, stream);
+cudaError_t launch_merge(const DecodeParams &p, int D, bool bf16, cudaStream_t stream) {
+  if (bf16) return D == 128 ? launch_merge_d<128, false>(p, stream) : launch_merge_d<64, false>(p, stream);
+  return D == 128 ? launch_merge_d<128, true>(p, stream) : launch_merge_d<64, true>(p, stream);
 }
 
 }  // namespace kv4

@@ -81,6 +81,10 @@ typedef struct kv4_cache kv4_cache;   /* opaque host handle */
 /* Human-readable name of a status. Never NULL. */
 const char *kv4_status_string(kv4_status s);
 
+/* Text of the last CUDA runtime error behind a KV4_ERR_CUDA returned to the
+ * calling thread ("no error" if none); a static string, not to be freed. */
+const char *kv4_last_cuda_error(void);
+
 /*
  * kv4_cache_bytes -- sizes of the two caller-owned device buffers.
  *  page_pool_bytes: num_pages pages. One page holds 16 positions of every KV
@@ -329,6 +333,10 @@ kv4_status kv4_debug_set_wait_limit(kv4_cache *cache, int64_t cycles);
  */
 kv4_status kv4_timing_enable(int32_t max_records, int32_t every);
 kv4_status kv4_timing_read(int32_t kind, double *total_ms, int32_t *count);
+/* The same records as kv4_timing_read, one duration per recorded call
+ * (milliseconds, oldest first): fills min(cap, count) entries of the host
+ * array ms_out, sets *count to the number recorded, and clears them. */
+kv4_status kv4_timing_read_each(int32_t kind, float *ms_out, int32_t cap, int32_t *count);
 kv4_status kv4_timing_disable(void);
 
 /* Number of multiprocessors and default worker count the library uses. */

@@ -9,6 +9,10 @@ outputs the oracle computes sequence by sequence.
   against the single-pass oracle.
 - evict: B = 64, L = 16384; top-k masks bit-exact at every budget,
   masked decode at 10% and 50% on sampled sequences, 100% = unmasked bitwise.
+- prefill bytes: the benchmark's prefill of the qwen8b and async prompts in one
+  kv4_append; page and side-cache bytes of sampled sequences (the first and the
+  last ones of the batch among them, which only later grid-stride passes of the
+  page kernel reach) bit-exact against the oracle's writer.
 """
 import gc
 
@@ -166,6 +170,58 @@ def test_evict_full_size():
             assert torch.equal(full, unmasked)
     st, bits = cache.get_error()
     assert st == K.KV4_OK, (st, bits)
+    cache.close()
+    del cache
+    _cleanup()
+
+
+@pytest.mark.parametrize("name", ["qwen8b", "async"])
+def test_prefill_bytes_full_size(name):
+    wl = synth.workload(name)
+    L0 = wl.lens.astype(np.int64)
+    lens_pre = np.maximum(L0 - 64, 0).astype(np.int32)        # the benchmark's prefill lengths
+    k, v, off = synth.gen_kv(wl, device="cuda", lens=lens_pre)
+    pt, npages = synth.gen_page_table(wl, L0 + 64)
+    cache = K.KV4Cache(wl.Hkv, wl.D, wl.B, npages, wl.sink, wl.recent, fill=0xA5)
+    ptd = torch.as_tensor(pt, device="cuda")
+    cache.append(k, v, torch.as_tensor(off.astype(np.int32), device="cuda"),
+                 torch.zeros(wl.B, dtype=torch.int32, device="cuda"), ptd)
+    torch.cuda.synchronize()
+    st, bits = cache.get_error()
+    assert st == K.KV4_OK, (st, bits)
+    seqs = sorted(set(_sample(lens_pre, 3, 27)) | {0, 1, wl.B // 2, wl.B - 2, wl.B - 1})
+    n = len(seqs)
+    lens_s = lens_pre[seqs].astype(np.int32)
+    Lmax = int(lens_s.max())
+    kb = torch.zeros((n, Lmax, wl.Hkv, wl.D), dtype=torch.bfloat16)
+    vb = torch.zeros_like(kb)
+    for i, b in enumerate(seqs):
+        kb[i, : lens_s[i]] = k[int(off[b]): int(off[b + 1])].cpu()
+        vb[i, : lens_s[i]] = v[int(off[b]): int(off[b + 1])].cpu()
+    del k, v
+    _cleanup()
+    # the sampled sequences' pages renumbered into a compact pool for the oracle
+    npg = [(int(L) + 15) // 16 for L in lens_s]
+    pt_s = np.full((n, max(npg)), -1, np.int32)
+    nxt = 0
+    for i in range(n):
+        pt_s[i, : npg[i]] = np.arange(nxt, nxt + npg[i])
+        nxt += npg[i]
+    sh = O.shape(n, wl.Hq, wl.Hkv, wl.D, wl.sink, wl.recent)
+    pool_ref, side_ref, flags = O.write_cache(sh, synth.bf16_bits(kb), synth.bf16_bits(vb), lens_s, pt_s,
+                                              max(nxt, 1), fill=0xA5)
+    assert flags == 0
+    page_bytes = wl.Hkv * 18 * wl.D
+    side_blk = cache.side.numel() // wl.B
+    pool = cache.pool.view(npages, page_bytes)
+    side = cache.side.view(wl.B, side_blk)
+    for i, b in enumerate(seqs):
+        ids = torch.as_tensor(pt[b, : npg[i]].astype(np.int64), device="cuda")
+        got = pool.index_select(0, ids).cpu().numpy()
+        want = pool_ref.reshape(-1, page_bytes)[pt_s[i, : npg[i]]]
+        assert np.array_equal(got, want), "%s: pages of sequence %d differ" % (name, b)
+        assert np.array_equal(side[b].cpu().numpy(), side_ref.reshape(n, side_blk)[i]), \
+            "%s: side cache of sequence %d differs" % (name, b)
     cache.close()
     del cache
     _cleanup()

@@ -330,3 +330,51 @@ def test_append_exact_ties():
     pool, side, _ = c.oracle_cache()
     assert np.array_equal(c.cache.pool.cpu().numpy(), pool)
     assert np.array_equal(c.cache.side.cpu().numpy(), side)
+
+
+# ------------------------------------------------------------------ query magnitude
+def _scaled_queries(q, scale, spike_channels, spike):
+    """q * scale, with `spike_channels` channels of every query head multiplied by `spike` more
+    (queries after a QK-norm are far from N(0, 1) per channel)."""
+    x = q.float() * scale
+    if spike_channels:
+        g = torch.Generator().manual_seed(99)
+        ch = torch.randperm(q.shape[-1], generator=g)[:spike_channels]
+        x[..., ch] *= spike
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("scale,spike_channels,spike", [(8.0, 0, 1.0), (32.0, 0, 1.0), (1.0, 3, 100.0),
+                                                         (8.0, 4, 100.0), (0.01, 0, 1.0)])
+def test_decode_large_queries(scale, spike_channels, spike):
+    """q·K with queries far from N(0, 1): large magnitudes (peaky softmax, scores in the
+    hundreds), a few channels two orders of magnitude above the rest, and tiny queries
+    (near-uniform softmax). Outputs stay within the tolerance of the fp64 oracle."""
+    wl = small_wl([1, 17, 145, 300, 1000, 2049, 3001], seed=41)
+    c = Case(wl)
+    c.make_cache()
+    c.append_all()
+    q = _scaled_queries(c.q, scale, spike_channels, spike)
+    assert torch.isfinite(q.float()).all()
+    c.q = q
+    ref = c.oracle_decode()
+    out32 = c.decode(out_fp32=True)
+    out16 = c.decode(out_fp32=False)
+    assert c.cache.get_error()[0] == K.KV4_OK
+    assert_close(out32.cpu().numpy(), ref, what="q x%g, %d channels x%g" % (scale, spike_channels, spike))
+    assert_bf16_output(out16, out32, ref)
+
+
+def test_decode_query_beyond_fp16_range_is_reported():
+    """A query element whose magnitude exceeds the fp16 range cannot enter the fp16 tiles:
+    the kernel reports KV4_ERR_RANGE instead of returning silently wrong scores."""
+    wl = small_wl([300, 40], seed=42, Hq=8, Hkv=2)
+    c = Case(wl)
+    c.make_cache()
+    c.append_all()
+    q = c.q.clone()
+    q[0, 1, 5] = 1.0e5
+    c.decode(q=q)
+    st, bits = c.cache.get_error()
+    assert st == K.KV4_ERR_RANGE and bits & (1 << K.KV4_ERR_RANGE)
+    assert c.cache.get_error()[0] == K.KV4_OK
