@@ -40,7 +40,6 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 CYCLE = 64
-TIMING_EVERY = 8
 
 
 def parse():
@@ -173,7 +172,7 @@ def peaks():
 
 
 # ---------------------------------------------------------------------------- ncu traffic
-PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_qwen8b.md")
+PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_qwen8b.json")
 KERNEL_SOURCES = ["kv4_decode.cu", "kv4_common.cuh", "kv4_internal.h"]
 
 
@@ -189,17 +188,16 @@ def kernel_source_hash():
 
 
 def ncu_traffic(wbytes):
-    """DRAM bytes (read + write) of one decode_kernel launch, from the committed
-    ncu summary, scaled from the captured launch's algorithmic bytes to
-    `wbytes`. None if the summary is absent or the kernel sources have changed
-    since the capture."""
+    """DRAM bytes (read + write) of one decode worker launch from the committed
+    ncu figures (profiles/decode_kernel_qwen8b.json), scaled from the captured
+    launch's algorithmic bytes to `wbytes`. None if the figures are absent or
+    the kernel sources have changed since the capture."""
     try:
-        vals = dict(re.findall(r"^- (\w+): (\S+)\s*$", open(PROFILE).read(), re.M))
-        if vals.get("kernel_sources_sha256") != kernel_source_hash():
+        d = json.load(open(PROFILE))
+        if d.get("kernel_sources_sha256") != kernel_source_hash():
             return None
-        return int(round(float(vals["dram_bytes_per_launch"]) * wbytes /
-                         float(vals["algorithmic_bytes_of_captured_launch"])))
-    except (OSError, KeyError, ValueError):
+        return int(round(float(d["dram_bytes_per_launch"]) * wbytes / float(d["algorithmic_bytes_of_captured_launch"])))
+    except (OSError, KeyError, ValueError, TypeError):
         return None
 
 
@@ -257,8 +255,227 @@ def prefill(cache, wl, lens_pre, ptd, purpose=1):
     return k, v, off
 
 
+class Steady:
+    """A workload in steady state: the cache is prefilled to L0 - 64 positions
+    and step s appends position L0 - 64 + (s mod 64) of every sequence and
+    attends over L0 - 63 + (s mod 64) positions, so the lengths keep the
+    workload's distribution however many steps run. The inputs of all 64
+    cycle steps are resident on the device."""
+
+    def __init__(self, wl, rank=0):
+        import compressed_kv_cache_kv4_b200 as K
+        from compressed_kv_cache_kv4_b200 import synth
+        self.wl = wl
+        L0 = wl.lens.astype(np.int64)
+        self.lens_pre = np.maximum(L0 - CYCLE, 0).astype(np.int32)
+        self.cache, self.ptd, self.pt_np, self.npages = build_kv4(wl, L0, CYCLE, rank)
+        self.kpre, self.vpre, self.offpre = prefill(self.cache, wl, self.lens_pre, self.ptd)
+        self.step_k, self.step_v, self.step_q, self.lens_old, self.lens_new = [], [], [], [], []
+        for c in range(CYCLE):
+            kn, vn = synth.gen_step_kv(wl, c, device="cuda")
+            self.step_k.append(kn.contiguous())
+            self.step_v.append(vn.contiguous())
+            self.step_q.append(synth.gen_q(wl, step=c, device="cuda"))
+            self.lens_old.append(torch.as_tensor(self.lens_pre + c, dtype=torch.int32, device="cuda"))
+            self.lens_new.append(torch.as_tensor(self.lens_pre + c + 1, dtype=torch.int32, device="cuda"))
+        self.out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
+        self.ws_buf = self.cache.workspace(wl.B, wl.Hq)
+        self.K = K
+
+    def step(self, s):
+        c = s % CYCLE
+        self.K.kv4_append(self.cache.handle, self.step_k[c], self.step_v[c], None, self.lens_old[c], self.ptd)
+        self.K.kv4_decode_attn(self.cache.handle, self.step_q[c], self.lens_new[c], self.ptd, self.wl.softmax_scale,
+                               self.ws_buf, self.out)
+
+    def positions(self, steps):
+        """KV positions attended by the given steps (sum over sequences of the length)."""
+        base = int(self.lens_pre.astype(np.int64).sum())
+        return float(sum(base + self.wl.B * (s % CYCLE + 1) for s in steps))
+
+    def mean_lens(self):
+        return self.lens_pre.astype(np.int64) + CYCLE // 2
+
+    def check(self, what):
+        st, bits = self.cache.get_error()
+        assert st == self.K.KV4_OK, ("device error " + what, st, bits)
+
+    def timed(self, s0, steps, ws, sampler=None):
+        """Device time (ms, this rank) of `steps` consecutive steps from s0,
+        bracketed by a barrier and a device synchronise."""
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(ws)
+        torch.cuda.synchronize()
+        ctx = sampler if sampler is not None else _Null()
+        with ctx:
+            e0.record(stream)
+            for s in range(s0, s0 + steps):
+                self.step(s)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        barrier(ws)
+        return e0.elapsed_time(e1)
+
+    def worker_pass(self, n):
+        """The decode worker kernel of n consecutive steps, each launch timed with
+        CUDA events on its stream (a pass of its own: an event between two kernels
+        keeps the second from starting early under programmatic dependent
+        launch, so the throughput steps carry none). Returns per-launch us."""
+        K = self.K
+        K.kv4_timing_enable(n, 1)
+        for s in range(n):
+            self.step(s)
+        torch.cuda.synchronize()
+        ms = K.kv4_timing_read_each(0, n)
+        K.kv4_timing_disable()
+        return [1e3 * x for x in ms]
+
+    def e2e(self, n, ws):
+        """The same steps through the public API with host buffers: every step
+        uploads its k_new, v_new and q from pinned memory and downloads its output.
+        Copies run on a second stream with two buffer sets, so step s+1's upload
+        and step s's download overlap the kernels of step s."""
+        K, wl = self.K, self.wl
+        hk = [t.cpu().pin_memory() for t in self.step_k]
+        hv = [t.cpu().pin_memory() for t in self.step_v]
+        hq = [t.cpu().pin_memory() for t in self.step_q]
+        dk = [torch.empty_like(self.step_k[0]) for _ in range(2)]
+        dv = [torch.empty_like(self.step_v[0]) for _ in range(2)]
+        dq = [torch.empty_like(self.step_q[0]) for _ in range(2)]
+        dout = [torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        hout = [torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        comp = torch.cuda.current_stream()
+        copy = torch.cuda.Stream()
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        out_copied = [torch.cuda.Event() for _ in range(2)]
+
+        def upload(s):
+            i, c = s % 2, s % CYCLE
+            with torch.cuda.stream(copy):
+                dk[i].copy_(hk[c], non_blocking=True)
+                dv[i].copy_(hv[c], non_blocking=True)
+                dq[i].copy_(hq[c], non_blocking=True)
+                in_ready[i].record(copy)
+
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(ws)
+        torch.cuda.synchronize()
+        e0.record(comp)
+        copy.wait_event(e0)
+        upload(0)
+        for s in range(n):
+            i, c = s % 2, s % CYCLE
+            comp.wait_event(in_ready[i])
+            if s >= 2:
+                comp.wait_event(out_copied[i])
+            K.kv4_append(self.cache.handle, dk[i], dv[i], None, self.lens_old[c], self.ptd)
+            K.kv4_decode_attn(self.cache.handle, dq[i], self.lens_new[c], self.ptd, wl.softmax_scale, self.ws_buf,
+                              dout[i])
+            done[i].record(comp)
+            if s + 1 < n:
+                if s >= 1:
+                    copy.wait_event(done[(s + 1) % 2])
+                upload(s + 1)
+            copy.wait_event(done[i])
+            with torch.cuda.stream(copy):
+                hout[i].copy_(dout[i], non_blocking=True)
+                out_copied[i].record(copy)
+        comp.wait_event(out_copied[(n - 1) % 2])
+        e1.record(comp)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1), ws)
+        positions = sum_over_ranks(self.positions(range(n)), ws)
+        h2d = (self.step_k[0].numel() + self.step_v[0].numel() + self.step_q[0].numel()) * 2
+        return {"value": positions / (ms / 1e3), "unit": "KV positions/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": dout[0].numel() * 2, "steps": n,
+                "overlap": "uploads and downloads on a second stream, two buffer sets"}
+
+    def bf16(self, n=50):
+        """The bf16 paged kernel on the same K/V at the prefilled lengths: worker
+        kernel per launch (median) and whole call."""
+        K, wl = self.K, self.wl
+        pages = torch.zeros((self.npages, wl.Hkv, 2, 16, wl.D), dtype=torch.bfloat16, device="cuda")
+        for b in range(wl.B):
+            L = int(self.lens_pre[b])
+            p = torch.arange(L, device="cuda")
+            pid = self.ptd[b][p // 16].long()
+            slot = (p % 16).long()
+            pages[pid, :, 0, slot, :] = self.kpre[int(self.offpre[b]): int(self.offpre[b]) + L]
+            pages[pid, :, 1, slot, :] = self.vpre[int(self.offpre[b]): int(self.offpre[b]) + L]
+        lens_t = torch.as_tensor(self.lens_pre, dtype=torch.int32, device="cuda")
+        o = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
+        wsb = torch.zeros(K.bf16_paged_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device="cuda")
+        fn = lambda: K.bf16_paged_decode_attn(self.step_q[0], pages, self.ptd, lens_t, wl.softmax_scale, wsb, o,
+                                              wl.Hkv)
+        call, _ = time_calls(fn, n)
+        K.kv4_timing_enable(n, 1)
+        for _ in range(n):
+            fn()
+        torch.cuda.synchronize()
+        kern = float(np.median(K.kv4_timing_read_each(1, n)))
+        K.kv4_timing_disable()
+        pos = int(self.lens_pre.astype(np.int64).sum())
+        nbytes = pos * wl.Hkv * 4 * wl.D + int(((self.lens_pre + 15) // 16).sum()) * 4 + wl.B * wl.Hq * wl.D * 2
+        peak, _ = peaks()
+        del pages
+        return {"positions_per_s": pos / (call / 1e3), "call_us": call * 1e3, "worker_us_median": kern * 1e3,
+                "worker_gbs": nbytes / (kern / 1e3) / 1e9, "frac_of_peak": nbytes / (kern / 1e3) / 1e9 / peak}
+
+    def close(self):
+        self.cache.close()
+        for name in ("kpre", "vpre", "step_k", "step_v", "step_q", "out", "ws_buf", "ptd"):
+            setattr(self, name, None)
+        torch.cuda.empty_cache()
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def roofline(st, worker_us, peak, peak_src):
+    """Roofline object of the decode worker kernel: algorithmic bytes at the
+    cycle's mean lengths over the median of per-launch event timings."""
+    wbytes = worker_bytes(st.mean_lens(), st.wl)
+    med = float(np.median(worker_us))
+    achieved = wbytes / (med / 1e6) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": None, "kernel": "kv4_decode_kernel (page-major workers)",
+            "algorithmic_bytes_per_launch": wbytes, "launches": len(worker_us), "median_us": med,
+            "mean_us": float(np.mean(worker_us)), "peak_source": peak_src}
+
+
+def measure_workload(name, steps=128, warmup=16, ws=1, rank=0, bf16=True):
+    """Steady-state figures of one workload: positions/s of whole steps, the
+    worker kernel against the roofline, end to end with host buffers, and the
+    bf16 kernel on the same data."""
+    from compressed_kv_cache_kv4_b200 import synth
+    wl = synth.workload(name)
+    st = Steady(wl, rank)
+    for s in range(warmup):
+        st.step(s)
+    ms = st.timed(warmup, steps, ws)
+    st.check(name)
+    peak, src = peaks()
+    rf = roofline(st, st.worker_pass(max(64, CYCLE)), peak, src)
+    res = {"workload": workload_config(wl)["workload"], "positions_per_step": st.positions(range(steps)) / steps,
+           "ms_per_step": ms / steps, "positions_per_s": st.positions(range(warmup, warmup + steps)) / (ms / 1e3),
+           "worker_us_median": rf["median_us"], "worker_gbs": rf["achieved"], "worker_frac_of_peak": rf["frac"],
+           "worker_launches": rf["launches"], "e2e": st.e2e(64, ws)}
+    if bf16:
+        res["bf16"] = st.bf16()
+        res["kv4_speedup_over_bf16_worker"] = res["bf16"]["worker_us_median"] / rf["median_us"]
+    st.check(name)
+    st.close()
+    return res
+
+
 def run_kv4(args, ws, rank):
-    import compressed_kv_cache_kv4_b200 as K
     from compressed_kv_cache_kv4_b200 import synth
 
     dev = torch.cuda.current_device()
@@ -268,153 +485,42 @@ def run_kv4(args, ws, rank):
     if args.recent is not None:
         wl.recent = args.recent
     wl.seed += 7919 * rank                      # each rank its own batch (same length law)
-    L0 = wl.lens.astype(np.int64)
-    lens_pre = np.maximum(L0 - CYCLE, 0).astype(np.int32)
-    cache, ptd, pt_np, npages = build_kv4(wl, L0, CYCLE, rank)
-    kpre, vpre, offpre = prefill(cache, wl, lens_pre, ptd)
-
-    # per-cycle-step inputs, resident on the device
-    step_k, step_v, step_q, lens_old, lens_new = [], [], [], [], []
-    for c in range(CYCLE):
-        kn, vn = synth.gen_step_kv(wl, c, device="cuda")
-        step_k.append(kn.contiguous())
-        step_v.append(vn.contiguous())
-        step_q.append(synth.gen_q(wl, step=c, device="cuda"))
-        lens_old.append(torch.as_tensor(lens_pre + c, dtype=torch.int32, device="cuda"))
-        lens_new.append(torch.as_tensor(lens_pre + c + 1, dtype=torch.int32, device="cuda"))
-    offs = torch.arange(wl.B + 1, dtype=torch.int32, device="cuda")
-    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
-    ws_buf = cache.workspace(wl.B, wl.Hq)
-    handle = cache.handle
-
-    def step(s):
-        c = s % CYCLE
-        K.kv4_append(handle, step_k[c], step_v[c], None, lens_old[c], ptd)
-        K.kv4_decode_attn(handle, step_q[c], lens_new[c], ptd, wl.softmax_scale, ws_buf, out)
-
+    st = Steady(wl, rank)
     for s in range(args.warmup):
-        step(s)
+        st.step(s)
     torch.cuda.synchronize()
-    st, bits = cache.get_error()
-    assert st == K.KV4_OK, ("device error before timing", st, bits)
-
-    # the worker kernel is timed with CUDA events on every TIMING_EVERY-th step
-    # of the timed region (an event between two kernels stops the next one from
-    # starting early, so timing every step would slow the steps it measures)
-    K.kv4_timing_enable(args.steps, TIMING_EVERY)
-    stream = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(ws)
-    torch.cuda.synchronize()
+    st.check("before timing")
     with ClockSampler(dev) as clk:
-        e0.record(stream)
-        for s in range(args.warmup, args.warmup + args.steps):
-            step(s)
-        e1.record(stream)
-        torch.cuda.synchronize()
-    barrier(ws)
-    elapsed_ms = e0.elapsed_time(e1)
-    worker_ms, worker_n = K.kv4_timing_read(0)
-    K.kv4_timing_disable()
-    st, bits = cache.get_error()
-    assert st == K.KV4_OK, ("device error in timed region", st, bits)
-
-    cyc = [(args.warmup + s) % CYCLE for s in range(args.steps)]
-    positions = float(sum(int(lens_pre.astype(np.int64).sum()) + wl.B * (c + 1) for c in cyc))
+        elapsed_ms = st.timed(args.warmup, args.steps, ws)
+    st.check("in timed region")
+    positions = st.positions(range(args.warmup, args.warmup + args.steps))
     value, elapsed_max = aggregate(positions, elapsed_ms, ws)
-    mean_lens = lens_pre.astype(np.int64) + CYCLE // 2
-    wbytes = worker_bytes(mean_lens, wl)
-    sbytes = step_bytes(mean_lens, wl)
-    worker_avg_ms = worker_ms / max(worker_n, 1)
     peak, peak_src = peaks()
-    achieved = wbytes / (worker_avg_ms / 1e3) / 1e9
-
+    worker_us = st.worker_pass(max(64, CYCLE))
+    rf = roofline(st, worker_us, peak, peak_src)
+    rf["traffic"] = ncu_traffic(rf["algorithmic_bytes_per_launch"])
+    sbytes = step_bytes(st.mean_lens(), wl)
     res = {
         "elapsed_ms": elapsed_max, "ms_per_step": elapsed_max / args.steps, "value": value,
         "positions_per_step": positions / args.steps, "clocks": clk.summary(),
         "step_gbs": sbytes / (elapsed_max / args.steps / 1e3) / 1e9,
-        "worker_avg_us": worker_avg_ms * 1e3, "worker_launches_timed": worker_n,
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic(wbytes),
-                     "kernel": "decode_kernel (split-K worker)", "algorithmic_bytes_per_launch": wbytes,
-                     "peak_source": peak_src},
+        "worker_avg_us": rf["mean_us"], "roofline": rf,
         "gpu_launches": 3 * args.steps,   # per step: append, decode workers, merge
     }
-
-    if rank == 0 and not args.no_secondary and args.workload == "qwen8b":
-        res["secondary"] = secondary(wl, L0, cache, ptd, pt_np, npages, kpre, vpre, offpre, lens_pre, step_k,
-                                     step_v, step_q)
     # e2e through host buffers: per step H2D of (k_new, v_new, q) from pinned memory, D2H of the output
-    res["e2e"] = e2e(wl, handle, ptd, lens_old, lens_new, offs, step_k, step_v, step_q, ws_buf, lens_pre, ws,
-                     min(args.steps, 512))
+    res["e2e"] = st.e2e(max(64, min(args.steps, 512)), ws)
+    st.check("after e2e")
+    if rank == 0 and not args.no_secondary and args.workload == "qwen8b":
+        res["secondary"] = secondary(st)
     if rank == 0 and not args.no_cpu:
-        res["cpu_baseline"] = cpu_baseline(wl, kpre, vpre, offpre, lens_pre)
+        res["cpu_baseline"] = cpu_baseline(wl, st.kpre, st.vpre, st.offpre, st.lens_pre)
         if "secondary" in res:   # the oracle beside the other measured rows
             res["cpu_baseline"]["rows"] = cpu_rows()
-    cache.close()
+    st.close()
+    if rank == 0 and not args.no_secondary and args.workload == "qwen8b":
+        # the other four workloads in steady state, each next to the bf16 kernel on its data
+        res["secondary"]["workloads"] = {name: measure_workload(name) for name in ("async", "long", "evict", "tiny")}
     return wl, res
-
-
-def e2e(wl, handle, ptd, lens_old, lens_new, offs, step_k, step_v, step_q, ws_buf, lens_pre, ws, n):
-    """The same steps through the public API with host buffers: every step
-    uploads its k_new, v_new and q from pinned memory and downloads its output.
-    Copies run on a second stream with two buffer sets, so step s+1's upload and
-    step s's download overlap the kernels of step s."""
-    import compressed_kv_cache_kv4_b200 as K
-    hk = [t.cpu().pin_memory() for t in step_k]
-    hv = [t.cpu().pin_memory() for t in step_v]
-    hq = [t.cpu().pin_memory() for t in step_q]
-    dk = [torch.empty_like(step_k[0]) for _ in range(2)]
-    dv = [torch.empty_like(step_v[0]) for _ in range(2)]
-    dq = [torch.empty_like(step_q[0]) for _ in range(2)]
-    dout = [torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    hout = [torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    comp = torch.cuda.current_stream()
-    copy = torch.cuda.Stream()
-    in_ready = [torch.cuda.Event() for _ in range(2)]
-    done = [torch.cuda.Event() for _ in range(2)]
-    out_copied = [torch.cuda.Event() for _ in range(2)]
-
-    def upload(s):
-        i, c = s % 2, s % CYCLE
-        with torch.cuda.stream(copy):
-            dk[i].copy_(hk[c], non_blocking=True)
-            dv[i].copy_(hv[c], non_blocking=True)
-            dq[i].copy_(hq[c], non_blocking=True)
-            in_ready[i].record(copy)
-
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(ws)
-    torch.cuda.synchronize()
-    e0.record(comp)
-    copy.wait_event(e0)
-    upload(0)
-    for s in range(n):
-        i, c = s % 2, s % CYCLE
-        comp.wait_event(in_ready[i])
-        if s >= 2:
-            comp.wait_event(out_copied[i])
-        K.kv4_append(handle, dk[i], dv[i], None, lens_old[c], ptd)
-        K.kv4_decode_attn(handle, dq[i], lens_new[c], ptd, wl.softmax_scale, ws_buf, dout[i])
-        done[i].record(comp)
-        if s + 1 < n:
-            if s >= 1:
-                copy.wait_event(done[(s + 1) % 2])
-            upload(s + 1)
-        copy.wait_event(done[i])
-        with torch.cuda.stream(copy):
-            hout[i].copy_(dout[i], non_blocking=True)
-            out_copied[i].record(copy)
-    comp.wait_event(out_copied[(n - 1) % 2])
-    e1.record(comp)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), ws)
-    positions = sum(int(lens_pre.astype(np.int64).sum()) + wl.B * (s % CYCLE + 1) for s in range(n))
-    positions = sum_over_ranks(float(positions), ws)
-    h2d = (step_k[0].numel() + step_v[0].numel() + step_q[0].numel()) * 2
-    return {"value": positions / (ms / 1e3), "unit": "KV positions/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": dout[0].numel() * 2, "steps": n,
-            "overlap": "uploads and downloads on a second stream, two buffer sets"}
 
 
 def time_calls(fn, n, kind=None):
@@ -440,16 +546,18 @@ def time_calls(fn, n, kind=None):
     return call_ms, kern_ms
 
 
-def secondary(wl, L0, cache, ptd, pt_np, npages, kpre, vpre, offpre, lens_pre, step_k, step_v, step_q):
-    """Comparisons on the same data: bf16 kernel, pure INT4 (no INT8 protection),
-    and the eviction path (top-k + masked decode)."""
+def secondary(st):
+    """Comparisons on the qwen8b data: decode only, pure INT4 (no INT8
+    protection), the bf16 kernel, the prefill append, the eviction path (top-k +
+    masked decode, page eviction) and the learner-side attention."""
     import compressed_kv_cache_kv4_b200 as K
-    from compressed_kv_cache_kv4_b200 import synth
+    wl, cache, ptd = st.wl, st.cache, st.ptd
+    lens_pre, kpre, vpre, offpre = st.lens_pre, st.kpre, st.vpre, st.offpre
     out = {}
     peak, _ = peaks()
     lens_t = torch.as_tensor(lens_pre, dtype=torch.int32, device="cuda")
     pos = int(lens_pre.astype(np.int64).sum())
-    q0 = step_q[0]
+    q0 = st.step_q[0]
     o = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
     ws_buf = cache.workspace(wl.B, wl.Hq)
 
@@ -461,7 +569,7 @@ def secondary(wl, L0, cache, ptd, pt_np, npages, kpre, vpre, offpre, lens_pre, s
                               "worker_gbs": wb / (kern / 1e3) / 1e9, "frac_of_peak": wb / (kern / 1e3) / 1e9 / peak}
 
     # pure KV4 (sink = recent = 0): the throughput ratio the KV4-RL review quotes (~94%)
-    pure, _, _, _ = build_kv4(wl, L0, CYCLE, 0, sink=0, recent=0)
+    pure, _, _, _ = build_kv4(wl, wl.lens.astype(np.int64), CYCLE, 0, sink=0, recent=0)
     pure.append(kpre, vpre, torch.as_tensor(offpre.astype(np.int32), device="cuda"),
                 torch.zeros(wl.B, dtype=torch.int32, device="cuda"), ptd)
     wsp = pure.workspace(wl.B, wl.Hq)
@@ -474,23 +582,8 @@ def secondary(wl, L0, cache, ptd, pt_np, npages, kpre, vpre, offpre, lens_pre, s
     del pure
 
     # bf16 paged kernel on the same K/V
-    pages = torch.zeros((npages, wl.Hkv, 2, 16, wl.D), dtype=torch.bfloat16, device="cuda")
-    for b in range(wl.B):
-        L = int(lens_pre[b])
-        p = torch.arange(L, device="cuda")
-        pid = ptd[b][p // 16].long()
-        slot = (p % 16).long()
-        pages[pid, :, 0, slot, :] = kpre[int(offpre[b]): int(offpre[b]) + L]
-        pages[pid, :, 1, slot, :] = vpre[int(offpre[b]): int(offpre[b]) + L]
-    wsb = torch.zeros(K.bf16_paged_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.D), dtype=torch.uint8, device="cuda")
-    callb, kernb = time_calls(lambda: K.bf16_paged_decode_attn(q0, pages, ptd, lens_t, wl.softmax_scale, wsb, o,
-                                                               wl.Hkv), 100, kind=1)
-    bbytes = pos * wl.Hkv * 4 * wl.D + int(((lens_pre + 15) // 16).sum()) * 4 + wl.B * wl.Hq * wl.D * 2
-    out["bf16_decode_only"] = {"positions_per_s": pos / (callb / 1e3), "call_us": callb * 1e3,
-                               "worker_us": kernb * 1e3, "worker_gbs": bbytes / (kernb / 1e3) / 1e9,
-                               "frac_of_peak": bbytes / (kernb / 1e3) / 1e9 / peak,
-                               "kv4_speedup": callb / call}
-    del pages
+    out["bf16_decode_only"] = st.bf16(100)
+    out["bf16_decode_only"]["kv4_speedup"] = out["bf16_decode_only"]["call_us"] / (call * 1e3)
 
     # prefill: append of every prompt position (rewrites the same bytes each call)
     offs_t = torch.as_tensor(offpre.astype(np.int32), device="cuda")
@@ -664,6 +757,21 @@ def learner_secondary(steps=20):
 
 
 # ---------------------------------------------------------------------------- CPU oracle
+def oracle_build_flags():
+    from oracle import build as ob
+    return "gcc " + " ".join(ob.FLAGS)
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def oracle_threads():
     try:
         import ctypes
@@ -718,7 +826,8 @@ def cpu_baseline(wl, k, v, off, lens_pre, budget_s=20.0):
         b += 8
     return {"value": total_pos / total_t, "unit": "KV positions/s", "cores": oracle_threads(), "kind": "oracle",
             "sample": "%d of %d sequences of the %s workload (%d positions): oracle cache image + fp64 decode, "
-                      "%.1f s" % (len(seqs_done), wl.B, wl.name, total_pos, total_t)}
+                      "%.1f s" % (len(seqs_done), wl.B, wl.name, total_pos, total_t),
+            "build": oracle_build_flags(), "cpu": cpu_model()}
 
 
 def cpu_rows():
@@ -800,7 +909,8 @@ def run_reference(args, ws, rank):
                              "kind": "oracle",
                              "sample": "%d %s per step of the %s workload: oracle cache image + fp64 decode"
                                        % (per_step, "(sequence, KV head) pair(s)" if head_mode else "sequence(s)",
-                                          wl.name)},
+                                          wl.name),
+                             "build": oracle_build_flags(), "cpu": cpu_model()},
             "e2e": {"value": value, "unit": "KV positions/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
 
