@@ -544,31 +544,31 @@ struct RangeCtx {
 // accumulator start removes the offsets), exact running-max softmax, P.V on
 // fp16 tiles with V^T codes and P * scale_V as hi + lo fp16 columns.
 template <int D, int G>
-__device__ __forceinline__ void int4_item(const DecodeParams &p, const uint8_t *stg, const uint8_t *qsm, int pg,
+__device__ __forceinline__ void int4_item(const DecodeParams &p, uint32_t stg, uint32_t qsm, int pg,
                                           const RangeCtx &rc, SoftmaxState<D / 16> &st, int lane) {
   constexpr int NG = D / 32, NMT = D / 16, NSW = (NG + 1) / 2;
   const int g = lane >> 2, t = lane & 3;
   uint32_t kw0[NG], kw1[NG], ksw0[NSW], ksw1[NSW], vsw0[NSW], vsw1[NSW];
   if constexpr (NG == 4) {
-    const uint4 a0 = *reinterpret_cast<const uint4 *>(stg + g * (D / 2) + t * (D / 8));
-    const uint4 a1 = *reinterpret_cast<const uint4 *>(stg + (g + 8) * (D / 2) + t * (D / 8));
+    const uint4 a0 = lds128(stg + g * (D / 2) + t * (D / 8));
+    const uint4 a1 = lds128(stg + (g + 8) * (D / 2) + t * (D / 8));
     kw0[0] = a0.x; kw0[1] = a0.y; kw0[2] = a0.z; kw0[3] = a0.w;
     kw1[0] = a1.x; kw1[1] = a1.y; kw1[2] = a1.z; kw1[3] = a1.w;
-    const uint2 s0 = *reinterpret_cast<const uint2 *>(stg + 16 * D + g * 8);
-    const uint2 s1 = *reinterpret_cast<const uint2 *>(stg + 16 * D + (g + 8) * 8);
-    const uint2 u0 = *reinterpret_cast<const uint2 *>(stg + 17 * D + g * 8);
-    const uint2 u1 = *reinterpret_cast<const uint2 *>(stg + 17 * D + (g + 8) * 8);
+    const uint2 s0 = lds64(stg + 16 * D + g * 8);
+    const uint2 s1 = lds64(stg + 16 * D + (g + 8) * 8);
+    const uint2 u0 = lds64(stg + 17 * D + g * 8);
+    const uint2 u1 = lds64(stg + 17 * D + (g + 8) * 8);
     ksw0[0] = s0.x; ksw0[1] = s0.y; ksw1[0] = s1.x; ksw1[1] = s1.y;
     vsw0[0] = u0.x; vsw0[1] = u0.y; vsw1[0] = u1.x; vsw1[1] = u1.y;
   } else {
-    const uint2 a0 = *reinterpret_cast<const uint2 *>(stg + g * (D / 2) + t * (D / 8));
-    const uint2 a1 = *reinterpret_cast<const uint2 *>(stg + (g + 8) * (D / 2) + t * (D / 8));
+    const uint2 a0 = lds64(stg + g * (D / 2) + t * (D / 8));
+    const uint2 a1 = lds64(stg + (g + 8) * (D / 2) + t * (D / 8));
     kw0[0] = a0.x; kw0[1] = a0.y;
     kw1[0] = a1.x; kw1[1] = a1.y;
-    ksw0[0] = *reinterpret_cast<const uint32_t *>(stg + 16 * D + g * 4);
-    ksw1[0] = *reinterpret_cast<const uint32_t *>(stg + 16 * D + (g + 8) * 4);
-    vsw0[0] = *reinterpret_cast<const uint32_t *>(stg + 17 * D + g * 4);
-    vsw1[0] = *reinterpret_cast<const uint32_t *>(stg + 17 * D + (g + 8) * 4);
+    ksw0[0] = lds32(stg + 16 * D + g * 4);
+    ksw1[0] = lds32(stg + 16 * D + (g + 8) * 4);
+    vsw0[0] = lds32(stg + 17 * D + g * 4);
+    vsw1[0] = lds32(stg + 17 * D + (g + 8) * 4);
   }
   float ks0[NG], ks1[NG], vs0a[NG], vs1a[NG];
 #pragma unroll
@@ -583,9 +583,9 @@ __device__ __forceinline__ void int4_item(const DecodeParams &p, const uint8_t *
   float2 sc01 = make_float2(0.f, 0.f), sc23 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < NG; ++i) {
-    const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + i * 512 + lane * 16);
+    const uint4 qv = lds128(qsm + i * 512 + lane * 16);
     // accumulator start of columns 2t, 2t+1 (query heads 2t & 3, (2t & 3) + 1)
-    const float2 qi = *reinterpret_cast<const float2 *>(qsm + NG * 512 + 16 * i + 8 * (t & 1));
+    const float2 qi = lds64f(qsm + NG * 512 + 16 * i + 8 * (t & 1));
     float acc[4];
     const uint32_t k80 = kw0[i] >> 8, k81 = kw1[i] >> 8;
     {   // elements 0, 4 (k-slots 2t, 2t+1) and 2, 6 (2t+8, 2t+9): bf16, 136 + c
@@ -632,7 +632,7 @@ __device__ __forceinline__ void int4_item(const DecodeParams &p, const uint8_t *
   uint32_t vw[NMT];
 #pragma unroll
   for (int q4 = 0; q4 < NMT / 4; ++q4) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(stg + 8 * D + q4 * 512 + lane * 16);
+    const uint4 w = lds128(stg + 8 * D + q4 * 512 + lane * 16);
     vw[4 * q4 + 0] = w.x;
     vw[4 * q4 + 1] = w.y;
     vw[4 * q4 + 2] = w.z;
@@ -666,7 +666,7 @@ __device__ __forceinline__ int side_row_pos(const DecodeParams &p, const RangeCt
 // K half of INT8 side page j: q.K on fp16 tiles (codes exact in fp16), softmax,
 // and the P * scale_V weights (hi + lo) kept for the V half that follows.
 template <int D>
-__device__ __forceinline__ void int8k_item(const DecodeParams &p, const uint8_t *stg, const uint8_t *qsm, int j,
+__device__ __forceinline__ void int8k_item(const DecodeParams &p, uint32_t stg, uint32_t qsm, int j,
                                            const RangeCtx &rc, SoftmaxState<D / 16> &st, uint32_t &wb0,
                                            uint32_t &wb1, int lane) {
   constexpr int NJ = D / 16, NMT = D / 16, NW = D / 8;
@@ -674,7 +674,7 @@ __device__ __forceinline__ void int8k_item(const DecodeParams &p, const uint8_t 
   uint32_t kw[NW];
 #pragma unroll
   for (int c = 0; c < NW / 4; ++c) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(stg + c * 512 + lane * 16);
+    const uint4 w = lds128(stg + c * 512 + lane * 16);
     kw[4 * c + 0] = w.x;
     kw[4 * c + 1] = w.y;
     kw[4 * c + 2] = w.z;
@@ -683,7 +683,7 @@ __device__ __forceinline__ void int8k_item(const DecodeParams &p, const uint8_t 
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int jj = 0; jj < NJ; jj += 2) {
-    const uint4 qv = *reinterpret_cast<const uint4 *>(qsm + (jj / 2) * 512 + lane * 16);
+    const uint4 qv = lds128(qsm + (jj / 2) * 512 + lane * 16);
     const uint32_t a0[4] = {i8x2_to_f16x2(kw[jj]), i8x2_to_f16x2(kw[NJ + jj]), i8x2_to_f16x2(kw[jj] >> 8),
                             i8x2_to_f16x2(kw[NJ + jj] >> 8)};
     mma_f16(acc, a0, qv.x, qv.y);
@@ -691,9 +691,8 @@ __device__ __forceinline__ void int8k_item(const DecodeParams &p, const uint8_t 
                             i8x2_to_f16x2(kw[jj + 1] >> 8), i8x2_to_f16x2(kw[NJ + jj + 1] >> 8)};
     mma_f16(acc, a1, qv.z, qv.w);
   }
-  const __half *ks = reinterpret_cast<const __half *>(stg + 16 * D);
-  const __half *vs = reinterpret_cast<const __half *>(stg + 16 * D + 32);
-  const float k0 = __half2float(ks[g]) * p.scale_log2, k1 = __half2float(ks[g + 8]) * p.scale_log2;
+  const float k0 = half_bits_to_f32(lds16(stg + 16 * D + 2 * g)) * p.scale_log2;
+  const float k1 = half_bits_to_f32(lds16(stg + 16 * D + 2 * (g + 8))) * p.scale_log2;
   const bool v0 = side_row_pos(p, rc, j, g) >= 0, v1 = side_row_pos(p, rc, j, g + 8) >= 0;
   float sl[4];
   sl[0] = v0 ? acc[0] * k0 : -INFINITY;
@@ -702,19 +701,20 @@ __device__ __forceinline__ void int8k_item(const DecodeParams &p, const uint8_t 
   sl[3] = v1 ? acc[3] * k1 : -INFINITY;
   float pr[4];
   softmax_update<NMT, 0>(st, sl, pr);
-  const float s0 = __half2float(vs[g]), s1 = __half2float(vs[g + 8]);
+  const float s0 = half_bits_to_f32(lds16(stg + 16 * D + 32 + 2 * g));
+  const float s1 = half_bits_to_f32(lds16(stg + 16 * D + 32 + 2 * (g + 8)));
   weights_f16(pr[0] * s0, pr[1] * s0, pr[2] * s1, pr[3] * s1, t >= 2 ? 1.f : 0.f, wb0, wb1);
 }
 
 // V half of an INT8 side page: P.V on fp16 tiles with the weights of the K half.
 template <int D>
-__device__ __forceinline__ void int8v_item(const uint8_t *stg, SoftmaxState<D / 16> &st, uint32_t wb0, uint32_t wb1,
+__device__ __forceinline__ void int8v_item(uint32_t stg, SoftmaxState<D / 16> &st, uint32_t wb0, uint32_t wb1,
                                            int lane) {
   constexpr int NMT = D / 16, NW = D / 8;
   uint32_t vw[NW];
 #pragma unroll
   for (int c = 0; c < NW / 4; ++c) {
-    const uint4 w = *reinterpret_cast<const uint4 *>(stg + c * 512 + lane * 16);
+    const uint4 w = lds128(stg + c * 512 + lane * 16);
     vw[4 * c + 0] = w.x;
     vw[4 * c + 1] = w.y;
     vw[4 * c + 2] = w.z;
@@ -744,6 +744,7 @@ __global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
   int *plan = reinterpret_cast<int *>(smem + lay.plan);   // [NVB + 1]
   int *wtot = reinterpret_cast<int *>(smem + lay.wtot);   // [8]
   const int stage_bytes = HB * 18 * D;
+  const uint32_t smem_base = smem_u32(smem), qsm_u32 = smem_u32(qsm);
 
   if (tid < NS) {
     mbar_init(&full[tid], 1);
@@ -857,9 +858,9 @@ __global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
         break;
       }
       phase ^= 1u << s;
-      const uint8_t *stg = smem + s * stage_bytes + warp * 18 * D;
-      if (kind == kItemInt4) int4_item<D, G>(p, stg, qsm, pj, rc, st, lane);
-      else if (kind == kItemInt8K) int8k_item<D>(p, stg, qsm, pj, rc, st, wb0, wb1, lane);
+      const uint32_t stg = smem_base + s * stage_bytes + warp * 18 * D;
+      if (kind == kItemInt4) int4_item<D, G>(p, stg, qsm_u32, pj, rc, st, lane);
+      else if (kind == kItemInt8K) int8k_item<D>(p, stg, qsm_u32, pj, rc, st, wb0, wb1, lane);
       else int8v_item<D>(stg, st, wb0, wb1, lane);
       // release the stage (no result to wait for); one warp per item, in
       // turn, refills the stage of the item before this one once every warp
