@@ -520,7 +520,46 @@ def run_kv4(args, ws, rank):
     if rank == 0 and not args.no_secondary and args.workload == "qwen8b":
         # the other four workloads in steady state, each next to the bf16 kernel on its data
         res["secondary"]["workloads"] = {name: measure_workload(name) for name in ("async", "long", "evict", "tiny")}
+        res["secondary"]["context_parallel"] = cp_secondary()
     return wl, res
+
+
+def cp_secondary(n_shards=(2, 4, 8), steps=50):
+    """Context-parallel decode of the long workload (4 x 131072 positions) on
+    this GPU: each page-range shard decoded by kv4_decode_partials, one after
+    another, and the partials merged by kv4_merge_partials. On N GPUs each rank
+    runs one shard and all-gathers (D + 4) * 4 bytes per (sequence, query head)
+    before the merge; that exchange is not measured here (one GPU)."""
+    import compressed_kv_cache_kv4_b200 as K
+    from compressed_kv_cache_kv4_b200 import cp, synth
+    wl = synth.workload("long")
+    cache, ptd, _, _ = build_kv4(wl, wl.lens, 0, 0)
+    k, v, _ = prefill(cache, wl, wl.lens, ptd)
+    del k, v
+    q = synth.gen_q(wl, device="cuda")
+    lens = torch.as_tensor(wl.lens, device="cuda")
+    ws = cache.workspace(wl.B, wl.Hq)
+    o = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
+    single, _ = time_calls(lambda: K.kv4_decode_attn(cache.handle, q, lens, ptd, wl.softmax_scale, ws, o), steps)
+    res = {"workload": "long: B=4, L=131072, 32/8 heads, D=128", "single_call_us": single * 1e3,
+           "partial_bytes_per_rank": wl.B * wl.Hq * (wl.D + 4) * 4, "exchange": "not measured (one GPU)"}
+    for n in n_shards:
+        pb, pe = cp.shard_pages(wl.lens, n, wl.sink, wl.recent)
+        pbt = [torch.as_tensor(pb[r], device="cuda") for r in range(n)]
+        pet = [torch.as_tensor(pe[r], device="cuda") for r in range(n)]
+        parts = torch.empty((n, wl.B, wl.Hq, wl.D + 4), dtype=torch.float32, device="cuda")
+        per = []
+        for r in range(n):
+            t, _ = time_calls(lambda: K.kv4_decode_partials(cache.handle, q, lens, ptd, wl.softmax_scale, ws, parts[r],
+                                                            pbt[r], pet[r], with_int8=(r == n - 1)), steps)
+            per.append(t * 1e3)
+        merge, _ = time_calls(lambda: K.kv4_merge_partials(parts, o), steps)
+        res["%d_shards" % n] = {"shard_call_us": per, "max_shard_us": max(per), "merge_us": merge * 1e3,
+                                "step_us_if_one_gpu_per_shard": max(per) + merge * 1e3}
+    st, bits = cache.get_error()
+    res["device_error"] = bits
+    cache.close()
+    return res
 
 
 def time_calls(fn, n, kind=None):
@@ -625,17 +664,39 @@ def evict_secondary(steps=50, page_only=False):
     o = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
     wsb = cache.workspace(wl.B, wl.Hq)
     res = {}
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def topk_flushed(permille, reps=20):
+        """kv_topk_retain timed alone after a 256 MB read evicts the scores from L2."""
+        ms = []
+        for r in range(reps + 3):
+            flush.max()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda._sleep(100000)   # the GPU stays busy until the launch below is queued
+            e0.record(stream)
+            K.kv_topk_retain(scores, lens, permille, mask, count, max_len=L)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if r >= 3:
+                ms.append(e0.elapsed_time(e1))
+        return float(np.median(ms))
+
     for permille in (100, 300, 500, 900, 1000):
         tk, _ = time_calls(lambda: K.kv_topk_retain(scores, lens, permille, mask, count, max_len=L), steps)
+        tkf = topk_flushed(permille)
         call, kern = time_calls(lambda: K.kv4_decode_attn(cache.handle, q, lens, ptd, wl.softmax_scale, wsb, o,
                                                           retain_mask=mask), steps, kind=0)
         kept = int(count.sum().item()) / wl.Hkv
-        res["%d" % permille] = {"topk_us": tk * 1e3, "masked_decode_us": call * 1e3, "worker_us": kern * 1e3,
+        res["%d" % permille] = {"topk_us": tk * 1e3, "topk_us_l2_flushed": tkf * 1e3,
+                                "masked_decode_us": call * 1e3, "worker_us": kern * 1e3,
                                 "retained_positions_per_s": kept / ((tk + call) / 1e3),
-                                "topk_gbs": wl.B * wl.Hkv * L * 4 / (tk / 1e3) / 1e9}
+                                "topk_gbs": wl.B * wl.Hkv * L * 4 / (tk / 1e3) / 1e9,
+                                "topk_gbs_l2_flushed": wl.B * wl.Hkv * L * 4 / (tkf / 1e3) / 1e9}
     call, kern = time_calls(lambda: K.kv4_decode_attn(cache.handle, q, lens, ptd, wl.softmax_scale, wsb, o), steps,
                             kind=0)
     res["unmasked_decode_us"] = call * 1e3
+    del flush
     res["page_evict"] = page_evict_secondary(wl, cache, scores, lens, ptd, q, o, wsb)
     st, bits = cache.get_error()
     res["device_error"] = bits

@@ -7,8 +7,10 @@ been built, importing the compute entry points raises ImportError; there is no
 fallback implementation.
 
 Names mirror the C ABI (kv4_cache_bytes, kv4_cache_create, kv4_append,
-kv4_workspace_bytes, kv4_decode_attn, kv_topk_retain, kv4_evict_pages,
-smd_masked_attn, bf16_paged_decode_attn, kv4_get_error); ``KV4Cache`` bundles the buffers and handle of one cache.
+kv4_workspace_bytes, kv4_decode_attn, kv4_decode_partials, kv4_merge_partials,
+kv_topk_retain, kv4_evict_pages, smd_masked_attn, bf16_paged_decode_attn,
+kv4_get_error); ``KV4Cache`` bundles the buffers and handle of one cache;
+``cp`` holds the context-parallel plumbing (shard plan, gather of partials).
 """
 import ctypes as C
 import os
@@ -62,6 +64,9 @@ def lib():
                                       _P, _I32, _I32]),
         "kv4_decode_attn_noalloc": (C.c_int, [_P, _P, _P, _I32, _P, _P, _I32, _P, _I32, C.c_float, _I32,
                                               _P, _I32, _I32]),
+        "kv4_decode_partials": (C.c_int, [_P, _P, _P, _I32, _P, _P, _I32, _P, _P, _I32, _P, _I32, C.c_float,
+                                          _I32, _P, _SZ, _P, _I32]),
+        "kv4_merge_partials": (C.c_int, [_P, _P, _I32, _I32, _I32, _I32, _P, _I32]),
         "kv_topk_retain": (C.c_int, [_P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P, _I32, _P, _I32]),
         "kv4_evict_pages": (C.c_int, [_P, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P, _I32]),
         "smd_masked_attn": (C.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P, _I32, C.c_float,
@@ -152,6 +157,27 @@ def kv4_decode_attn(handle, q, seq_lens, page_table, softmax_scale, workspace, o
                                num_workers, _ptr(workspace), workspace.numel() * workspace.element_size(),
                                _ptr(out), 1 if out.dtype == torch.float32 else 0, B)
     _check(st, "kv4_decode_attn")
+
+
+def kv4_decode_partials(handle, q, seq_lens, page_table, softmax_scale, workspace, partials, page_begin=None,
+                        page_end=None, with_int8=True, retain_mask=None, num_workers=0, stream=None):
+    """Exact softmax partials (m, l, o) of one page-range shard of every
+    sequence: partials is fp32 [B][Hq][D+4] (m, l, two unused words, o)."""
+    B, Hq, _ = q.shape
+    mstride = 0 if retain_mask is None else retain_mask.shape[-1]
+    st = lib().kv4_decode_partials(handle, _stream(stream), _ptr(q), Hq, _ptr(seq_lens), _ptr(page_table),
+                                   page_table.shape[1], _ptr(page_begin), _ptr(page_end), 1 if with_int8 else 0,
+                                   _ptr(retain_mask), mstride, C.c_float(softmax_scale), num_workers, _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _ptr(partials), B)
+    _check(st, "kv4_decode_partials")
+
+
+def kv4_merge_partials(partials, out, stream=None):
+    """Exact merge of partials [N][B][Hq][D+4] into out [B][Hq][D] (bf16 or fp32)."""
+    N, B, Hq, D4 = partials.shape
+    st = lib().kv4_merge_partials(_stream(stream), _ptr(partials), N, B, Hq, D4 - 4, _ptr(out),
+                                  1 if out.dtype == torch.float32 else 0)
+    _check(st, "kv4_merge_partials")
 
 
 # Size of the fixed per-device scratch of kv4_decode_attn_noalloc (KV4_NOALLOC_SCRATCH_BYTES).

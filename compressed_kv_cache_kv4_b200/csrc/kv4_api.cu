@@ -364,10 +364,18 @@ kv4_status kv4_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t num_q_
   return KV4_OK;
 }
 
-kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_t Hq, const int32_t *seq_lens,
-                           const int32_t *page_table, int32_t pt_stride, const uint32_t *retain_mask,
-                           int32_t mask_stride, float softmax_scale, int32_t num_workers, void *workspace,
-                           size_t ws_bytes, void *out, int32_t out_is_fp32, int32_t B) {
+}  // extern "C"
+
+namespace {
+
+// kv4_decode_attn and kv4_decode_partials: the whole INT4 region and the INT8
+// region of every sequence, or one page-range shard of the INT4 region
+// (page_begin/page_end) with or without the INT8 region.
+kv4_status decode_call(kv4_cache *cache, void *stream, const void *q, int32_t Hq, const int32_t *seq_lens,
+                       const int32_t *page_table, int32_t pt_stride, const int32_t *page_begin,
+                       const int32_t *page_end, int32_t with_int8, const uint32_t *retain_mask, int32_t mask_stride,
+                       float softmax_scale, int32_t num_workers, void *workspace, size_t ws_bytes, void *out,
+                       int32_t out_is_fp32, float *partials, int32_t B) {
   if (!cache || B < 0 || pt_stride < 1 || num_workers < 0) return KV4_ERR_INVALID;
   if (B == 0) return KV4_OK;
   if (B > cache->cfg.max_seqs) return KV4_ERR_CAPACITY;
@@ -376,8 +384,11 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   if (Hq < 1 || Hq % Hkv) return KV4_ERR_INVALID;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4) return KV4_ERR_UNSUPPORTED;
-  if (!q || !seq_lens || !page_table || !workspace || !out) return KV4_ERR_INVALID;
-  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 16)) return KV4_ERR_INVALID;
+  if (!q || !seq_lens || !page_table || !workspace || (!out && !partials)) return KV4_ERR_INVALID;
+  if (!aligned(q, 16) || (out && !aligned(out, 16)) || (partials && !aligned(partials, 16)) ||
+      !aligned(workspace, 16))
+    return KV4_ERR_INVALID;
+  if ((page_begin == nullptr) != (page_end == nullptr)) return KV4_ERR_INVALID;
   if (retain_mask && (long long)mask_stride * 32 < (long long)pt_stride * kPageTokens) return KV4_ERR_INVALID;
   if (!isfinite(softmax_scale)) return KV4_ERR_INVALID;
   if (pt_stride > kMaxPtStride) return KV4_ERR_UNSUPPORTED;
@@ -387,7 +398,7 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   Kv4Plan pl{};
   const kv4_status ps = kv4_plan(D, G, Hkv, B, num_workers, &pl);
   if (ps != KV4_OK) return ps;
-  const bool has8 = cache->cfg.sink + cache->cfg.recent > 0;
+  const bool has8 = cache->cfg.sink + cache->cfg.recent > 0 && with_int8;
   if (ws_bytes < kv4_ws_bytes(pl, G, D)) return KV4_ERR_INVALID;
 
   DecodeParams p{};
@@ -421,12 +432,50 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.out = out;
   p.out_fp32 = out_is_fp32 ? 1 : 0;
+  p.page_begin = page_begin;
+  p.page_end = page_end;
+  p.partials = partials;
   p.err = cache->err;
   p.wait_cap = cache->wait_cap;
   carve_workspace(p, workspace, (size_t)pl.NVB + 1, (size_t)2 * pl.NVB);
   cudaEvent_t e0, e1;
   timing_pair(0, &e0, &e1);
   return cuda_status(launch_decode(p, D, false, static_cast<cudaStream_t>(stream), e0, e1));
+}
+
+}  // namespace
+
+extern "C" {
+
+kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_t Hq, const int32_t *seq_lens,
+                           const int32_t *page_table, int32_t pt_stride, const uint32_t *retain_mask,
+                           int32_t mask_stride, float softmax_scale, int32_t num_workers, void *workspace,
+                           size_t ws_bytes, void *out, int32_t out_is_fp32, int32_t B) {
+  if (!out && B > 0) return KV4_ERR_INVALID;
+  return decode_call(cache, stream, q, Hq, seq_lens, page_table, pt_stride, nullptr, nullptr, 1, retain_mask,
+                     mask_stride, softmax_scale, num_workers, workspace, ws_bytes, out, out_is_fp32, nullptr, B);
+}
+
+kv4_status kv4_decode_partials(kv4_cache *cache, void *stream, const void *q, int32_t Hq, const int32_t *seq_lens,
+                               const int32_t *page_table, int32_t pt_stride, const int32_t *page_begin,
+                               const int32_t *page_end, int32_t with_int8, const uint32_t *retain_mask,
+                               int32_t mask_stride, float softmax_scale, int32_t num_workers, void *workspace,
+                               size_t ws_bytes, float *partials, int32_t B) {
+  if (!partials && B > 0) return KV4_ERR_INVALID;
+  return decode_call(cache, stream, q, Hq, seq_lens, page_table, pt_stride, page_begin, page_end, with_int8,
+                     retain_mask, mask_stride, softmax_scale, num_workers, workspace, ws_bytes, nullptr, 0, partials,
+                     B);
+}
+
+kv4_status kv4_merge_partials(void *stream, const float *partials, int32_t N, int32_t B, int32_t Hq, int32_t D,
+                              void *out, int32_t out_is_fp32) {
+  if (N < 0 || B < 0 || Hq < 1) return KV4_ERR_INVALID;
+  if (D != 64 && D != 128) return KV4_ERR_UNSUPPORTED;
+  if (B == 0) return KV4_OK;
+  if (!out || (N > 0 && !partials)) return KV4_ERR_INVALID;
+  if (!aligned(out, 16) || (partials && !aligned(partials, 16))) return KV4_ERR_INVALID;
+  return cuda_status(launch_merge_partials(partials, N, (long long)B * Hq, D, out, out_is_fp32 ? 1 : 0,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 kv4_status kv_topk_retain(void *stream, const float *scores, int64_t score_stride, const int32_t *seq_lens,
@@ -449,6 +498,7 @@ kv4_status kv_topk_retain(void *stream, const float *scores, int64_t score_strid
   p.recent = recent;
   p.max_len = max_len;
   p.mask_stride = mask_stride;
+  p.vec_ok = (aligned(scores, 16) && score_stride % 4 == 0) ? 1 : 0;
   p.mask = mask_out;
   p.count = count_out;
   return cuda_status(launch_topk(p, static_cast<cudaStream_t>(stream)));

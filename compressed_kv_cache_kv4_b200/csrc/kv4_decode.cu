@@ -367,6 +367,18 @@ __device__ __forceinline__ bool side_page_attended(int j, int L, int S, int R) {
   return ((lo - a + R) % R) < nv || ((a - lo + R) % R) < 16;
 }
 
+// INT4 pages of sequence b attended by this call: the INT4 region's pages
+// [sink/16, ceil((L - recent)/16)), clipped to the shard [page_begin[b],
+// page_end[b]) when the call decodes one page-range shard of each sequence.
+__device__ __forceinline__ void int4_page_range(const DecodeParams &p, int b, int L, int &pg0, int &pg1) {
+  pg0 = int4_first_page(p.sink);
+  pg1 = pg0 + int4_num_pages(L, p.sink, p.recent);
+  if (p.page_begin) {
+    pg0 = max(pg0, p.page_begin[b]);
+    pg1 = max(pg0, min(pg1, p.page_end[b]));
+  }
+}
+
 // Descriptor of flat item x, or false if the item has nothing to attend
 // (or names a page outside the pool, which is reported). n8 = INT8 items per
 // virtual sequence (0 without side pages).
@@ -384,7 +396,9 @@ __device__ bool classify_item(const DecodeParams &p, const int *plan, int n8, lo
     d.y = 0;
     return true;
   }
-  const int pg = int4_first_page(p.sink) + off - n8;
+  int pg0, pg1;
+  int4_page_range(p, b, eff_len(p.seq_lens[b], cap), pg0, pg1);
+  const int pg = pg0 + off - n8;
   if (p.mask) {
     const int L = eff_len(p.seq_lens[b], cap);
     const int lo_tok = p.sink, hi_tok = L - p.recent;
@@ -764,8 +778,11 @@ __global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
     const int chunk = (NVB + nthr - 1) / nthr;
     const int v0 = min(NVB, tid * chunk), v1 = min(NVB, v0 + chunk);
     int mine = 0;
-    for (int vb = v0; vb < v1; ++vb)
-      mine += n8 + int4_num_pages(eff_len(p.seq_lens[vb % p.B], cap), p.sink, p.recent);
+    for (int vb = v0; vb < v1; ++vb) {
+      int pg0, pg1;
+      int4_page_range(p, vb % p.B, eff_len(p.seq_lens[vb % p.B], cap), pg0, pg1);
+      mine += n8 + pg1 - pg0;
+    }
     int incl = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -778,7 +795,9 @@ __global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
     for (int w = 0; w < warp; ++w) run += wtot[w];
     for (int vb = v0; vb < v1; ++vb) {
       plan[vb] = run;
-      run += n8 + int4_num_pages(eff_len(p.seq_lens[vb % p.B], cap), p.sink, p.recent);
+      int pg0, pg1;
+      int4_page_range(p, vb % p.B, eff_len(p.seq_lens[vb % p.B], cap), pg0, pg1);
+      run += n8 + pg1 - pg0;
     }
     if (tid == nthr - 1) plan[NVB] = run;
     __syncthreads();

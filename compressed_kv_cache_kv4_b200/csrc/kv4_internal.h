@@ -52,6 +52,11 @@ struct DecodeParams {
   float *slots;
   void *out;
   int out_fp32;
+  // page-range shard of every sequence (nullable, KV4 only): INT4 pages
+  // [page_begin[b], page_end[b]) of the INT4 region are attended
+  const int32_t *page_begin;
+  const int32_t *page_end;
+  float *partials;              // non-null: the merge writes (m, l, o) partials [B][Hq][D+4] instead of out
   uint32_t *err;
   long long wait_cap;           // 0 = simulate a copy that never lands
 };
@@ -61,6 +66,7 @@ struct TopkParams {
   long long score_stride;
   const int32_t *seq_lens;
   int B, Hkv, permille, sink, recent, max_len, mask_stride;
+  int vec_ok;                   // scores 16-byte aligned and score_stride % 4 == 0
   uint32_t *mask;
   int32_t *count;
 };
@@ -108,5 +114,8 @@ cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t 
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream);
 // Exact merge of the decode partials of kv4_decode_kernel or bf16_decode_kernel.
 cudaError_t launch_merge(const DecodeParams &p, int D, bool bf16, cudaStream_t stream);
+// Exact merge of N gathered (m, l, o) partials [N][rows][D+4] into out [rows][D].
+cudaError_t launch_merge_partials(const float *partials, int N, long long rows, int D, void *out, int out_fp32,
+                                  cudaStream_t stream);
 
 }  // namespace kv4

@@ -145,6 +145,15 @@ __global__ void __launch_bounds__(128) merge_kernel(DecodeParams p) {
     }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
+  if (p.partials) {
+    // the merged partial of this call, for a merge with other shards' partials:
+    // m (log2 units), l, two pad words, o (normalised)
+    float *pr = p.partials + ((long long)b * p.Hq + hq) * (D + 4);
+    if (lane == 0) *reinterpret_cast<float4 *>(pr) = make_float4(den > 0.f ? M : -INFINITY, den, 0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) pr[4 + lane * DPL + e] = acc[e] * inv;
+    return;
+  }
   const long long obase = ((long long)b * p.Hq + hq) * D + lane * DPL;
   if (p.out_fp32) {
     float *o = reinterpret_cast<float *>(p.out) + obase;
@@ -174,6 +183,79 @@ static cudaError_t launch_merge_d(const DecodeParams &p, cudaStream_t stream) {
     case 2: return launch_pdl(merge_kernel<D, 2, kKv4>, dim3(blocks), dim3(128), 0, stream, p);
     default: return launch_pdl(merge_kernel<D, 4, kKv4>, dim3(blocks), dim3(128), 0, stream, p);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of N gathered partials [N][rows][D+4] (m, l, pad, pad, o) into the
+// final output: the same exact merge, one warp per row, shards in order.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) merge_partials_kernel(const float *partials, int N, long long rows, void *out,
+                                                             int out_fp32) {
+  constexpr int DPL = D / 32;
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (row >= rows) return;
+  float M = -INFINITY, den = 0.f, acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  for (int c0 = 0; c0 < N; c0 += kBatch) {
+    float mk[kBatch], lk[kBatch], ok[kBatch][DPL];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      mk[k] = -INFINITY;
+      lk[k] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) ok[k][e] = 0.f;
+      if (c0 + k < N) {
+        const float *pr = partials + ((long long)(c0 + k) * rows + row) * (D + 4);
+        mk[k] = pr[0];
+        lk[k] = pr[1];
+        Vec<DPL>::load(pr + 4 + lane * DPL, ok[k]);
+      }
+    }
+    float mc = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k)
+      if (lk[k] > 0.f) mc = fmaxf(mc, mk[k]);
+    if (mc > M) {
+      const float f = ex2(M - mc);
+      den *= f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] *= f;
+      M = mc;
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      if (!(lk[k] > 0.f)) continue;
+      const float wk = lk[k] * ex2(mk[k] - M);
+      den += wk;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wk, ok[k][e], acc[e]);
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const long long obase = row * D + lane * DPL;
+  if (out_fp32) {
+    float *o = reinterpret_cast<float *>(out) + obase;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) o[e] = acc[e] * inv;
+  } else {
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(out) + obase;
+#pragma unroll
+    for (int e = 0; e < DPL; e += 2) *reinterpret_cast<uint32_t *>(o + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+  }
+}
+
+cudaError_t launch_merge_partials(const float *partials, int N, long long rows, int D, void *out, int out_fp32,
+                                  cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>((rows + 3) / 4);
+  if (D == 128)
+    return launch_pdl(merge_partials_kernel<128>, dim3(blocks), dim3(128), 0, stream, partials, N, rows, out, out_fp32);
+  return launch_pdl(merge_partials_kernel<64>, dim3(blocks), dim3(128), 0, stream, partials, N, rows, out, out_fp32);
 }
 
 cudaError_t launch_merge(const DecodeParams &p, int D, bool bf16, cudaStream_t stream) {

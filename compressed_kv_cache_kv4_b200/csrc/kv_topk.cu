@@ -7,20 +7,24 @@
 // kept. Shadow Mask Distillation, sec. 1: the result is a binary mask.
 //
 // One CTA per row. Scores become order-preserving 32-bit keys (larger score ->
-// larger key, -0 folded into +0). A 4-pass 8-bit radix select finds the key T
-// of the k-th best non-forced position in O(L) work; positions with key > T
-// are kept, and among keys == T the lowest indices fill the remainder (a scan
-// over 32-position tiles gives each tie its rank in index order). The forced
-// positions are two contiguous ranges, so the passes run over the candidate
-// range between them only, four keys per thread step. The row is held in
-// shared memory when it fits, otherwise re-read from global memory on each
-// pass.
+// larger key, -0 folded into +0). A 3-pass radix select with 11-, 11- and
+// 10-bit digits finds the key T of the k-th best non-forced position in O(L)
+// work; positions with key > T are kept, and among keys == T the lowest
+// indices fill the remainder (a scan over 32-position tiles gives each tie its
+// rank in index order). The first digit covers the sign, the exponent and the
+// top two mantissa bits, so scores that share an exponent still spread over
+// four bins and scores of one magnitude class do not pile onto a handful of
+// shared-memory counters. The forced positions are two contiguous ranges, so
+// the passes run over the candidate range between them only, four keys per
+// thread step. The row is held in shared memory when it fits, otherwise re-read
+// from global memory on each pass.
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
 
 namespace kv4 {
 
 constexpr int kTopkThreads = 512;
+constexpr int kTopkBins = 2048;            // 4 bins per thread in the scan
 constexpr int kTopkSmemKeys = 49152;   // rows up to this length are staged in shared memory
 
 __device__ __forceinline__ uint32_t score_key(float f) {
@@ -57,7 +61,8 @@ __device__ __forceinline__ void for_candidates(const uint32_t *keys, const float
 template <bool kSmem>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
   extern __shared__ __align__(16) uint32_t dyn[];
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[kTopkBins];
+  __shared__ int wsum[kTopkThreads / 32];
   __shared__ int sh_digit, sh_rem;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NWARP = kTopkThreads / 32;
@@ -88,7 +93,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
   const int mode = ksel == 0 ? 0 : (ksel == c1 - c0 ? 1 : 2);
   if (kSmem && mode == 2) {
     const int base = c0 & ~3;
-    for (int i = base + tid; i < c1; i += kTopkThreads) keys[i] = score_key(srow[i]);
+    if (p.vec_ok) {
+      // 16-byte loads: the row starts 16-byte aligned and its stride is a
+      // multiple of four, so the last vector ends inside the row's storage
+      for (int i = base + 4 * tid; i < c1; i += 4 * kTopkThreads) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(srow + i));
+        *reinterpret_cast<uint4 *>(keys + i) =
+            make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+      }
+    } else {
+      for (int i = base + tid; i < c1; i += kTopkThreads) keys[i] = score_key(srow[i]);
+    }
   }
   __syncthreads();
 
@@ -97,39 +112,45 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
   if (mode == 2) {
     uint32_t prefix = 0, pmask = 0;
     int rem = static_cast<int>(ksel);
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+      for (int i = tid; i < kTopkBins; i += kTopkThreads) hist[i] = 0;
       __syncthreads();
       for_candidates<kSmem>(keys, srow, c0, c1, tid, [&](int, uint32_t k) {
-        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
       });
       __syncthreads();
-      if (warp == 0) {
-        // lane l owns bins 255-8l .. 248-8l (descending)
-        int tot = 0;
+      // thread i owns bins kTopkBins-1-4i .. kTopkBins-4-4i (highest first):
+      // block-wide exclusive scan of the per-thread counts from the top
+      int cnt[4], tot = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) tot += hist[255 - 8 * lane - i];
-        int incl = tot;
+      for (int j = 0; j < 4; ++j) {
+        cnt[j] = hist[kTopkBins - 1 - 4 * tid - j];
+        tot += cnt[j];
+      }
+      int incl = tot;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      int c = incl - tot;
+      for (int w = 0; w < warp; ++w) c += wsum[w];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (c < rem && rem <= c + cnt[j]) {
+          sh_digit = kTopkBins - 1 - 4 * tid - j;
+          sh_rem = rem - c;
         }
-        int c = incl - tot;   // keys in bins above this lane's range
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int bin = 255 - 8 * lane - i;
-          const int hcount = hist[bin];
-          if (c < rem && rem <= c + hcount) {
-            sh_digit = bin;
-            sh_rem = rem - c;
-          }
-          c += hcount;
-        }
+        c += cnt[j];
       }
       __syncthreads();
       prefix |= static_cast<uint32_t>(sh_digit) << shift;
-      pmask |= 255u << shift;
+      pmask |= dmask << shift;
       rem = sh_rem;
       __syncthreads();
     }

@@ -169,6 +169,47 @@ kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_
                            int32_t out_is_fp32, int32_t B);
 
 /*
+ * kv4_decode_partials -- the decode step of kv4_decode_attn over one shard of
+ * each sequence's context, returning the exact softmax partial instead of the
+ * output, for context-parallel decoding of long sequences across GPUs (the
+ * TTKV promo of arXiv 2604.19769, opening section, puts contexts of about a
+ * million tokens beyond one GPU). KV4-RL review, sec. 3: partials of disjoint
+ * position sets combine exactly (kv4_merge_partials), so each GPU attends the
+ * pages it holds and only (m, l, o) crosses the interconnect.
+ *  page_begin, page_end: device int32 [B]; the shard attends the INT4 pages
+ *    [page_begin[b], page_end[b]) of sequence b (logical page indices, the
+ *    INT4 region's pages outside the range are skipped; page-table entries of
+ *    skipped pages are never read). Both NULL = every INT4 page.
+ *  with_int8: nonzero = the shard also attends the INT8 sink/recent positions
+ *    (exactly one shard per sequence must, normally the one holding the side
+ *    cache); zero = INT4 positions only.
+ *  partials: device fp32 [B][Hq][D+4], 16-byte aligned: per (sequence, query
+ *    head) m (the running maximum of the scores in log2 units, i.e. of
+ *    softmax_scale * log2(e) * q.k; -inf when nothing was attended), l (the
+ *    sum of 2^(s - m) over the attended positions), two unused words, then o
+ *    (the attended values' softmax average, D floats; 0 when l = 0).
+ *  Other arguments as kv4_decode_attn; the same workspace size applies.
+ */
+kv4_status kv4_decode_partials(kv4_cache *cache, void *stream, const void *q, int32_t Hq, const int32_t *seq_lens,
+                               const int32_t *page_table, int32_t pt_stride, const int32_t *page_begin,
+                               const int32_t *page_end, int32_t with_int8, const uint32_t *retain_mask,
+                               int32_t mask_stride, float softmax_scale, int32_t num_workers, void *workspace,
+                               size_t ws_bytes, float *partials, int32_t B);
+
+/*
+ * kv4_merge_partials -- exact softmax merge of N partials per (sequence, query
+ * head), e.g. those of N context shards gathered from N GPUs (KV4-RL review,
+ * sec. 3: the exact merge of (max, sum, output) triples): with
+ * M = max_s m_s and W_s = l_s 2^(m_s - M), out = sum_s W_s o_s / sum_s W_s;
+ * 0 when every l_s = 0.
+ *  partials: device fp32 [N][B][Hq][D+4] in the layout of kv4_decode_partials,
+ *    16-byte aligned. out: device [B][Hq][D], bf16 (RNE of the fp32 result) or
+ *    fp32 (out_is_fp32), 16-byte aligned. D = 64 or 128.
+ */
+kv4_status kv4_merge_partials(void *stream, const float *partials, int32_t N, int32_t B, int32_t Hq, int32_t D,
+                              void *out, int32_t out_is_fp32);
+
+/*
  * kv_topk_retain -- per (sequence, KV head) retained-position mask ([KVP] core
  * mechanism; [SMD] sec. 1).
  *  scores: device fp32 [B][Hkv][score_stride], one score per position.

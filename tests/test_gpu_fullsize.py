@@ -9,6 +9,9 @@ outputs the oracle computes sequence by sequence.
   against the single-pass oracle.
 - evict: B = 64, L = 16384; top-k masks bit-exact at every budget,
   masked decode at 10% and 50% on sampled sequences, 100% = unmasked bitwise.
+- long, context parallel: the same four 128K sequences decoded as four
+  page-range shards (kv4_decode_partials, the INT8 region with the last) and
+  merged (kv4_merge_partials), against the oracle.
 - prefill bytes: the benchmark's prefill of the qwen8b and async prompts in one
   kv4_append; page and side-cache bytes of sampled sequences (the first and the
   last ones of the batch among them, which only later grid-stride passes of the
@@ -129,6 +132,39 @@ def test_long_context_full_size():
     del k, v
     _cleanup()
     _check(wl, cache, ptd, wl.lens, q, seqs, rows_k, rows_v, "long")
+    cache.close()
+    del cache
+    _cleanup()
+
+
+def test_long_context_parallel_full_size():
+    from compressed_kv_cache_kv4_b200 import cp
+    wl = synth.workload("long")
+    cache, ptd, k, v, off = _prefill(wl, wl.lens, wl.lens)
+    q = synth.gen_q(wl, device="cuda")
+    seqs = list(range(wl.B))
+    rows_k = [k[int(off[b]): int(off[b + 1])].cpu() for b in seqs]
+    rows_v = [v[int(off[b]): int(off[b + 1])].cpu() for b in seqs]
+    del k, v
+    _cleanup()
+    lens = torch.as_tensor(wl.lens, device="cuda")
+    n = 4
+    pb, pe = cp.shard_pages(wl.lens, n, wl.sink, wl.recent)
+    parts = torch.empty((n, wl.B, wl.Hq, wl.D + 4), dtype=torch.float32, device="cuda")
+    ws = cache.workspace(wl.B, wl.Hq)
+    for r in range(n):
+        K.kv4_decode_partials(cache.handle, q, lens, ptd, wl.softmax_scale, ws, parts[r],
+                              torch.as_tensor(pb[r], device="cuda"), torch.as_tensor(pe[r], device="cuda"),
+                              with_int8=(r == n - 1))
+    out32 = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32, device="cuda")
+    out16 = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
+    K.kv4_merge_partials(parts, out32)
+    K.kv4_merge_partials(parts, out16)
+    st, bits = cache.get_error()
+    assert st == K.KV4_OK, (st, bits)
+    ref = _oracle(wl, rows_k, rows_v, q.cpu(), [int(x) for x in wl.lens])
+    assert_close(out32.cpu().numpy(), ref, what="long, 4 shards")
+    assert_bf16_output(out16, out32, ref)
     cache.close()
     del cache
     _cleanup()
