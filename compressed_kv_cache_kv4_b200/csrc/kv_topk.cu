@@ -35,11 +35,13 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 
 // Keys of candidate positions [c0, c1) in steps of four per thread: f(i, key)
 // for each. With the row in shared memory four keys come from one 16-byte load
-// (c0 rounded down to a multiple of four; lanes skip the indices outside).
+// (c0 rounded down to a multiple of four); only the first and the last step
+// of the range test each index, the steps between hold four candidates.
 template <bool kSmem, typename F>
 __device__ __forceinline__ void for_candidates(const uint32_t *keys, const float *srow, int c0, int c1, int tid,
                                                F &&f) {
   const int base = c0 & ~3;
+  const int lo = (c0 + 3) & ~3, hi = c1 & ~3;   // [lo, hi): whole steps inside [c0, c1)
   for (int i = base + 4 * tid; i < c1; i += 4 * kTopkThreads) {
     uint32_t k[4];
     if constexpr (kSmem) {
@@ -52,9 +54,14 @@ __device__ __forceinline__ void for_candidates(const uint32_t *keys, const float
 #pragma unroll
       for (int e = 0; e < 4; ++e) k[e] = i + e < c1 ? score_key(srow[i + e]) : 0u;
     }
+    if (i >= lo && i < hi) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if (i + e >= c0 && i + e < c1) f(i + e, k[e]);
+      for (int e = 0; e < 4; ++e) f(i + e, k[e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i + e >= c0 && i + e < c1) f(i + e, k[e]);
+    }
   }
 }
 
@@ -63,7 +70,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
   extern __shared__ __align__(16) uint32_t dyn[];
   __shared__ uint32_t hist[kTopkBins];
   __shared__ int wsum[kTopkThreads / 32];
-  __shared__ int sh_digit, sh_rem;
+  __shared__ int sh_digit, sh_rem, sh_cnt;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NWARP = kTopkThreads / 32;
   pdl_wait();
@@ -109,6 +116,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
 
   uint32_t T = 0;
   int need_eq = 0;
+  bool ties = false;
   if (mode == 2) {
     uint32_t prefix = 0, pmask = 0;
     int rem = static_cast<int>(ksel);
@@ -118,9 +126,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
       const uint32_t dmask = pass == 2 ? 1023u : 2047u;
       for (int i = tid; i < kTopkBins; i += kTopkThreads) hist[i] = 0;
       __syncthreads();
-      for_candidates<kSmem>(keys, srow, c0, c1, tid, [&](int, uint32_t k) {
-        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
-      });
+      if (pass == 0) {
+        for_candidates<kSmem>(keys, srow, c0, c1, tid,
+                              [&](int, uint32_t k) { atomicAdd(&hist[k >> shift], 1u); });
+      } else {
+        for_candidates<kSmem>(keys, srow, c0, c1, tid, [&](int, uint32_t k) {
+          if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
+        });
+      }
       __syncthreads();
       // thread i owns bins kTopkBins-1-4i .. kTopkBins-4-4i (highest first):
       // block-wide exclusive scan of the per-thread counts from the top
@@ -145,6 +158,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
         if (c < rem && rem <= c + cnt[j]) {
           sh_digit = kTopkBins - 1 - 4 * tid - j;
           sh_rem = rem - c;
+          sh_cnt = cnt[j];
         }
         c += cnt[j];
       }
@@ -156,49 +170,60 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
     }
     T = prefix;
     need_eq = rem;
-    // ranks of the ties in index order: count per 32-position tile, then scan
-    for (int w = warp; w < nt; w += NWARP) {
-      const int pos = 32 * w + lane;
-      const bool eq = pos >= c0 && pos < c1 && (kSmem ? keys[pos] : score_key(srow[pos])) == T;
-      const uint32_t bal = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) tile_rank[w] = __popc(bal);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      int carry = 0;
-      for (int base = 0; base < nt; base += 32) {
-        const int w = base + lane;
-        const int v = w < nt ? tile_rank[w] : 0;
-        int incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        if (w < nt) tile_rank[w] = carry + incl - v;
-        carry += __shfl_sync(0xffffffffu, incl, 31);
+    // sh_cnt = keys equal to T; ranks among them are needed only when some of
+    // them stay out: count per 32-position tile, then scan
+    ties = need_eq < sh_cnt;
+    if (ties) {
+      for (int w = warp; w < nt; w += NWARP) {
+        const int pos = 32 * w + lane;
+        const bool eq = pos >= c0 && pos < c1 && (kSmem ? keys[pos] : score_key(srow[pos])) == T;
+        const uint32_t bal = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) tile_rank[w] = __popc(bal);
       }
+      __syncthreads();
+      if (warp == 0) {
+        int carry = 0;
+        for (int base = 0; base < nt; base += 32) {
+          const int w = base + lane;
+          const int v = w < nt ? tile_rank[w] : 0;
+          int incl = v;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          if (w < nt) tile_rank[w] = carry + incl - v;
+          carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+      }
+      __syncthreads();
     }
-    __syncthreads();
   }
 
+  // mask words: a warp builds 32 consecutive words (lane i keeps word i) and
+  // stores them together
   uint32_t *mrow = p.mask + (long long)row * p.mask_stride;
-  for (int w = warp; w < nt; w += NWARP) {
-    const int pos = 32 * w + lane;
-    bool sel = false, eq = false;
-    if (pos < L) {
-      if (forced(pos) || mode == 1) {
-        sel = true;
-      } else if (mode == 2) {
-        const uint32_t k = kSmem ? keys[pos] : score_key(srow[pos]);
-        sel = k > T;
-        eq = k == T;
+  for (int w0 = 32 * warp; w0 < nt; w0 += 32 * NWARP) {
+    uint32_t mine = 0;
+    const int n = min(32, nt - w0);
+    for (int i = 0; i < n; ++i) {
+      const int w = w0 + i;
+      const int pos = 32 * w + lane;
+      bool sel = pos < L && (forced(pos) || mode == 1);
+      if (mode == 2) {
+        const bool cand = pos >= c0 && pos < c1;
+        const uint32_t k = cand ? (kSmem ? keys[pos] : score_key(srow[pos])) : 0u;
+        if (cand) sel = k > T || (!ties && k == T);
+        if (ties) {
+          const bool eq = cand && k == T;
+          const uint32_t eqbal = __ballot_sync(0xffffffffu, eq);
+          if (eq) sel = tile_rank[w] + __popc(eqbal & ((1u << lane) - 1u)) < need_eq;
+        }
       }
+      const uint32_t word = __ballot_sync(0xffffffffu, sel);
+      if (lane == i) mine = word;
     }
-    const uint32_t eqbal = __ballot_sync(0xffffffffu, eq);
-    if (eq) sel = tile_rank[w] + __popc(eqbal & ((1u << lane) - 1u)) < need_eq;
-    const uint32_t word = __ballot_sync(0xffffffffu, sel);
-    if (lane == 0) mrow[w] = word;
+    if (lane < n) mrow[w0 + lane] = mine;
   }
   if (tid == 0 && p.count) p.count[row] = nF + static_cast<int>(ksel);
 }
