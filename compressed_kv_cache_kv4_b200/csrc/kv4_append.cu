@@ -9,9 +9,13 @@
 //
 // Two kernels. append_pages_kernel takes every page the append fills
 // completely (a prefill, or a multi-token append that crosses page
-// boundaries): one warp per (page, KV head), lane l quantises row l % 16 of K
-// (l < 16) or V (l >= 16) group by group into a shared-memory image of the
-// 18*D-byte head block, which the warp then writes out with 16-byte stores.
+// boundaries): one warp per (page, KV head); for K, then for V, lane l
+// quantises half a group (16 elements) of row l % 16 -- the two lanes of a
+// group combine their maxima with one shuffle -- into a shared-memory image
+// of the 18*D-byte head block, which the warp then writes out with 16-byte
+// stores. Codes are packed arithmetically: with u = c + 8 in [1, 15], four
+// codes make an exact fp32 integer u0 + 16 u1 + 256 u2 + 4096 u3 whose bits
+// an added 2^23 exposes, and XOR with 0x8 per nibble gives c mod 16.
 // append_kernel takes the rest: one warp per (new position, KV head, K or V),
 // lane l holding D/32 consecutive elements, for the INT4 slots of partially
 // filled pages and for every INT8 side-cache row.
@@ -38,11 +42,40 @@ __device__ __forceinline__ uint32_t nib(int c) { return static_cast<uint32_t>(c)
 __device__ __forceinline__ float round_code(float x, float s, float r) {
   float c = rintf(x * r);
   const float d = fmaf(c, s, -x);   // c*s - x, exact
-  if (2.f * fabsf(d) == s) {        // half-way: x/s = c - sign(d)/2
-    const float other = c - copysignf(1.f, d);
-    c = (fmodf(c, 2.f) == 0.f) ? c : other;
+  if (2.f * fabsf(d) == s) {        // half-way: x/s = c - sign(d)/2; keep the even one
+    if (static_cast<int>(c) & 1) c -= copysignf(1.f, d);
   }
   return c;
+}
+
+// The same for two values with one scale (packed f32x2 arithmetic); r only
+// has to be within 2^-20 of 1/s (an approximate reciprocal will do): the
+// half-way test uses the exact residual, not r.
+__device__ __forceinline__ float2 round_code2(float2 x, float s, float r) {
+  const float2 q = __fmul2_rn(x, make_float2(r, r));
+  float2 c = make_float2(rintf(q.x), rintf(q.y));
+  const float2 d = __ffma2_rn(c, make_float2(s, s), make_float2(-x.x, -x.y));   // c*s - x, exact
+  if (2.f * fabsf(d.x) == s || 2.f * fabsf(d.y) == s) {   // rare: an exact half-way point
+    if (2.f * fabsf(d.x) == s && (static_cast<int>(c.x) & 1)) c.x -= copysignf(1.f, d.x);
+    if (2.f * fabsf(d.y) == s && (static_cast<int>(c.y) & 1)) c.y -= copysignf(1.f, d.y);
+  }
+  return c;
+}
+
+// 1/s to within an ulp or two (fp32 approximate reciprocal).
+__device__ __forceinline__ float rcp_approx(float s) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+  return r;
+}
+
+// Codes c0..c3 in [-7, 7] -> 16 bits of four 4-bit two's-complement nibbles
+// (c0 lowest). With u = c + 8 in [1, 15], u0 + 16 u1 + 256 u2 + 4096 u3 is an
+// integer below 2^16, exact in fp32; adding 2^23 puts it in the low mantissa
+// bits, and nibble u ^ 8 = c mod 16 (the caller XORs 0x8888).
+__device__ __forceinline__ uint32_t nib4_biased(float c0, float c1, float c2, float c3) {
+  const float v = fmaf(c3, 4096.f, fmaf(c2, 256.f, fmaf(c1, 16.f, c0 + 34952.f)));   // 34952 = 8 * 0x1111
+  return __float_as_uint(v + 8388608.f);
 }
 
 // Quantise this lane's EPL values with a scale shared by `span` lanes
@@ -173,7 +206,9 @@ __global__ void __launch_bounds__(256, 3) append_pages_kernel(AppendParams p) {
 
   const long long units = (long long)fplan[p.B] * p.Hkv;
   uint8_t *im = img[warp];
-  const int r = lane & 15, kv = lane >> 4;
+  // lane (r, hh): row r of the page, elements [16 hh, 16 hh + 16) of each group;
+  // K first, then V, so that the whole warp runs one code path at a time
+  const int r = lane & 15, hh = lane >> 4;
   for (long long u = (long long)blockIdx.x * WARPS + warp; u < units; u += (long long)gridDim.x * WARPS) {
     const int unit = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
     int lo = 0, hi = p.B - 1;   // sequence: largest b with fplan[b] <= unit
@@ -196,46 +231,75 @@ __global__ void __launch_bounds__(256, 3) append_pages_kernel(AppendParams p) {
     }
     // rows j .. j+15 are the page's slots 0..15 (all new, all of sequence b)
     const long long j = p.offsets[b] + (pg * kPageTokens - L_old);
-    const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + ((j + r) * p.Hkv + h) * D;
 #pragma unroll 1
-    for (int i = 0; i < NG; ++i) {
-      float x[kGroup];
+    for (int kv = 0; kv < 2; ++kv) {
+      const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + ((j + r) * p.Hkv + h) * D + 16 * hh;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(src + kGroup * i + 8 * q);
-        x[8 * q + 0] = bf16lo_to_f32(w.x);
-        x[8 * q + 1] = bf16hi_to_f32(w.x);
-        x[8 * q + 2] = bf16lo_to_f32(w.y);
-        x[8 * q + 3] = bf16hi_to_f32(w.y);
-        x[8 * q + 4] = bf16lo_to_f32(w.z);
-        x[8 * q + 5] = bf16hi_to_f32(w.z);
-        x[8 * q + 6] = bf16lo_to_f32(w.w);
-        x[8 * q + 7] = bf16hi_to_f32(w.w);
-      }
-      int c[kGroup];
-      const uint16_t sbits = quant_group32(x, c, p.err);
-      if (kv == 0) {
-        // K: element 32i + 8t + k of row r is nibble k of the word at
-        // r*D/2 + t*D/8 + 4i
+      for (int i = 0; i < NG; ++i) {   // unrolled: the groups' loads are in flight together
+        float x[16];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          uint32_t w = 0;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) w |= nib(c[8 * t + k]) << (4 * k);
-          *reinterpret_cast<uint32_t *>(im + r * (D / 2) + t * (D / 8) + 4 * i) = w;
+        for (int q = 0; q < 2; ++q) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(src + kGroup * i + 8 * q);
+          x[8 * q + 0] = bf16lo_to_f32(w.x);
+          x[8 * q + 1] = bf16hi_to_f32(w.x);
+          x[8 * q + 2] = bf16lo_to_f32(w.y);
+          x[8 * q + 3] = bf16hi_to_f32(w.y);
+          x[8 * q + 4] = bf16lo_to_f32(w.z);
+          x[8 * q + 5] = bf16hi_to_f32(w.z);
+          x[8 * q + 6] = bf16lo_to_f32(w.w);
+          x[8 * q + 7] = bf16hi_to_f32(w.w);
         }
-        *reinterpret_cast<uint16_t *>(im + 16 * D + 2 * (r * NG + i)) = sbits;
-      } else {
-        // V: the byte of (slot r, element d) pairs d and d+8 (low, high nibble)
+        // scale of the group: max |x| over both lanes of the pair (lane ^ 16)
+        float a = 0.f;
 #pragma unroll
-        for (int e = 0; e < kGroup; ++e) {
-          if ((e % 16) >= 8) continue;
-          const int d = kGroup * i + e;
-          const int m = d / 16, g8 = d % 8, tt = (r % 8) / 2;
-          const int word = (m / 4) * 128 + (4 * g8 + tt) * 4 + (m % 4);
-          im[8 * D + 4 * word + 2 * (r % 2) + r / 8] = static_cast<uint8_t>(nib(c[e]) | nib(c[e + 8]) << 4);
+        for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(x[e]));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
+        uint16_t sbits = 0;
+        float c[16];
+        if (a == 0.f) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) c[e] = 0.f;
+        } else {
+          sbits = __half_as_ushort(__float2half_ru(__fdiv_rn(a, 7.f)));
+          const bool sat = sbits == 0x7C00u;
+          if (sat) {                       // a/7 > 65504: saturate and flag
+            sbits = 0x7BFFu;
+            if (hh == 0) set_error(p.err, kErrRange);
+          }
+          const float sc = half_bits_to_f32(sbits);
+          const float rc = rcp_approx(sc);
+          // sc >= max|x| / 7 makes |x / sc| <= 7: a clamp only when sc saturated
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float2 v = round_code2(make_float2(x[e], x[e + 1]), sc, rc);
+            if (sat) v = make_float2(fminf(fmaxf(v.x, -7.f), 7.f), fminf(fmaxf(v.y, -7.f), 7.f));
+            c[e] = v.x;
+            c[e + 1] = v.y;
+          }
         }
-        *reinterpret_cast<uint16_t *>(im + 17 * D + 2 * (r * NG + i)) = sbits;
+        if (kv == 0) {
+          // K: element 32i + 8t + k of row r is nibble k of the word at
+          // r*D/2 + t*D/8 + 4i; this lane's elements are chunks t = 2hh, 2hh+1
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint32_t w = __byte_perm(nib4_biased(c[8 * q], c[8 * q + 1], c[8 * q + 2], c[8 * q + 3]),
+                                           nib4_biased(c[8 * q + 4], c[8 * q + 5], c[8 * q + 6], c[8 * q + 7]),
+                                           0x5410) ^ 0x88888888u;
+            *reinterpret_cast<uint32_t *>(im + r * (D / 2) + (2 * hh + q) * (D / 8) + 4 * i) = w;
+          }
+          if (hh == 0) *reinterpret_cast<uint16_t *>(im + 16 * D + 2 * (r * NG + i)) = sbits;
+        } else {
+          // V: the byte of (slot r, element d) pairs d and d+8 (low, high nibble);
+          // this lane's d = 32i + 16hh + e, e < 8 (m = 2i + hh, d mod 8 = e)
+          const int m = 2 * i + hh, tt = (r % 8) / 2;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int word = (m / 4) * 128 + (4 * e + tt) * 4 + (m % 4);
+            const uint32_t byte = (__float_as_uint(fmaf(c[e + 8], 16.f, c[e] + 136.f) + 8388608.f) & 0xFFu) ^ 0x88u;
+            im[8 * D + 4 * word + 2 * (r % 2) + r / 8] = static_cast<uint8_t>(byte);
+          }
+          if (hh == 0) *reinterpret_cast<uint16_t *>(im + 17 * D + 2 * (r * NG + i)) = sbits;
+        }
       }
     }
     __syncwarp();
