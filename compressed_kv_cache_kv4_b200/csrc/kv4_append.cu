@@ -25,10 +25,11 @@
 // or has a periodic binary expansion whose bits past the fp16 precision are
 // never all zero, so the fp32 rounding cannot land on an fp16 value.
 // Code: x/s differs from every half-integer it is not equal to by at least
-// 2^-10, while x * RN(1/s) differs from x/s by less than 2^-20, so rounding
-// x * RN(1/s) to the nearest integer is exact except at true half-way points;
-// those are detected exactly through the residual c*s - x (exact in fp32) and
-// resolved to the even code.
+// 2^-10, while x * r, with r = 1/s rounded (or approximated to an ulp or two),
+// differs from x/s by less than 2^-19 for |x/s| <= 7, so rounding x * r to the
+// nearest integer is exact except at true half-way points; those are detected
+// exactly through the residual c*s - x (exact in fp32) and resolved to the
+// even code.
 #include <algorithm>
 
 #include "kv4_common.cuh"
