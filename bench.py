@@ -490,13 +490,18 @@ def run_kv4(args, ws, rank):
         st.step(s)
     torch.cuda.synchronize()
     st.check("before timing")
-    with ClockSampler(dev) as clk:
+    # clocks sampled over every measured part: the timed steps, the worker's
+    # per-launch pass and the end-to-end steps
+    clk = ClockSampler(dev)
+    with clk:
         elapsed_ms = st.timed(args.warmup, args.steps, ws)
-    st.check("in timed region")
+        st.check("in timed region")
+        worker_us = st.worker_pass(max(64, CYCLE))
+        e2e = st.e2e(max(64, min(args.steps, 512)), ws)
+    st.check("after e2e")
     positions = st.positions(range(args.warmup, args.warmup + args.steps))
     value, elapsed_max = aggregate(positions, elapsed_ms, ws)
     peak, peak_src = peaks()
-    worker_us = st.worker_pass(max(64, CYCLE))
     rf = roofline(st, worker_us, peak, peak_src)
     rf["traffic"] = ncu_traffic(rf["algorithmic_bytes_per_launch"])
     sbytes = step_bytes(st.mean_lens(), wl)
@@ -508,8 +513,7 @@ def run_kv4(args, ws, rank):
         "gpu_launches": 3 * args.steps,   # per step: append, decode workers, merge
     }
     # e2e through host buffers: per step H2D of (k_new, v_new, q) from pinned memory, D2H of the output
-    res["e2e"] = st.e2e(max(64, min(args.steps, 512)), ws)
-    st.check("after e2e")
+    res["e2e"] = e2e
     if rank == 0 and not args.no_secondary and args.workload == "qwen8b":
         res["secondary"] = secondary(st)
     if rank == 0 and not args.no_cpu:

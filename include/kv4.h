@@ -59,7 +59,8 @@ typedef enum {
   KV4_ERR_UNSUPPORTED = 2,  /* valid but not built (head_dim, GQA group, sink/recent) */
   KV4_ERR_CAPACITY = 3,     /* a length exceeds the page-table / side-cache capacity */
   KV4_ERR_BOUNDS = 4,       /* a page id outside [0, num_pages) */
-  KV4_ERR_RANGE = 5,        /* a value too large for an fp16 scale (|x| > 458,528) */
+  KV4_ERR_RANGE = 5,        /* a K/V value too large for an fp16 scale (|x| > 458,528),
+                               or a query component beyond the fp16 range */
   KV4_ERR_TIMEOUT = 6,      /* a bounded device wait ran out */
   KV4_ERR_CUDA = 7          /* a CUDA runtime call failed */
 } kv4_status;
@@ -154,13 +155,21 @@ kv4_status kv4_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t num_q_
  *    p/32 set = position p retained ([SMD] Figure 1). Positions with a clear bit
  *    are excluded; pages with no retained position are not read.
  *  softmax_scale: tau, scores are tau * q.k.
- *  num_workers: 0 = default; otherwise the number of warp workers among which
- *    the INT4 pages are split (results agree within rounding for any value).
+ *  num_workers: 0 = default (as many CTAs as are resident at once); otherwise
+ *    the number of warps, rounded up to whole CTAs of HB warps (HB = the
+ *    largest divisor of Hkv not above 8), among which every (sequence, head)'s
+ *    pages are split (results agree within rounding for any value).
  *  workspace: device, >= kv4_workspace_bytes(), 256-byte aligned.
  *  out: device [B][Hq][D], bf16 (out_is_fp32 = 0) or fp32 (1).
  * The INT4 region [sink, L - recent) and the INT8 region (the rest) are
  * attended separately into (max, sum, output) partials and merged exactly
  * ([KV4RL] sec. 3). An empty retained set gives an output of 0.
+ * Errors found on the device set bits in the cache's error word
+ * (kv4_get_error). After KV4_ERR_TIMEOUT the output is undefined: a CTA whose
+ * wait ran out leaves its partials empty, so out holds the attention over the
+ * other CTAs' pages only. A query component beyond the fp16 range
+ * (|q| > 65504) sets KV4_ERR_RANGE; that query head's output is then
+ * undefined.
  */
 kv4_status kv4_decode_attn(kv4_cache *cache, void *stream, const void *q, int32_t Hq,
                            const int32_t *seq_lens, const int32_t *page_table, int32_t pt_stride,
@@ -321,7 +330,7 @@ kv4_status bf16_paged_decode_attn(void *stream, const void *q, int32_t Hq, int32
  *  Limit: returns KV4_ERR_CAPACITY, with nothing enqueued, when
  *    kv4_workspace_bytes() for the same (B, Hq, num_workers) exceeds
  *    KV4_NOALLOC_SCRATCH_BYTES (with Hkv = 8, head_dim = 128, Hq = 32 and the
- *    default workers on a 148-SM B200: up to about 340 sequences). A smaller
+ *    default 296 CTAs on a 148-SM B200: up to about 350 sequences). A smaller
  *    num_workers lowers the need.
  *  Set-up: the first call on each device looks up the array's address (this
  *    makes the CUDA runtime load the library's module on that device); make
