@@ -55,6 +55,10 @@ def parse():
                     help="time only kv4_evict_pages on the eviction workload and print its figures")
     ap.add_argument("--learner-only", action="store_true",
                     help="time only smd_masked_attn on the learner workload and print its figures")
+    ap.add_argument("--topk-only", action="store_true",
+                    help="print only kv_topk_retain on the evict workload at a 10%% budget (the ncu capture's command)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="print only the prefill append of the qwen8b prompt (the ncu capture's command)")
     ap.add_argument("--sink", type=int, default=None, help="override the INT8 sink size (0 = pure INT4)")
     ap.add_argument("--recent", type=int, default=None, help="override the INT8 recent window")
     return ap.parse_args()
@@ -645,6 +649,53 @@ def secondary(st):
     return out
 
 
+def topk_only(permille=100, reps=20):
+    """kv_topk_retain alone on the evict workload's scores (B = 64 x 8 rows of
+    16384 positions), each launch timed after a 256 MB read flushes L2."""
+    import compressed_kv_cache_kv4_b200 as K
+    from compressed_kv_cache_kv4_b200 import synth
+    wl = synth.workload("evict")
+    k, v, off = synth.gen_kv(wl, device="cuda", lens=wl.lens)
+    del v
+    scores = synth.gen_scores(wl, k, off, device="cuda")
+    del k
+    lens = torch.as_tensor(wl.lens, device="cuda")
+    L = int(wl.lens.max())
+    mask = torch.zeros((wl.B, wl.Hkv, (L + 31) // 32), dtype=torch.int32, device="cuda")
+    count = torch.zeros((wl.B, wl.Hkv), dtype=torch.int32, device="cuda")
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    ms = []
+    for r in range(reps + 3):
+        flush.max()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        K.kv_topk_retain(scores, lens, permille, mask, count, max_len=L)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if r >= 3:
+            ms.append(e0.elapsed_time(e1))
+    med = float(np.median(ms))
+    nbytes = wl.B * wl.Hkv * (L * 4 + (L + 31) // 32 * 4)
+    return {"rows": wl.B * wl.Hkv, "L": L, "permille": permille, "us_l2_flushed": med * 1e3,
+            "gbs": nbytes / (med / 1e3) / 1e9, "retained": int(count.sum().item())}
+
+
+def prefill_only(reps=20):
+    """The prefill append of the qwen8b prompt (lengths L0 - 64) alone."""
+    from compressed_kv_cache_kv4_b200 import synth
+    wl = synth.workload("qwen8b")
+    lens_pre = np.maximum(wl.lens.astype(np.int64) - CYCLE, 0).astype(np.int32)
+    cache, ptd, _, _ = build_kv4(wl, wl.lens, CYCLE, 0)
+    k, v, off = prefill(cache, wl, lens_pre, ptd)
+    offs_t = torch.as_tensor(off.astype(np.int32), device="cuda")
+    zeros = torch.zeros(wl.B, dtype=torch.int32, device="cuda")
+    call, _ = time_calls(lambda: cache.append(k, v, offs_t, zeros, ptd), reps)
+    st = cache.get_error()[0]
+    cache.close()
+    return {"positions": int(off[-1]), "us": call * 1e3, "device_error": st}
+
+
 def evict_secondary(steps=50, page_only=False):
     import compressed_kv_cache_kv4_b200 as K
     from compressed_kv_cache_kv4_b200 import synth
@@ -1006,6 +1057,14 @@ def main():
     if args.learner_only:
         if rank == 0:
             print(json.dumps(learner_secondary()), flush=True)
+        return
+    if args.topk_only:
+        if rank == 0:
+            print(json.dumps(topk_only()), flush=True)
+        return
+    if args.prefill_only:
+        if rank == 0:
+            print(json.dumps(prefill_only()), flush=True)
         return
     wl, res = run_kv4(args, ws, rank)
     if rank == 0:

@@ -18,6 +18,8 @@
 // the passes run over the candidate range between them only, four keys per
 // thread step. The row is held in shared memory when it fits, otherwise re-read
 // from global memory on each pass.
+#include <algorithm>
+
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
 
@@ -26,6 +28,7 @@ namespace kv4 {
 constexpr int kTopkThreads = 512;
 constexpr int kTopkBins = 2048;            // 4 bins per thread in the scan
 constexpr int kTopkSmemKeys = 49152;   // rows up to this length are staged in shared memory
+constexpr int kStageVec = 8;           // 16-byte loads in flight per thread while staging
 
 __device__ __forceinline__ uint32_t score_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -37,12 +40,12 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 // for each. With the row in shared memory four keys come from one 16-byte load
 // (c0 rounded down to a multiple of four); only the first and the last step
 // of the range test each index, the steps between hold four candidates.
-template <bool kSmem, typename F>
+template <bool kSmem, int NT, typename F>
 __device__ __forceinline__ void for_candidates(const uint32_t *keys, const float *srow, int c0, int c1, int tid,
                                                F &&f) {
   const int base = c0 & ~3;
   const int lo = (c0 + 3) & ~3, hi = c1 & ~3;   // [lo, hi): whole steps inside [c0, c1)
-  for (int i = base + 4 * tid; i < c1; i += 4 * kTopkThreads) {
+  for (int i = base + 4 * tid; i < c1; i += 4 * NT) {
     uint32_t k[4];
     if constexpr (kSmem) {
       const uint4 v = *reinterpret_cast<const uint4 *>(keys + i);
@@ -65,17 +68,23 @@ __device__ __forceinline__ void for_candidates(const uint32_t *keys, const float
   }
 }
 
-template <bool kSmem>
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
-  extern __shared__ __align__(16) uint32_t dyn[];
-  __shared__ uint32_t hist[kTopkBins];
-  __shared__ int wsum[kTopkThreads / 32];
-  __shared__ int sh_digit, sh_rem, sh_cnt;
+// Shared state of one row's selection.
+struct TopkShared {
+  uint32_t hist[kTopkBins];
+  int wsum[32];
+  int digit, rem, cnt, listn, kmin, kmax;
+};
+
+// The whole selection of one row by a CTA of NT threads, with the row staged
+// as 32-bit keys in shared memory (kSmem) or re-read from global memory on
+// every pass. dyn: keys [round_up(max_len, 4)] when staged, then tile ranks.
+template <bool kSmem, int NT>
+__device__ void topk_row(const TopkParams &p, int row, uint32_t *dyn, TopkShared &sh) {
+  uint32_t *hist = sh.hist;
+  int *wsum = sh.wsum;
+  int &sh_digit = sh.digit, &sh_rem = sh.rem, &sh_cnt = sh.cnt;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NWARP = kTopkThreads / 32;
-  pdl_wait();
-  pdl_launch_dependents();
-  const int row = blockIdx.x;
+  constexpr int NWARP = NT / 32, BPT = kTopkBins / NT;
   const int b = row / p.Hkv;
   int L = p.seq_lens[b];
   L = L < 0 ? 0 : (L > p.max_len ? p.max_len : L);
@@ -98,18 +107,54 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
 
   // mode: 0 = select none, 1 = select all, 2 = threshold
   const int mode = ksel == 0 ? 0 : (ksel == c1 - c0 ? 1 : 2);
-  if (kSmem && mode == 2) {
+  // with the row staged in shared memory, the first pass's histogram is taken
+  // while staging
+  const bool fused = kSmem && mode == 2;
+  if (fused) {
+    for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0;
+    __syncthreads();
     const int base = c0 & ~3;
     if (p.vec_ok) {
-      // 16-byte loads: the row starts 16-byte aligned and its stride is a
-      // multiple of four, so the last vector ends inside the row's storage
-      for (int i = base + 4 * tid; i < c1; i += 4 * kTopkThreads) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(srow + i));
-        *reinterpret_cast<uint4 *>(keys + i) =
-            make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+      // 16-byte loads, kStageVec of them in flight per thread: the row starts
+      // 16-byte aligned and its stride is a multiple of four, so the last
+      // vector ends inside the row's storage
+      const int nvec = (c1 - base + 3) >> 2;
+      const float4 *src = reinterpret_cast<const float4 *>(srow + base);
+      for (int v0 = tid; v0 < nvec; v0 += kStageVec * NT) {
+        float4 buf[kStageVec];
+#pragma unroll
+        for (int u = 0; u < kStageVec; ++u) {
+          const int v = v0 + u * NT;
+          if (v < nvec) buf[u] = __ldg(src + v);
+        }
+#pragma unroll
+        for (int u = 0; u < kStageVec; ++u) {
+          const int v = v0 + u * NT;
+          if (v < nvec) {
+            const int i = base + 4 * v;
+            const uint4 k4 = make_uint4(score_key(buf[u].x), score_key(buf[u].y), score_key(buf[u].z),
+                                        score_key(buf[u].w));
+            *reinterpret_cast<uint4 *>(keys + i) = k4;
+            if (i >= c0 && i + 4 <= c1) {
+              atomicAdd(&hist[k4.x >> 21], 1u);
+              atomicAdd(&hist[k4.y >> 21], 1u);
+              atomicAdd(&hist[k4.z >> 21], 1u);
+              atomicAdd(&hist[k4.w >> 21], 1u);
+            } else {
+              const uint32_t ka[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (i + e >= c0 && i + e < c1) atomicAdd(&hist[ka[e] >> 21], 1u);
+            }
+          }
+        }
       }
     } else {
-      for (int i = base + tid; i < c1; i += kTopkThreads) keys[i] = score_key(srow[i]);
+      for (int i = base + tid; i < c1; i += NT) {
+        const uint32_t k = score_key(srow[i]);
+        keys[i] = k;
+        if (i >= c0) atomicAdd(&hist[k >> 21], 1u);
+      }
     }
   }
   __syncthreads();
@@ -124,23 +169,26 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
     for (int pass = 0; pass < 3; ++pass) {
       const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
       const uint32_t dmask = pass == 2 ? 1023u : 2047u;
-      for (int i = tid; i < kTopkBins; i += kTopkThreads) hist[i] = 0;
-      __syncthreads();
+      if (pass > 0 || !fused) {
+        for (int i = tid; i < kTopkBins; i += NT) hist[i] = 0;
+        __syncthreads();
+      }
       if (pass == 0) {
-        for_candidates<kSmem>(keys, srow, c0, c1, tid,
-                              [&](int, uint32_t k) { atomicAdd(&hist[k >> shift], 1u); });
+        if (!fused)
+          for_candidates<kSmem, NT>(keys, srow, c0, c1, tid,
+                                [&](int, uint32_t k) { atomicAdd(&hist[k >> shift], 1u); });
       } else {
-        for_candidates<kSmem>(keys, srow, c0, c1, tid, [&](int, uint32_t k) {
+        for_candidates<kSmem, NT>(keys, srow, c0, c1, tid, [&](int, uint32_t k) {
           if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
         });
       }
       __syncthreads();
-      // thread i owns bins kTopkBins-1-4i .. kTopkBins-4-4i (highest first):
-      // block-wide exclusive scan of the per-thread counts from the top
-      int cnt[4], tot = 0;
+      // thread i owns bins kTopkBins-1-BPT*i .. kTopkBins-BPT-BPT*i (highest
+      // first): block-wide exclusive scan of the per-thread counts from the top
+      int cnt[BPT], tot = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        cnt[j] = hist[kTopkBins - 1 - 4 * tid - j];
+      for (int j = 0; j < BPT; ++j) {
+        cnt[j] = hist[kTopkBins - 1 - BPT * tid - j];
         tot += cnt[j];
       }
       int incl = tot;
@@ -154,9 +202,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
       int c = incl - tot;
       for (int w = 0; w < warp; ++w) c += wsum[w];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < BPT; ++j) {
         if (c < rem && rem <= c + cnt[j]) {
-          sh_digit = kTopkBins - 1 - 4 * tid - j;
+          sh_digit = kTopkBins - 1 - BPT * tid - j;
           sh_rem = rem - c;
           sh_cnt = cnt[j];
         }
@@ -200,9 +248,55 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
     }
   }
 
+  uint32_t *mrow = p.mask + (long long)row * p.mask_stride;
+  if (kSmem && mode == 2) {
+    // mask words from the staged keys: a warp covers 128 positions (4 words)
+    // per step, lane l positions 4l .. 4l+3 from one 16-byte load; the 8 lanes
+    // of a word OR their 4-bit pieces together
+    const int sub = lane & 7;
+    for (int it = warp; 4 * it < nt; it += NWARP) {
+      const int pos = 128 * it + 4 * lane;
+      uint4 k4 = make_uint4(0, 0, 0, 0);
+      if (pos + 4 > c0 && pos < c1) k4 = *reinterpret_cast<const uint4 *>(keys + pos);
+      const uint32_t ka[4] = {k4.x, k4.y, k4.z, k4.w};
+      uint32_t sel = 0, eq = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int q = pos + e;
+        const bool cand = q >= c0 && q < c1;
+        const bool f = q < L && !cand;
+        sel |= static_cast<uint32_t>(f || (cand && (ka[e] > T || (!ties && ka[e] == T)))) << e;
+        eq |= static_cast<uint32_t>(cand && ties && ka[e] == T) << e;
+      }
+      sel <<= 4 * sub;
+      eq <<= 4 * sub;
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        sel |= __shfl_xor_sync(0xffffffffu, sel, o);
+        eq |= __shfl_xor_sync(0xffffffffu, eq, o);
+      }
+      const int w = 4 * it + (lane >> 3);
+      if (ties) {   // uniform over the CTA
+        // equal keys in index order take the remaining places
+        uint32_t mine = (eq >> (4 * sub)) & 15u;
+        if (mine) {
+          const int r0 = tile_rank[w];
+          while (mine) {
+            const int b = 4 * sub + __ffs(mine) - 1;
+            mine &= mine - 1;
+            if (r0 + __popc(eq & ((1u << b) - 1u)) < need_eq) sel |= 1u << b;
+          }
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) sel |= __shfl_xor_sync(0xffffffffu, sel, o);
+      }
+      if (sub == 0 && w < nt) mrow[w] = sel;
+    }
+    if (tid == 0 && p.count) p.count[row] = nF + static_cast<int>(ksel);
+    return;
+  }
   // mask words: a warp builds 32 consecutive words (lane i keeps word i) and
   // stores them together
-  uint32_t *mrow = p.mask + (long long)row * p.mask_stride;
   for (int w0 = 32 * warp; w0 < nt; w0 += 32 * NWARP) {
     uint32_t mine = 0;
     const int n = min(32, nt - w0);
@@ -228,9 +322,351 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
   if (tid == 0 && p.count) p.count[row] = nF + static_cast<int>(ksel);
 }
 
+// ---------------------------------------------------------------------------
+// Rows of up to kFastMaxLen positions with 16-byte aligned scores: the row is
+// staged as the top 16 bits of its keys (so four CTAs share an SM and a batch
+// of rows runs in one wave). The first histogram bins the candidates' key
+// prefixes relative to the row's own range, (prefix - min) >> s with the
+// smallest s that fits 2048 bins: scores that span a few octaves spread over
+// about a thousand counters instead of the few dozen that fixed sign and
+// exponent bits would give, so the shared-memory atomics rarely collide. One
+// pass over the staged prefixes then writes every mask bit except those of the
+// threshold bin and lists that bin's positions; the exact threshold is
+// selected among the listed keys (full keys re-read from global memory, cached
+// in L2 by then) and their bits are set last. A threshold bin larger than
+// kListCap falls back to the general path.
+// ---------------------------------------------------------------------------
+constexpr int kFastThreads = 256;
+constexpr int kFastMaxLen = 16384;
+constexpr int kListCap = 2048;
+constexpr int kFastStageVec = 4;   // 16-byte loads in flight per thread while staging
+
+// score_key with -0 folded by adding +0 (rounding to nearest gives +0).
+__device__ __forceinline__ uint32_t score_key2(float f) {
+  const uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
+  return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
+}
+
+// Bits of the positions [lo, hi) that fall in mask word w.
+__device__ __forceinline__ uint32_t range_bits(int w, int lo, int hi) {
+  const int a = max(lo - 32 * w, 0), z = min(hi - 32 * w, 32);
+  if (z <= a) return 0u;
+  return (z >= 32 ? 0xFFFFFFFFu : ((1u << z) - 1u)) & ~((1u << a) - 1u);
+}
+
+// Block-wide: the bin (highest first) holding the rem-th largest key of the
+// histogram, the rank left inside it and its count, into sh.digit / rem / cnt.
+template <int NT>
+__device__ void select_bin(TopkShared &sh, int rem, int tid) {
+  constexpr int BPT = kTopkBins / NT;
+  const int lane = tid & 31, warp = tid >> 5;
+  int cnt[BPT], tot = 0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    cnt[j] = sh.hist[kTopkBins - 1 - BPT * tid - j];
+    tot += cnt[j];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sh.wsum[warp] = incl;
+  __syncthreads();
+  int c = incl - tot;
+  for (int w = 0; w < warp; ++w) c += sh.wsum[w];
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) {
+    if (c < rem && rem <= c + cnt[j]) {
+      sh.digit = kTopkBins - 1 - BPT * tid - j;
+      sh.rem = rem - c;
+      sh.cnt = cnt[j];
+    }
+    c += cnt[j];
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p) {
+  constexpr int NT = kFastThreads, NWARP = NT / 32;
+  extern __shared__ __align__(16) uint8_t dynb[];
+  __shared__ TopkShared sh;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int row = blockIdx.x;
+  const int b = row / p.Hkv;
+  int L = p.seq_lens[b];
+  L = L < 0 ? 0 : (L > p.max_len ? p.max_len : L);
+  const float *srow = p.scores + (long long)row * p.score_stride;
+  const int nt = (L + 31) / 32;
+  const int c0 = min(p.sink, L), c1 = max(c0, L - p.recent);
+  const int nF = L - (c1 - c0);
+  const long long kb = (long long)L * p.permille / 1000;
+  long long ksel = kb - nF;
+  if (ksel < 0) ksel = 0;
+  if (ksel > c1 - c0) ksel = c1 - c0;
+  const int mode = ksel == 0 ? 0 : (ksel == c1 - c0 ? 1 : 2);
+  uint32_t *mrow = p.mask + (long long)row * p.mask_stride;
+  if (mode != 2) {
+    // no selection: the forced positions, or every position
+    for (int w = tid; w < nt; w += NT)
+      mrow[w] = mode == 1 ? range_bits(w, 0, L) : (range_bits(w, 0, c0) | range_bits(w, c1, L));
+    if (tid == 0 && p.count) p.count[row] = nF + static_cast<int>(ksel);
+    return;
+  }
+  // shared memory: key prefixes [KR] u16 | mask words [round_up(nt_max, 4)] |
+  // listed keys [kListCap] u32 | listed positions [kListCap] u16
+  // (the prefix area also holds 2 * NTW words of tie bookkeeping later)
+  const int NTW = ((p.max_len + 31) / 32 + 3) & ~3, KR = max((p.max_len + 7) & ~7, 4 * NTW);
+  uint16_t *keys16 = reinterpret_cast<uint16_t *>(dynb);
+  uint32_t *maskw = reinterpret_cast<uint32_t *>(dynb + 2 * KR);
+  uint32_t *list_key = maskw + NTW;
+  uint16_t *list_pos = reinterpret_cast<uint16_t *>(list_key + kListCap);
+
+  // A. stage the key prefixes and find the candidates' prefix range
+  for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
+  if (tid == 0) sh.listn = 0;
+  uint32_t kmin = 0xFFFFu, kmax = 0u;
+  const int base = c0 & ~3;
+  const int nvec = (c1 - base + 3) >> 2;
+  const float4 *src = reinterpret_cast<const float4 *>(srow + base);
+  for (int v0 = tid; v0 < nvec; v0 += kFastStageVec * NT) {
+    float4 buf[kFastStageVec];
+#pragma unroll
+    for (int u = 0; u < kFastStageVec; ++u) {
+      const int v = v0 + u * NT;
+      if (v < nvec) buf[u] = __ldg(src + v);
+    }
+#pragma unroll
+    for (int u = 0; u < kFastStageVec; ++u) {
+      const int v = v0 + u * NT;
+      if (v < nvec) {
+        const int i = base + 4 * v;
+        const uint32_t k0 = score_key2(buf[u].x), k1 = score_key2(buf[u].y), k2 = score_key2(buf[u].z),
+                       k3 = score_key2(buf[u].w);
+        *reinterpret_cast<uint2 *>(keys16 + i) = make_uint2(__byte_perm(k0, k1, 0x7632), __byte_perm(k2, k3, 0x7632));
+        if (i >= c0 && i + 4 <= c1) {
+          kmin = min(kmin, min(min(k0, k1), min(k2, k3)) >> 16);
+          kmax = max(kmax, max(max(k0, k1), max(k2, k3)) >> 16);
+        } else {
+          const uint32_t ka[4] = {k0, k1, k2, k3};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (i + e >= c0 && i + e < c1) {
+              kmin = min(kmin, ka[e] >> 16);
+              kmax = max(kmax, ka[e] >> 16);
+            }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) {
+    sh.wsum[warp] = static_cast<int>(kmin);
+    sh.wsum[16 + warp] = static_cast<int>(kmax);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int a = sh.wsum[0], z = sh.wsum[16];
+    for (int w = 1; w < NWARP; ++w) {
+      a = min(a, sh.wsum[w]);
+      z = max(z, sh.wsum[16 + w]);
+    }
+    sh.kmin = a;
+    sh.kmax = z;
+  }
+  __syncthreads();
+  const uint32_t pmin = static_cast<uint32_t>(sh.kmin);
+  int sh16 = 0;   // bin of a candidate: (prefix - pmin) >> sh16 < kTopkBins
+  while (((static_cast<uint32_t>(sh.kmax) - pmin) >> sh16) >= static_cast<uint32_t>(kTopkBins)) ++sh16;
+  // B. histogram of the bins (prefixes from shared memory, 4 per load), the
+  // threshold bin d0 and the rank left inside it
+  for (int i = base + 4 * tid; i < c1; i += 4 * NT) {
+    const uint2 k2 = *reinterpret_cast<const uint2 *>(keys16 + i);
+    const uint32_t kp[4] = {k2.x & 0xFFFFu, k2.x >> 16, k2.y & 0xFFFFu, k2.y >> 16};
+    if (i >= c0 && i + 4 <= c1) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) atomicAdd(&sh.hist[(kp[e] - pmin) >> sh16], 1u);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i + e >= c0 && i + e < c1) atomicAdd(&sh.hist[(kp[e] - pmin) >> sh16], 1u);
+    }
+  }
+  __syncthreads();
+  select_bin<NT>(sh, static_cast<int>(ksel), tid);
+  const uint32_t d0 = static_cast<uint32_t>(sh.digit);
+  const int rem0 = sh.rem, n0 = sh.cnt;
+  if (n0 > kListCap) {
+    // a crowded threshold bin: the general path, keys re-read from global memory
+    __syncthreads();
+    topk_row<false, NT>(p, row, reinterpret_cast<uint32_t *>(dynb), sh);
+    return;
+  }
+  // C. mask bits of every position outside bin d0; bin d0's positions listed
+  // (their full keys are fetched after the pass, from L2).
+  // A warp covers 128 positions (4 words) per step: lane l positions 4l..4l+3
+  // from one 8-byte load; the 8 lanes of a word OR their 4-bit pieces.
+  // Bin d0 holds the prefixes [lo16, lo16 + 2^s); with four candidates per
+  // lane the bounds are compared two prefixes at a time.
+  const int sub = lane & 7;
+  const uint32_t lo16 = pmin + (d0 << sh16), hi16 = lo16 + (1u << sh16);
+  const bool top = hi16 > 0xFFFFu;   // no prefix lies above bin d0
+  const uint32_t lo2 = lo16 * 0x10001u, hi2 = (top ? 0xFFFFu : hi16) * 0x10001u;
+  for (int it = warp; 4 * it < nt; it += NWARP) {
+    const int pos = 128 * it + 4 * lane;
+    uint32_t sel = 0, lst = 0;
+    if (pos >= c0 && pos + 4 <= c1) {
+      const uint2 k2 = *reinterpret_cast<const uint2 *>(keys16 + pos);
+      // 0xFFFF in a half where its prefix is >= the bound
+      const uint32_t gl0 = __vcmpgeu2(k2.x, lo2), gl1 = __vcmpgeu2(k2.y, lo2);
+      const uint32_t gh0 = top ? 0u : __vcmpgeu2(k2.x, hi2), gh1 = top ? 0u : __vcmpgeu2(k2.y, hi2);
+      const uint32_t in0 = gl0 & ~gh0, in1 = gl1 & ~gh1;
+      sel = (gh0 & 1u) | ((gh0 >> 15) & 2u) | ((gh1 & 1u) << 2) | ((gh1 >> 13) & 8u);
+      lst = (in0 & 1u) | ((in0 >> 15) & 2u) | ((in1 & 1u) << 2) | ((in1 >> 13) & 8u);
+    } else {
+      uint2 k2 = make_uint2(0, 0);
+      if (pos + 4 > c0 && pos < c1) k2 = *reinterpret_cast<const uint2 *>(keys16 + pos);
+      const uint32_t kp[4] = {k2.x & 0xFFFFu, k2.x >> 16, k2.y & 0xFFFFu, k2.y >> 16};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int q = pos + e;
+        const bool cand = q >= c0 && q < c1;
+        const bool above = !top && kp[e] >= hi16, inbin = kp[e] >= lo16 && !above;
+        sel |= static_cast<uint32_t>((q < L && !cand) || (cand && above)) << e;
+        lst |= static_cast<uint32_t>(cand && inbin) << e;
+      }
+    }
+    sel <<= 4 * sub;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) sel |= __shfl_xor_sync(0xffffffffu, sel, o);
+    const int w = 4 * it + (lane >> 3);
+    if (sub == 0 && w < nt) maskw[w] = sel;
+    if (!__any_sync(0xffffffffu, lst != 0)) continue;
+    // list bin d0: warp-wide slots, one shared-memory atomic per warp
+    const int nl = __popc(lst);
+    int excl = nl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, excl, o);
+      if (lane >= o) excl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, excl, 31);
+    excl -= nl;
+    int at = 0;
+    if (lane == 0 && total) at = atomicAdd(&sh.listn, total);
+    at = __shfl_sync(0xffffffffu, at, 0) + excl;
+    while (lst) {
+      const int e = __ffs(lst) - 1;
+      lst &= lst - 1;
+      list_pos[at++] = static_cast<uint16_t>(pos + e);
+    }
+  }
+  __syncthreads();
+  // the listed positions' full keys, all loads in flight together
+  for (int i = tid; i < n0; i += NT) list_key[i] = score_key2(srow[list_pos[i]]);
+  __syncthreads();
+  // D. the exact threshold inside bin d0: its keys lie in [kbase, kbase + 2^(16+s))
+  // with s <= 5, so two 11-bit digits of key - kbase finish the selection
+  const int n = n0;
+  const uint32_t kbase = (pmin + (d0 << sh16)) << 16;
+  for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += NT) atomicAdd(&sh.hist[(list_key[i] - kbase) >> 11], 1u);
+  __syncthreads();
+  select_bin<NT>(sh, rem0, tid);
+  const uint32_t d1 = static_cast<uint32_t>(sh.digit);
+  const int rem1 = sh.rem;
+  __syncthreads();
+  for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += NT) {
+    const uint32_t k = list_key[i] - kbase;
+    if ((k >> 11) == d1) atomicAdd(&sh.hist[k & 2047u], 1u);
+  }
+  __syncthreads();
+  select_bin<NT>(sh, rem1, tid);
+  const uint32_t T = kbase + (d1 << 11) + static_cast<uint32_t>(sh.digit);
+  const int need_eq = sh.rem;
+  const bool ties = need_eq < sh.cnt;
+  // E. bits of the listed positions: keys above T, and keys equal to T by
+  // index order (ranks from a bitmap of the equal keys and a scan over words)
+  if (!ties) {
+    for (int i = tid; i < n; i += NT)
+      if (list_key[i] >= T) {
+        const int q = list_pos[i];
+        atomicOr(&maskw[q >> 5], 1u << (q & 31));
+      }
+  } else {
+    uint32_t *eqw = reinterpret_cast<uint32_t *>(dynb);   // the key prefixes are no longer needed
+    int *tile_rank = reinterpret_cast<int *>(eqw + NTW);
+    for (int w = tid; w < nt; w += NT) eqw[w] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += NT)
+      if (list_key[i] == T) {
+        const int q = list_pos[i];
+        atomicOr(&eqw[q >> 5], 1u << (q & 31));
+      }
+    __syncthreads();
+    if (warp == 0) {
+      int carry = 0;
+      for (int w0 = 0; w0 < nt; w0 += 32) {
+        const int w = w0 + lane;
+        const int v = w < nt ? __popc(eqw[w]) : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (w < nt) tile_rank[w] = carry + incl - v;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += NT) {
+      const uint32_t k = list_key[i];
+      const int q = list_pos[i], w = q >> 5;
+      bool take = k > T;
+      if (k == T) take = tile_rank[w] + __popc(eqw[w] & ((1u << (q & 31)) - 1u)) < need_eq;
+      if (take) atomicOr(&maskw[w], 1u << (q & 31));
+    }
+  }
+  __syncthreads();
+  for (int w = tid; w < nt; w += NT) mrow[w] = maskw[w];
+  if (tid == 0 && p.count) p.count[row] = nF + static_cast<int>(ksel);
+}
+
+template <bool kSmem>
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p) {
+  extern __shared__ __align__(16) uint32_t dyn[];
+  __shared__ TopkShared sh;
+  pdl_wait();
+  pdl_launch_dependents();
+  topk_row<kSmem, kTopkThreads>(p, blockIdx.x, dyn, sh);
+}
+
+size_t topk_fast_smem(int max_len) {
+  const size_t NTW = ((size_t)(max_len + 31) / 32 + 3) & ~(size_t)3;
+  const size_t KR = std::max((size_t)(max_len + 7) & ~(size_t)7, 4 * NTW);
+  return 2 * KR + 4 * NTW + 6 * (size_t)kListCap;
+}
+
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream) {
   const int rows = p.B * p.Hkv;
   if (rows == 0) return cudaSuccess;
+  if (p.vec_ok && p.max_len <= kFastMaxLen) {
+    const size_t smem = topk_fast_smem(p.max_len);
+    cudaError_t e = cudaFuncSetAttribute(topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(topk_fast_kernel, dim3(rows), dim3(kFastThreads), smem, stream, p);
+  }
   const bool use_smem = p.max_len <= kTopkSmemKeys;
   const size_t smem = (use_smem ? (size_t)(p.max_len + 3) / 4 * 16 : 0) + (size_t)((p.max_len + 31) / 32) * 4;
   auto kern = use_smem ? topk_kernel<true> : topk_kernel<false>;

@@ -219,6 +219,33 @@ def test_topk_matches_oracle(permille):
     assert np.array_equal(count.cpu().numpy(), c_ref)
 
 
+@pytest.mark.parametrize("permille", [100, 500])
+def test_topk_crowded_threshold_bin(permille):
+    """Rows whose threshold bin (sign, exponent and two mantissa bits) holds
+    more keys than the short list of the staged path: equal scores, one large
+    block of equal scores among random ones, and distinct scores that all lie
+    in [1, 1.25). The selection falls back to the general path and must give
+    the same masks."""
+    rng = np.random.default_rng(permille + 7)
+    B, Hkv, Lmax = 2, 2, 6000
+    lens = np.array([6000, 5003], np.int32)
+    sc = rng.standard_normal((B, Hkv, Lmax)).astype(np.float32)
+    sc[0, 0, :] = 1.0
+    sc[0, 1, 1000:4000] = 2.0
+    sc[1, 0, :] = (1.0 + 0.25 * rng.random(Lmax)).astype(np.float32)
+    sc[1, 1, :] = np.float32(1.0) + np.float32(2.0 ** -20) * rng.integers(0, 64, Lmax).astype(np.float32)
+    mstride = (Lmax + 31) // 32
+    mask = torch.zeros((B, Hkv, mstride), dtype=torch.int32, device="cuda")
+    count = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+    K.kv_topk_retain(torch.as_tensor(sc, device="cuda"), torch.as_tensor(lens, device="cuda"), permille, mask, count)
+    m_ref, c_ref = O.topk(sc, lens, permille)
+    got = mask.cpu().numpy().view(np.uint32)
+    for b in range(B):
+        nw = (int(lens[b]) + 31) // 32
+        assert np.array_equal(got[b, :, :nw], m_ref[b, :, :nw]), b
+    assert np.array_equal(count.cpu().numpy(), c_ref)
+
+
 def test_topk_long_rows_global_path():
     rng = np.random.default_rng(9)
     B, Hkv, Lmax = 1, 2, 70000
