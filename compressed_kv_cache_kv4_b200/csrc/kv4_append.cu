@@ -54,7 +54,9 @@ __device__ __forceinline__ float round_code(float x, float s, float r) {
 // half-way test uses the exact residual, not r.
 __device__ __forceinline__ float2 round_code2(float2 x, float s, float r) {
   const float2 q = __fmul2_rn(x, make_float2(r, r));
-  float2 c = make_float2(rintf(q.x), rintf(q.y));
+  // nearest-even integer of q (|q| < 2^22): adding 1.5 * 2^23 rounds q to an
+  // integer in the last mantissa place, subtracting it again is exact
+  float2 c = __fadd2_rn(__fadd2_rn(q, make_float2(12582912.f, 12582912.f)), make_float2(-12582912.f, -12582912.f));
   const float2 d = __ffma2_rn(c, make_float2(s, s), make_float2(-x.x, -x.y));   // c*s - x, exact
   if (2.f * fabsf(d.x) == s || 2.f * fabsf(d.y) == s) {   // rare: an exact half-way point
     if (2.f * fabsf(d.x) == s && (static_cast<int>(c.x) & 1)) c.x -= copysignf(1.f, d.x);
