@@ -743,8 +743,12 @@ def evict_secondary(steps=50, page_only=False):
         call, kern = time_calls(lambda: K.kv4_decode_attn(cache.handle, q, lens, ptd, wl.softmax_scale, wsb, o,
                                                           retain_mask=mask), steps, kind=0)
         kept = int(count.sum().item()) / wl.Hkv
+        # the gathered path: retained INT4 rows packed into compact pages, then decoded
+        bound = L * permille // 1000
+        callg, _ = time_calls(lambda: cache.decode_masked(q, lens, ptd, wl.softmax_scale, mask, bound, out=o), steps)
         res["%d" % permille] = {"topk_us": tk * 1e3, "topk_us_l2_flushed": tkf * 1e3,
                                 "masked_decode_us": call * 1e3, "worker_us": kern * 1e3,
+                                "masked_gather_decode_us": callg * 1e3,
                                 "retained_positions_per_s": kept / ((tk + call) / 1e3),
                                 "topk_gbs": wl.B * wl.Hkv * L * 4 / (tk / 1e3) / 1e9,
                                 "topk_gbs_l2_flushed": wl.B * wl.Hkv * L * 4 / (tkf / 1e3) / 1e9}

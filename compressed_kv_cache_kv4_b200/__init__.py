@@ -8,6 +8,7 @@ fallback implementation.
 
 Names mirror the C ABI (kv4_cache_bytes, kv4_cache_create, kv4_append,
 kv4_workspace_bytes, kv4_decode_attn, kv4_decode_partials, kv4_merge_partials,
+kv4_masked_workspace_bytes, kv4_decode_attn_masked,
 kv_topk_retain, kv4_evict_pages, smd_masked_attn, bf16_paged_decode_attn,
 kv4_get_error); ``KV4Cache`` bundles the buffers and handle of one cache;
 ``cp`` holds the context-parallel plumbing (shard plan, gather of partials).
@@ -67,6 +68,9 @@ def lib():
         "kv4_decode_partials": (C.c_int, [_P, _P, _P, _I32, _P, _P, _I32, _P, _P, _I32, _P, _I32, C.c_float,
                                           _I32, _P, _SZ, _P, _I32]),
         "kv4_merge_partials": (C.c_int, [_P, _P, _I32, _I32, _I32, _I32, _P, _I32]),
+        "kv4_masked_workspace_bytes": (C.c_int, [_P, _I32, _I32, _I32, _I32, C.POINTER(_SZ)]),
+        "kv4_decode_attn_masked": (C.c_int, [_P, _P, _P, _I32, _P, _P, _I32, _P, _I32, _I32, C.c_float, _P, _SZ,
+                                             _P, _I32, _I32]),
         "kv_topk_retain": (C.c_int, [_P, _P, _I64, _P, _I32, _I32, _I32, _I32, _I32, _P, _I32, _P, _I32]),
         "kv4_evict_pages": (C.c_int, [_P, _P, _P, _I64, _I32, _P, _P, _I32, _P, _P, _I32]),
         "smd_masked_attn": (C.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P, _I32, C.c_float,
@@ -178,6 +182,27 @@ def kv4_merge_partials(partials, out, stream=None):
     st = lib().kv4_merge_partials(_stream(stream), _ptr(partials), N, B, Hq, D4 - 4, _ptr(out),
                                   1 if out.dtype == torch.float32 else 0)
     _check(st, "kv4_merge_partials")
+
+
+def kv4_masked_workspace_bytes(handle, B, Hq, pt_stride, max_retained):
+    n = _SZ()
+    _check(lib().kv4_masked_workspace_bytes(handle, B, Hq, pt_stride, max_retained, C.byref(n)),
+           "kv4_masked_workspace_bytes")
+    return n.value
+
+
+def kv4_decode_attn_masked(handle, q, seq_lens, page_table, softmax_scale, retain_mask, max_retained, workspace, out,
+                           stream=None):
+    """Masked decode with the INT4 region's retained rows gathered into compact
+    pages first (reads and work follow the retained count); out [B][Hq][D]
+    bf16 or fp32."""
+    B, Hq, _ = q.shape
+    st = lib().kv4_decode_attn_masked(handle, _stream(stream), _ptr(q), Hq, _ptr(seq_lens), _ptr(page_table),
+                                      page_table.shape[1], _ptr(retain_mask), retain_mask.shape[-1], max_retained,
+                                      C.c_float(softmax_scale), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _ptr(out),
+                                      1 if out.dtype == torch.float32 else 0, B)
+    _check(st, "kv4_decode_attn_masked")
 
 
 # Size of the fixed per-device scratch of kv4_decode_attn_noalloc (KV4_NOALLOC_SCRATCH_BYTES).
@@ -338,6 +363,22 @@ class KV4Cache:
         ws = self.workspace(B, Hq, num_workers)
         kv4_decode_attn(self.handle, q, seq_lens, page_table, softmax_scale, ws, out, retain_mask,
                         num_workers, stream)
+        return out
+
+    def decode_masked(self, q, seq_lens, page_table, softmax_scale, retain_mask, max_retained, out=None,
+                      out_fp32=False, stream=None):
+        """kv4_decode_attn_masked: the retained INT4 rows gathered into compact
+        pages first; max_retained bounds the retained INT4-region positions of
+        any (sequence, head)."""
+        B, Hq, D = q.shape
+        if out is None:
+            out = torch.empty((B, Hq, D), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+        key = ("masked", B, Hq, page_table.shape[1], max_retained)
+        if key not in self._ws:
+            n = kv4_masked_workspace_bytes(self.handle, B, Hq, page_table.shape[1], max_retained)
+            self._ws[key] = torch.zeros(n, dtype=torch.uint8, device=self.pool.device)
+        kv4_decode_attn_masked(self.handle, q, seq_lens, page_table, softmax_scale, retain_mask, max_retained,
+                               self._ws[key], out, stream)
         return out
 
     def evict_pages(self, scores, budget_permille, seq_lens, page_table, stream=None):

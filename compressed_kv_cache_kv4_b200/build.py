@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libkv4.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-SOURCES = ["kv4_api.cu", "kv4_append.cu", "kv4_decode.cu", "kv4_merge.cu", "kv_topk.cu", "kv4_noalloc.cu", "kv4_evict.cu", "smd_attn.cu"]
+SOURCES = ["kv4_api.cu", "kv4_append.cu", "kv4_decode.cu", "kv4_merge.cu", "kv_topk.cu", "kv4_noalloc.cu", "kv4_evict.cu", "smd_attn.cu", "kv4_masked.cu"]
 HEADERS = ["kv4_common.cuh", "kv4_internal.h", "kv4_evict.h", "smd_attn.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -206,6 +206,40 @@ kv4_status kv4_decode_partials(kv4_cache *cache, void *stream, const void *q, in
                                size_t ws_bytes, float *partials, int32_t B);
 
 /*
+ * kv4_masked_workspace_bytes / kv4_decode_attn_masked -- kv4_decode_attn under
+ * a retained-position mask, with the INT4 region's reads and work following
+ * the retained count. Shadow Mask Distillation, sec. 1 and Figure 1: eviction
+ * is a binary mask applied inside attention instead of slicing the cache;
+ * KV4-RL review, sec. 3: the INT4 and INT8 regions are attended separately
+ * and merged exactly.
+ * The retained INT4-region positions of every (sequence, KV head) are gathered,
+ * in position order, into dense pages of the ordinary layout in the workspace
+ * (K rows and scales whole; V rows from the 4-row groups that hold them), the
+ * ordinary decode attends those pages, the INT8 region is attended from the
+ * side cache under the same mask, and the two partials are merged. The result
+ * is the same attention as kv4_decode_attn with retain_mask (within rounding).
+ *  retain_mask: device uint32 [B][Hkv][mask_stride], required; mask_stride *
+ *    32 >= pt_stride * 16.
+ *  max_retained: host bound on the retained positions of the INT4 region
+ *    [sink, L - recent) of any (sequence, head); it sizes the workspace
+ *    (ceil(max_retained / 16) pages per sequence). For a kv_topk_retain mask
+ *    with budget k = floor(L * permille / 1000) it is at most k. A row with more
+ *    sets KV4_ERR_CAPACITY and only its first max_retained positions are
+ *    attended.
+ *  workspace: device, >= kv4_masked_workspace_bytes(), 256-byte aligned.
+ * Other arguments as kv4_decode_attn (the default worker count is used).
+ * Launches: a count kernel, a gather kernel, two decode worker + merge pairs
+ * and a partial merge, all on `stream`.
+ */
+kv4_status kv4_masked_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t Hq, int32_t pt_stride,
+                                      int32_t max_retained, size_t *bytes);
+kv4_status kv4_decode_attn_masked(kv4_cache *cache, void *stream, const void *q, int32_t Hq,
+                                  const int32_t *seq_lens, const int32_t *page_table, int32_t pt_stride,
+                                  const uint32_t *retain_mask, int32_t mask_stride, int32_t max_retained,
+                                  float softmax_scale, void *workspace, size_t ws_bytes, void *out,
+                                  int32_t out_is_fp32, int32_t B);
+
+/*
  * kv4_merge_partials -- exact softmax merge of N partials per (sequence, query
  * head), e.g. those of N context shards gathered from N GPUs (KV4-RL review,
  * sec. 3: the exact merge of (max, sum, output) triples): with
