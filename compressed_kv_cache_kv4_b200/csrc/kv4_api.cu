@@ -471,38 +471,29 @@ kv4_status kv4_decode_partials(kv4_cache *cache, void *stream, const void *q, in
 
 namespace {
 
-// Workspace of kv4_decode_attn_masked: the ordinary decode workspace, then
-// counts [B*Hkv] | compact lengths [B] and B zeros (one memset) | compact page
-// table [B*PPS] | word prefix counts [B*Hkv*words] | compact mask
-// [B*Hkv*MSC] | two partial arrays [2][B][Hq][D+4] | compact pool [B*PPS pages].
+// Workspace of kv4_decode_attn_masked: the ordinary decode workspace (for the
+// INT8 region), then counts [B*Hkv] | B zeros (empty page ranges) | word prefix
+// counts [B*Hkv*words] | partials [W+1][B][Hq][D+4] (one per warp of the
+// gathering kernel, then the INT8 region's).
 struct MaskedLayout {
-  size_t counts, lens, pt, wpre, mask, parts, pool, total;
-  int PPS, words, MSC;
+  size_t counts, lens, wpre, parts, total;
+  int words, nparts;
 };
 
-MaskedLayout masked_layout(const kv4_cache *cache, const Kv4Plan &pl, int B, int Hq, int pt_stride,
-                           int max_retained) {
+MaskedLayout masked_layout(const kv4_cache *cache, const Kv4Plan &pl, int B, int Hq, int pt_stride) {
   const int D = cache->cfg.head_dim, Hkv = cache->cfg.num_kv_heads, G = Hq / Hkv;
   MaskedLayout l{};
-  l.PPS = (max_retained + kPageTokens - 1) / kPageTokens;
   l.words = (pt_stride * kPageTokens + 31) / 32;
-  l.MSC = std::max(1, (l.PPS * kPageTokens + 31) / 32);
-  const size_t page_bytes = (size_t)page_head_bytes(D) * Hkv;
+  l.nparts = masked_decode_warps() + 1;
   size_t o = round_up(kv4_ws_bytes(pl, G, D), kAlign);
   l.counts = o;
   o += round_up((size_t)B * Hkv * 4, kAlign);
   l.lens = o;
-  o += round_up((size_t)2 * B * 4, kAlign);
-  l.pt = o;
-  o += round_up((size_t)B * l.PPS * 4, kAlign);
+  o += round_up((size_t)B * 4, kAlign);
   l.wpre = o;
   o += round_up((size_t)B * Hkv * l.words * 4, kAlign);
-  l.mask = o;
-  o += round_up((size_t)B * Hkv * l.MSC * 4, kAlign);
   l.parts = o;
-  o += round_up((size_t)2 * B * Hq * (D + 4) * 4, kAlign);
-  l.pool = o;
-  o += round_up((size_t)B * l.PPS * page_bytes, kAlign);
+  o += round_up((size_t)l.nparts * B * Hq * (D + 4) * 4, kAlign);
   l.total = o;
   return l;
 }
@@ -515,7 +506,6 @@ kv4_status masked_check(const kv4_cache *cache, int B, int Hq, int pt_stride, in
   if (G != 1 && G != 2 && G != 4) return KV4_ERR_UNSUPPORTED;
   if (B > cache->cfg.max_seqs) return KV4_ERR_CAPACITY;
   if (B > kMaxBatch || pt_stride > kMaxPtStride) return KV4_ERR_UNSUPPORTED;
-  if ((long long)B * ((max_retained + kPageTokens - 1) / kPageTokens) > INT32_MAX / 2) return KV4_ERR_UNSUPPORTED;
   return kv4_plan(D, G, Hkv, B > 0 ? B : 1, 0, pl);
 }
 
@@ -529,7 +519,7 @@ kv4_status kv4_masked_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t
   Kv4Plan pl{};
   const kv4_status st = masked_check(cache, B, Hq, pt_stride, max_retained, &pl);
   if (st != KV4_OK) return st;
-  *bytes = masked_layout(cache, pl, B, Hq, pt_stride, max_retained).total;
+  *bytes = masked_layout(cache, pl, B, Hq, pt_stride).total;
   return KV4_OK;
 }
 
@@ -549,60 +539,52 @@ kv4_status kv4_decode_attn_masked(kv4_cache *cache, void *stream, const void *q,
   int dev = -1;
   if (bad(cudaGetDevice(&dev))) return KV4_ERR_CUDA;
   if (dev != cache->device) return KV4_ERR_INVALID;
-  const MaskedLayout l = masked_layout(cache, pl, B, Hq, pt_stride, max_retained);
+  const MaskedLayout l = masked_layout(cache, pl, B, Hq, pt_stride);
   if (ws_bytes < l.total) return KV4_ERR_INVALID;
   const int D = cache->cfg.head_dim, Hkv = cache->cfg.num_kv_heads, G = Hq / Hkv;
   uint8_t *w = static_cast<uint8_t *>(workspace);
   const size_t dec_bytes = kv4_ws_bytes(pl, G, D);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int *lens_c = reinterpret_cast<int *>(w + l.lens), *zeros = lens_c + B;
+  int *zeros = reinterpret_cast<int *>(w + l.lens);
   float *parts = reinterpret_cast<float *>(w + l.parts);
   const long long part_floats = (long long)B * Hq * (D + 4);
-  if (bad(cudaMemsetAsync(lens_c, 0, (size_t)2 * B * 4, s))) return KV4_ERR_CUDA;
-  int nparts = 0;
-  if (l.PPS > 0) {
-    // 1. the retained INT4-region rows of every (sequence, head) into compact pages
-    GatherParams g{};
-    g.mask = retain_mask;
-    g.seq_lens = seq_lens;
-    g.page_table = page_table;
-    g.pool = cache->pool;
-    g.head_bytes = page_head_bytes(D);
-    g.page_bytes = g.head_bytes * Hkv;
-    g.B = B;
-    g.Hkv = Hkv;
-    g.sink = cache->cfg.sink;
-    g.recent = cache->cfg.recent;
-    g.num_pages = cache->cfg.num_pages;
-    g.pt_stride = pt_stride;
-    g.mask_stride = mask_stride;
-    g.max_retained = max_retained;
-    g.PPS = l.PPS;
-    g.words = l.words;
-    g.wpre = reinterpret_cast<int *>(w + l.wpre);
-    g.counts = reinterpret_cast<int *>(w + l.counts);
-    g.lens_c = lens_c;
-    g.pt_c = reinterpret_cast<int *>(w + l.pt);
-    g.mask_c = reinterpret_cast<uint32_t *>(w + l.mask);
-    g.mask_stride_c = l.MSC;
-    g.pool_c = w + l.pool;
-    g.err = cache->err;
-    if (bad(launch_masked_gather(g, D, s))) return KV4_ERR_CUDA;
-    // 2. the compact pages: INT4 only (no sink, no recent window), each head's
-    //    first count rows valid
-    kv4_cache cv = *cache;
-    cv.cfg.sink = 0;
-    cv.cfg.recent = 0;
-    cv.cfg.num_pages = B * l.PPS;
-    cv.pool = g.pool_c;
-    cv.pool_bytes = (size_t)B * l.PPS * g.page_bytes;
-    cv.side = nullptr;
-    cv.side_bytes = 0;
-    const kv4_status s1 = decode_call(&cv, stream, q, Hq, lens_c, g.pt_c, l.PPS, nullptr, nullptr, 0, g.mask_c,
-                                      l.MSC, softmax_scale, 0, w, dec_bytes, nullptr, 0, parts, B);
-    if (s1 != KV4_OK) return s1;
-    ++nparts;
-  }
+  if (bad(cudaMemsetAsync(zeros, 0, (size_t)B * 4, s))) return KV4_ERR_CUDA;
+  // 1. retained INT4-region rows per (sequence, head), and prefix counts per mask word
+  GatherParams g{};
+  g.mask = retain_mask;
+  g.seq_lens = seq_lens;
+  g.B = B;
+  g.Hkv = Hkv;
+  g.sink = cache->cfg.sink;
+  g.recent = cache->cfg.recent;
+  g.pt_stride = pt_stride;
+  g.mask_stride = mask_stride;
+  g.max_retained = max_retained;
+  g.words = l.words;
+  g.wpre = reinterpret_cast<int *>(w + l.wpre);
+  g.counts = reinterpret_cast<int *>(w + l.counts);
+  g.err = cache->err;
+  if (bad(launch_masked_count(g, s))) return KV4_ERR_CUDA;
+  // 2. the retained rows gathered on chip and attended, one partial per warp
+  DecodeParams dp{};
+  dp.B = B;
+  dp.Hq = Hq;
+  dp.Hkv = Hkv;
+  dp.G = G;
+  dp.sink = cache->cfg.sink;
+  dp.recent = cache->cfg.recent;
+  dp.num_pages = cache->cfg.num_pages;
+  dp.pt_stride = pt_stride;
+  dp.q = static_cast<const __nv_bfloat16 *>(q);
+  dp.seq_lens = seq_lens;
+  dp.page_table = page_table;
+  dp.pool = cache->pool;
+  dp.head_bytes = page_head_bytes(D);
+  dp.page_bytes = dp.head_bytes * Hkv;
+  dp.scale_log2 = softmax_scale * 1.4426950408889634f;
+  dp.err = cache->err;
+  if (bad(launch_masked_decode(dp, g, parts, D, s))) return KV4_ERR_CUDA;
+  int nparts = l.nparts - 1;
   // 3. the INT8 sink and recent positions from the side cache (no INT4 pages)
   if (cache->cfg.sink + cache->cfg.recent > 0) {
     const kv4_status s2 = decode_call(cache, stream, q, Hq, seq_lens, page_table, pt_stride, zeros, zeros, 1,
@@ -611,7 +593,7 @@ kv4_status kv4_decode_attn_masked(kv4_cache *cache, void *stream, const void *q,
     if (s2 != KV4_OK) return s2;
     ++nparts;
   }
-  // 4. the exact merge of the two partials
+  // 4. the exact merge of the partials
   return cuda_status(launch_merge_partials(parts, nparts, (long long)B * Hq, D, out, out_is_fp32 ? 1 : 0, s));
 }
 

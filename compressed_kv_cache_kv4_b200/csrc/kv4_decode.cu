@@ -921,6 +921,188 @@ __global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
 }
 
 // ---------------------------------------------------------------------------
+// Masked decode with the retained rows gathered on chip (Shadow Mask
+// Distillation, sec. 1 and Figure 1: the mask is applied inside attention).
+// One CTA per (sequence, KV head). Its retained INT4-region positions, in
+// order, form "compact pages" of 16 rows; a warp at a time gathers one compact
+// page of the head into a shared-memory image of the ordinary head-block
+// layout (lanes i and i + 16 load the two halves of row i: K codes, the K or V
+// scales, and the 16-byte pieces of the V block that hold the row's bytes;
+// the V bytes are moved to the row's place in the fragment order) and runs
+// the ordinary page computation on it. Rows past the count are zero and not
+// attended. Reads and work follow the retained count; nothing is written back
+// but one (m, l, o) partial per warp, in the layout of kv4_decode_partials.
+// ---------------------------------------------------------------------------
+constexpr int kMaskedWarps = 4, kMaskedChunk = 4096;
+
+__device__ __forceinline__ uint32_t word_bits_in(int w, int c0, int c1) {
+  const int a = max(c0 - 32 * w, 0), z = min(c1 - 32 * w, 32);
+  if (z <= a) return 0u;
+  return (z >= 32 ? 0xFFFFFFFFu : ((1u << z) - 1u)) & ~((1u << a) - 1u);
+}
+
+// The partial of a warp's softmax state for query heads h*G .. h*G+G-1 in the
+// layout of kv4_decode_partials: m (log2 units), l, two unused words, o.
+template <int D, int NMT>
+__device__ __forceinline__ void write_cp_partial(int G, SoftmaxState<NMT> &st, float *pr, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    st.l[0] += __shfl_xor_sync(0xffffffffu, st.l[0], o);
+    st.l[1] += __shfl_xor_sync(0xffffffffu, st.l[1], o);
+  }
+#pragma unroll
+  for (int mt = 0; mt < NMT; ++mt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) st.o[mt][c] += __shfl_xor_sync(0xffffffffu, st.o[mt][c], 2);
+  if (t < 2) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int head = 2 * t + c;
+      if (head < G) {
+        const bool nonempty = st.l[c] > 0.f;
+        const float inv = nonempty ? 1.f / st.l[c] : 0.f;
+        float *ph = pr + head * (D + 4);
+#pragma unroll
+        for (int mt = 0; mt < NMT; ++mt) {
+          ph[4 + 16 * mt + g] = st.o[mt][c] * inv;
+          ph[4 + 16 * mt + g + 8] = st.o[mt][c + 2] * inv;
+        }
+        if (g == 0) {
+          ph[0] = nonempty ? st.m[c] : -INFINITY;
+          ph[1] = st.l[c];
+          ph[2] = 0.f;
+          ph[3] = 0.f;
+        }
+      }
+    }
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(DecodeParams p, GatherParams gp,
+                                                                             float *parts) {
+  constexpr int NMT = D / 16, HEAD = 18 * D, KROW = D / 2, NP = D / 16, QB = kv4_q_bytes(D);
+  extern __shared__ __align__(128) uint8_t msm[];
+  int *list = reinterpret_cast<int *>(msm);                 // [kMaskedChunk]
+  uint8_t *qarea = msm + 4 * kMaskedChunk;                 // [QB], shared by the warps
+  uint8_t *img_all = qarea + QB;                           // [kMaskedWarps][HEAD]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NT = kMaskedWarps * 32;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int row = blockIdx.x, b = row / p.Hkv, h = row - b * p.Hkv;
+  const int cap = p.pt_stride * kPageTokens;
+  int L = p.seq_lens[b];
+  L = L < 0 ? 0 : (L > cap ? cap : L);
+  const int c0 = min(p.sink, L), c1 = max(c0, L - p.recent);
+  const int n = gp.counts[row];
+  const int npg = (n + kPageTokens - 1) / kPageTokens;
+  const uint32_t *mrow = gp.mask + (long long)row * gp.mask_stride;
+  const int *wpre = gp.wpre + (long long)row * gp.words;
+  const int nw = (L + 31) / 32;
+  uint8_t *im = img_all + warp * HEAD;
+  if (warp == 0) load_q<D, G>(p, b, h, true, qarea, lane);
+  SoftmaxState<NMT> st;
+  st.reset();
+  RangeCtx rc{};
+  rc.b = b;
+  rc.h = h;
+  rc.L = n;
+  rc.lo_tok = 0;
+  rc.hi_tok = n;   // rows of compact page j are retained indices 16 j .. 16 j + 15
+  rc.mrow = nullptr;
+  const uint32_t im_u32 = smem_u32(im), q_u32 = smem_u32(qarea);
+  const int i = lane & 15, half = lane >> 4;
+  for (int t0 = 0; t0 < npg * kPageTokens; t0 += kMaskedChunk) {
+    const int t1 = min(t0 + kMaskedChunk, n);
+    __syncthreads();   // the query is in place; the previous chunk's list is no longer read
+    for (int w = tid; w < nw; w += NT) {
+      const int hi_ = wpre[w], lo_ = w > 0 ? wpre[w - 1] : 0;   // retained indices [lo_, hi_) lie in word w
+      if (hi_ <= t0 || lo_ >= t1) continue;
+      uint32_t bits = mrow[w] & word_bits_in(w, c0, c1);
+      for (int k = lo_; bits; ++k) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (k >= t0 && k < t1) list[k - t0] = 32 * w + bit;
+      }
+    }
+    __syncthreads();
+    const int pg_end = min(npg, (t0 + kMaskedChunk) / kPageTokens);
+    for (int j = t0 / kPageTokens + warp; j < pg_end; j += kMaskedWarps) {
+      for (int q = lane; q < HEAD / 16; q += 32) reinterpret_cast<uint4 *>(im)[q] = make_uint4(0, 0, 0, 0);
+      const int t = kPageTokens * j + i;
+      int page = -1, r = 0;
+      if (t < n) {
+        const int pos = list[t - t0];
+        r = pos % kPageTokens;
+        page = p.page_table[(long long)b * p.pt_stride + pos / kPageTokens];
+        if (page < 0 || page >= p.num_pages) {
+          if (half == 0) set_error(p.err, kErrBounds);
+          page = -1;   // the row stays zero
+        }
+      }
+      __syncwarp();
+      if (page >= 0) {
+        const uint8_t *src = p.pool + (long long)page * p.page_bytes + (long long)h * p.head_bytes;
+        uint4 kc[D / 64];
+#pragma unroll
+        for (int u = 0; u < D / 64; ++u)
+          kc[u] = __ldg(reinterpret_cast<const uint4 *>(src + r * KROW + half * (KROW / 2)) + u);
+        const int sb = half ? 17 * D : 16 * D;   // K scales (half 0) or V scales (half 1)
+        uint2 sc = make_uint2(0, 0);
+        if constexpr (D == 128) sc = __ldg(reinterpret_cast<const uint2 *>(src + sb + r * (D / 16)));
+        else sc.x = __ldg(reinterpret_cast<const uint32_t *>(src + sb + r * (D / 16)));
+        // V: word (m/4)*128 + 4*(4*dm8 + (r%8)/2) + m%4 holds the row's byte
+        // 2*(r%2) + r/8; a 16-byte piece (m/4, dm8) has four of the row's bytes
+        uint4 vp[NP];
+#pragma unroll
+        for (int u = 0; u < NP; ++u) {
+          const int m4 = D == 128 ? half : 0, dm8 = D == 128 ? u : 4 * half + u;
+          vp[u] = __ldg(reinterpret_cast<const uint4 *>(src + 8 * D + 16 * (m4 * 32 + 4 * dm8 + (r % 8) / 2)));
+        }
+#pragma unroll
+        for (int u = 0; u < D / 64; ++u) reinterpret_cast<uint4 *>(im + i * KROW + half * (KROW / 2))[u] = kc[u];
+        if constexpr (D == 128) *reinterpret_cast<uint2 *>(im + sb + i * (D / 16)) = sc;
+        else *reinterpret_cast<uint32_t *>(im + sb + i * (D / 16)) = sc.x;
+        const int sh_src = 8 * (2 * (r % 2) + r / 8), b_dst = 2 * (i % 2) + i / 8;
+#pragma unroll
+        for (int u = 0; u < NP; ++u) {
+          const int m4 = D == 128 ? half : 0, dm8 = D == 128 ? u : 4 * half + u;
+          uint8_t *dst = im + 8 * D + 16 * (m4 * 32 + 4 * dm8 + (i % 8) / 2) + b_dst;
+          dst[0] = static_cast<uint8_t>(vp[u].x >> sh_src);
+          dst[4] = static_cast<uint8_t>(vp[u].y >> sh_src);
+          dst[8] = static_cast<uint8_t>(vp[u].z >> sh_src);
+          dst[12] = static_cast<uint8_t>(vp[u].w >> sh_src);
+        }
+      }
+      __syncwarp();
+      int4_item<D, G>(p, im_u32, q_u32, j, rc, st, lane);
+      __syncwarp();
+    }
+  }
+  write_cp_partial<D, NMT>(G, st, parts + (((long long)warp * p.B + b) * p.Hq + h * G) * (D + 4), lane);
+}
+
+size_t masked_decode_smem(int D) { return 4 * kMaskedChunk + kv4_q_bytes(D) + (size_t)kMaskedWarps * 18 * D; }
+
+template <int D>
+static cudaError_t launch_masked_d(const DecodeParams &p, const GatherParams &g, float *parts, cudaStream_t s) {
+  const size_t smem = masked_decode_smem(D);
+  auto kern = p.G == 1 ? masked_decode_kernel<D, 1> : (p.G == 2 ? masked_decode_kernel<D, 2> : masked_decode_kernel<D, 4>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(p.B * p.Hkv), dim3(kMaskedWarps * 32), smem, s, p, g, parts);
+}
+
+cudaError_t launch_masked_decode(const DecodeParams &p, const GatherParams &g, float *parts, int D, cudaStream_t s) {
+  if (p.B * p.Hkv == 0) return cudaSuccess;
+  return D == 128 ? launch_masked_d<128>(p, g, parts, s) : launch_masked_d<64>(p, g, parts, s);
+}
+
+int masked_decode_warps() { return kMaskedWarps; }
+
+// ---------------------------------------------------------------------------
 // bf16 pages of one piece (the uncompressed comparison).
 // Head block in a page: K[16][D] bf16 then V[16][D] bf16. Each row is copied
 // to a padded shared-memory row so ldmatrix reads are conflict-free.

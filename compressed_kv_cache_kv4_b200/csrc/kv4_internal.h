@@ -113,27 +113,25 @@ cudaError_t launch_decode(const DecodeParams &p, int D, bool bf16, cudaStream_t 
                           cudaEvent_t ev1);
 cudaError_t launch_topk(const TopkParams &p, cudaStream_t stream);
 
-// Gather of the retained INT4-region rows into compact pages (kv4_masked.cu).
+// Masked decode with the retained rows gathered on chip (kv4_masked.cu counts,
+// kv4_decode.cu gathers and attends).
 struct GatherParams {
   const uint32_t *mask;         // [B][Hkv][mask_stride]
   const int32_t *seq_lens;      // [B]
-  const int32_t *page_table;    // [B][pt_stride]
-  const uint8_t *pool;
-  long long page_bytes, head_bytes;
-  int B, Hkv, sink, recent, num_pages, pt_stride, mask_stride;
-  int max_retained;             // rows kept per (sequence, head), at most
-  int PPS;                      // compact pages per sequence: ceil(max_retained / 16)
+  int B, Hkv, sink, recent, pt_stride, mask_stride;
+  int max_retained;             // rows attended per (sequence, head), at most
   int words;                    // prefix entries per row: ceil(pt_stride * 16 / 32)
   int *wpre;                    // [B][Hkv][words] inclusive retained counts per mask word
   int *counts;                  // [B][Hkv]
-  int *lens_c;                  // [B] compact length (max over heads); zero before the call
-  int *pt_c;                    // [B][PPS] compact page table
-  uint32_t *mask_c;             // [B][Hkv][mask_stride_c] valid compact rows
-  int mask_stride_c;
-  uint8_t *pool_c;              // [B * PPS] compact pages
   uint32_t *err;
 };
-cudaError_t launch_masked_gather(const GatherParams &p, int D, cudaStream_t stream);
+// Counts and per-word prefix counts of the retained INT4-region rows.
+cudaError_t launch_masked_count(const GatherParams &p, cudaStream_t stream);
+// Gathered masked decode of the INT4 region: one partial per warp into
+// parts [masked_decode_warps()][B][Hq][D+4] (the layout of kv4_decode_partials).
+cudaError_t launch_masked_decode(const DecodeParams &p, const GatherParams &g, float *parts, int D,
+                                 cudaStream_t stream);
+int masked_decode_warps();
 // Exact merge of the decode partials of kv4_decode_kernel or bf16_decode_kernel.
 cudaError_t launch_merge(const DecodeParams &p, int D, bool bf16, cudaStream_t stream);
 // Exact merge of N gathered (m, l, o) partials [N][rows][D+4] into out [rows][D].

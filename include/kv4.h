@@ -212,24 +212,27 @@ kv4_status kv4_decode_partials(kv4_cache *cache, void *stream, const void *q, in
  * is a binary mask applied inside attention instead of slicing the cache;
  * KV4-RL review, sec. 3: the INT4 and INT8 regions are attended separately
  * and merged exactly.
- * The retained INT4-region positions of every (sequence, KV head) are gathered,
- * in position order, into dense pages of the ordinary layout in the workspace
- * (K rows and scales whole; V rows from the 4-row groups that hold them), the
- * ordinary decode attends those pages, the INT8 region is attended from the
- * side cache under the same mask, and the two partials are merged. The result
- * is the same attention as kv4_decode_attn with retain_mask (within rounding).
+ * The retained INT4-region positions of every (sequence, KV head), in position
+ * order, are gathered 16 at a time into a page image in shared memory (K rows
+ * and scales whole; a V row's bytes from the 16-byte pieces of the V block
+ * that hold them) and attended there, so only the retained rows' K codes and
+ * scales and the V pieces of their 4-row groups are read, and the work is
+ * proportional to the retained rows. The INT8 region is attended from the side
+ * cache under the same mask, and the partials are merged. The result is the
+ * same attention as kv4_decode_attn with retain_mask (within rounding).
+ * Each (sequence, head) is gathered by one CTA, page after page, so the call
+ * gains on sparse masks (an H2O-style 10% budget: 0.45x the unmasked decode
+ * time on the eviction workload) and loses on dense ones (beyond about a third
+ * of the positions, kv4_decode_attn with retain_mask is faster).
  *  retain_mask: device uint32 [B][Hkv][mask_stride], required; mask_stride *
  *    32 >= pt_stride * 16.
- *  max_retained: host bound on the retained positions of the INT4 region
- *    [sink, L - recent) of any (sequence, head); it sizes the workspace
- *    (ceil(max_retained / 16) pages per sequence). For a kv_topk_retain mask
- *    with budget k = floor(L * permille / 1000) it is at most k. A row with more
- *    sets KV4_ERR_CAPACITY and only its first max_retained positions are
- *    attended.
+ *  max_retained: bound on the retained INT4-region positions [sink, L - recent)
+ *    of any (sequence, head). A row with more sets KV4_ERR_CAPACITY and only
+ *    its first max_retained positions are attended.
  *  workspace: device, >= kv4_masked_workspace_bytes(), 256-byte aligned.
- * Other arguments as kv4_decode_attn (the default worker count is used).
- * Launches: a count kernel, a gather kernel, two decode worker + merge pairs
- * and a partial merge, all on `stream`.
+ * Other arguments as kv4_decode_attn (the default worker count is used for the
+ * INT8 region). Launches on `stream`: a count kernel, the gathering kernel, an
+ * INT8-region worker and merge pair, and a partial merge.
  */
 kv4_status kv4_masked_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t Hq, int32_t pt_stride,
                                       int32_t max_retained, size_t *bytes);
