@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(256, 3) append_pages_kernel(AppendParams p) {
           const int m = 2 * i + hh, tt = (r % 8) / 2;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int word = (m / 4) * 128 + (4 * e + tt) * 4 + (m % 4);
+            const int word = (m / 4) * 128 + (8 * tt + (e ^ (2 * tt))) * 4 + (m % 4);
             const uint32_t byte = (__float_as_uint(fmaf(c[e + 8], 16.f, c[e] + 136.f) + 8388608.f) & 0xFFu) ^ 0x88u;
             im[8 * D + 4 * word + 2 * (r % 2) + r / 8] = static_cast<uint8_t>(byte);
           }
@@ -379,7 +379,7 @@ __device__ __forceinline__ void append_row(const AppendParams &p, long long j, i
         for (int e = 0; e < EPL; ++e) {
           const int d = d0 + e;
           const int m = d / 16, g = d % 8, tt = (r % 8) / 2;
-          const int word = (m / 4) * 128 + (4 * g + tt) * 4 + (m % 4);
+          const int word = (m / 4) * 128 + (8 * tt + (g ^ (2 * tt))) * 4 + (m % 4);
           blk[8 * D + 4 * word + 2 * (r % 2) + r / 8] = static_cast<uint8_t>(nib(c[e]) | nib(partner[e]) << 4);
         }
       }

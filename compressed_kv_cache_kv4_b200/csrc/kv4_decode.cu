@@ -644,9 +644,11 @@ __device__ __forceinline__ void int4_item(const DecodeParams &p, uint32_t stg, u
                   __fmul2_rn(make_float2(pr[2], pr[3]), make_float2(vs1, vs1)), neg_sel, wb[i][0], wb[i][1]);
   }
   uint32_t vw[NMT];
+  // lane (g, t) = 4 g + t keeps its V words at position 8 t + (g ^ 2 t)
+  const int vpos = 8 * t + (g ^ (2 * t));
 #pragma unroll
   for (int q4 = 0; q4 < NMT / 4; ++q4) {
-    const uint4 w = lds128(stg + 8 * D + q4 * 512 + lane * 16);
+    const uint4 w = lds128(stg + 8 * D + q4 * 512 + vpos * 16);
     vw[4 * q4 + 0] = w.x;
     vw[4 * q4 + 1] = w.y;
     vw[4 * q4 + 2] = w.z;
@@ -1053,13 +1055,16 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
         uint2 sc = make_uint2(0, 0);
         if constexpr (D == 128) sc = __ldg(reinterpret_cast<const uint2 *>(src + sb + r * (D / 16)));
         else sc.x = __ldg(reinterpret_cast<const uint32_t *>(src + sb + r * (D / 16)));
-        // V: word (m/4)*128 + 4*(4*dm8 + (r%8)/2) + m%4 holds the row's byte
-        // 2*(r%2) + r/8; a 16-byte piece (m/4, dm8) has four of the row's bytes
+        // V: word (m/4)*128 + 4*P + m%4 with P = 8*tt + (dm8 ^ 2*tt), tt =
+        // (r%8)/2, holds the row's byte 2*(r%2) + r/8; a 16-byte piece (m/4,
+        // dm8) has four of the row's bytes, and the pieces of the row's 4-row
+        // group are 128 contiguous bytes of each 512-byte block
+        const int tts = (r % 8) / 2, ttd = (i % 8) / 2;
         uint4 vp[NP];
 #pragma unroll
         for (int u = 0; u < NP; ++u) {
           const int m4 = D == 128 ? half : 0, dm8 = D == 128 ? u : 4 * half + u;
-          vp[u] = __ldg(reinterpret_cast<const uint4 *>(src + 8 * D + 16 * (m4 * 32 + 4 * dm8 + (r % 8) / 2)));
+          vp[u] = __ldg(reinterpret_cast<const uint4 *>(src + 8 * D + 16 * (m4 * 32 + 8 * tts + (dm8 ^ (2 * tts)))));
         }
 #pragma unroll
         for (int u = 0; u < D / 64; ++u) reinterpret_cast<uint4 *>(im + i * KROW + half * (KROW / 2))[u] = kc[u];
@@ -1069,7 +1074,7 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
 #pragma unroll
         for (int u = 0; u < NP; ++u) {
           const int m4 = D == 128 ? half : 0, dm8 = D == 128 ? u : 4 * half + u;
-          uint8_t *dst = im + 8 * D + 16 * (m4 * 32 + 4 * dm8 + (i % 8) / 2) + b_dst;
+          uint8_t *dst = im + 8 * D + 16 * (m4 * 32 + 8 * ttd + (dm8 ^ (2 * ttd))) + b_dst;
           dst[0] = static_cast<uint8_t>(vp[u].x >> sh_src);
           dst[4] = static_cast<uint8_t>(vp[u].y >> sh_src);
           dst[8] = static_cast<uint8_t>(vp[u].z >> sh_src);

@@ -118,9 +118,11 @@ int kv4o_quant_int8(const uint16_t *x_bf16, int n, uint16_t *scale_bits, int8_t 
 /*   t*D/8, word i (i = d/32) at 4*i inside the chunk, element k = d%8  */
 /*   in nibble k of that 32-bit word (little-endian byte k/2, low nibble */
 /*   for even k).                                                       */
-/* V codes: 32 "lanes" (g, t) with g = d%8 and t = (r%8)/2, lane = 4g+t; */
-/*   m = d/16; 32-bit word (lane, m) at 4*((m/4)*128 + lane*4 + m%4);   */
-/*   inside the word byte 2*(r%2) + r/8, nibble (d%16)/8.               */
+/* V codes: 32 "lanes" (g, t) with g = d%8 and t = (r%8)/2, stored at  */
+/*   position P = 8t + (g XOR 2t), so the four rows {2t, 2t+1, 2t+8,    */
+/*   2t+9} own 128 contiguous bytes of each 512-byte block; m = d/16;   */
+/*   32-bit word (lane, m) at 4*((m/4)*128 + P*4 + m%4); inside the     */
+/*   word byte 2*(r%2) + r/8, nibble (d%16)/8.                          */
 /* Scales: fp16, row r group i at 2*(r*D/32 + i).                       */
 /* ------------------------------------------------------------------ */
 
@@ -135,8 +137,8 @@ int64_t kv4o_k_code_byte(int D, int r, int d, int *nibble) {
 int64_t kv4o_v_code_byte(int D, int r, int d, int *nibble) {
   int m = d / 16, g = d % 8, hi8 = (d % 16) / 8;
   int t = (r % 8) / 2, rodd = r % 2, r8 = r / 8;
-  int lane = 4 * g + t;
-  int64_t word = (int64_t)(m / 4) * 128 + lane * 4 + (m % 4);
+  int pos = 8 * t + (g ^ (2 * t));
+  int64_t word = (int64_t)(m / 4) * 128 + pos * 4 + (m % 4);
   *nibble = hi8;
   return 8LL * D + 4 * word + 2 * rodd + r8;
 }

@@ -21,12 +21,15 @@ def test_hand_computed_offsets():
     assert O.k_code_byte(128, 5, 37) == (326, 1)
     # K, slot 15, dim 127: i=3, t=3, k=7 -> 15*64 + 3*16 + 12 + 3 = 1023, high nibble
     assert O.k_code_byte(128, 15, 127) == (1023, 1)
-    # V, slot 5, dim 37: m=2, g=5, upper-8 flag 0; t=2, odd slot, first half -> lane 22,
-    # word 22*4 + 2 = 90 -> byte 1024 + 360 + 2 = 1386, low nibble
-    assert O.v_code_byte(128, 5, 37) == (1386, 0)
+    # V, slot 5, dim 37: m=2, g=5, upper-8 flag 0; t=2, odd slot, first half -> lane 22 at
+    # position 8*2 + (5 xor 4) = 17, word 17*4 + 2 = 70 -> byte 1024 + 280 + 2 = 1306, low nibble
+    assert O.v_code_byte(128, 5, 37) == (1306, 0)
     # V, slot 9, dim 120: m=7 (second 512-byte half), g=0, upper-8 flag 1; t=0, odd, r8=1
-    # -> lane 0, word 128 + 0 + 3 = 131 -> byte 1024 + 524 + 2 + 1 = 1551, high nibble
+    # -> position 0, word 128 + 0 + 3 = 131 -> byte 1024 + 524 + 2 + 1 = 1551, high nibble
     assert O.v_code_byte(128, 9, 120) == (1551, 1)
+    # V, slot 14, dim 3: m=0, g=3, t=3, even slot, r8=1 -> position 24 + (3 xor 6) = 29,
+    # word 116 -> byte 1024 + 464 + 1 = 1489, low nibble
+    assert O.v_code_byte(128, 14, 3) == (1489, 0)
     # scales: slot r, group i at 2*(4r + i) after the codes
     assert O.k_scale_byte(128, 3, 2) == 2048 + 28
     assert O.v_scale_byte(128, 3, 2) == 2176 + 28
@@ -61,6 +64,16 @@ def test_side_layout_is_a_bijection():
         assert seen == set(range(pb))
 
 
+def test_v_rows_of_a_group_are_contiguous():
+    """The V codes of the rows {2a, 2a+1, 2a+8, 2a+9} fill 128 contiguous bytes of
+    each 512-byte block of the V area, so they can be read without the other rows."""
+    for D in (64, 128):
+        for a in range(4):
+            got = {O.v_code_byte(D, r, d)[0] for r in (2 * a, 2 * a + 1, 2 * a + 8, 2 * a + 9) for d in range(D)}
+            want = {8 * D + 512 * blk + 128 * a + k for blk in range(D // 64) for k in range(128)}
+            assert got == want, (D, a)
+
+
 def test_layout_is_a_bijection():
     for D in (64, 128):
         seen = set()
@@ -86,7 +99,8 @@ def _decode_block_via_fragments(blk, D):
     kw = words[: 2 * D].reshape(16, 4, D // 32)
     kn = _nibbles(kw)                               # [16][t][i][k]
     K = kn.transpose(0, 2, 1, 3).reshape(16, D)     # [row][i][t][k] -> dim
-    # V: word (lane, m) at (m//4)*128 + lane*4 + m%4, lane = 4g + t; nibbles
+    # V: word (lane, m) at (m//4)*128 + P*4 + m%4, lane = 4g + t stored at
+    # position P = 8t + (g xor 2t); nibbles
     # n0 (2t, 16m+g) n1 (2t, 16m+g+8) n2 (2t+8, g) n3 (2t+8, g+8) n4 (2t+1, g)
     # n5 (2t+1, g+8) n6 (2t+9, g) n7 (2t+9, g+8) -- the A fragment of V^T
     vw = words[2 * D: 4 * D]
@@ -94,7 +108,7 @@ def _decode_block_via_fragments(blk, D):
     for lane in range(32):
         g, t = lane // 4, lane % 4
         for m in range(D // 16):
-            n = _nibbles(vw[(m // 4) * 128 + lane * 4 + m % 4])
+            n = _nibbles(vw[(m // 4) * 128 + (8 * t + (g ^ (2 * t))) * 4 + m % 4])
             for j, (tok, dd) in enumerate([(2 * t, g), (2 * t, g + 8), (2 * t + 8, g), (2 * t + 8, g + 8),
                                            (2 * t + 1, g), (2 * t + 1, g + 8), (2 * t + 9, g), (2 * t + 9, g + 8)]):
                 V[tok, 16 * m + dd] = n[j]
