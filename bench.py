@@ -57,6 +57,9 @@ def parse():
                     help="time only smd_masked_attn on the learner workload and print its figures")
     ap.add_argument("--topk-only", action="store_true",
                     help="print only kv_topk_retain on the evict workload at a 10%% budget (the ncu capture's command)")
+    ap.add_argument("--masked-only", action="store_true",
+                    help="print only the masked decode paths on the evict workload at a 10%% budget "
+                         "(the ncu capture's command)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="print only the prefill append of the qwen8b prompt (the ncu capture's command)")
     ap.add_argument("--sink", type=int, default=None, help="override the INT8 sink size (0 = pure INT4)")
@@ -681,6 +684,35 @@ def topk_only(permille=100, reps=20):
             "gbs": nbytes / (med / 1e3) / 1e9, "retained": int(count.sum().item())}
 
 
+def masked_only(permille=100, reps=20):
+    """Masked decode on the evict workload under a kv_topk_retain mask: the page
+    path (kv4_decode_attn with the mask) and the gathered path
+    (kv4_decode_attn_masked), each call timed with CUDA events."""
+    import compressed_kv_cache_kv4_b200 as K
+    from compressed_kv_cache_kv4_b200 import synth
+    wl = synth.workload("evict")
+    cache, ptd, _, _ = build_kv4(wl, wl.lens, 0, 0)
+    k, v, off = prefill(cache, wl, wl.lens, ptd)
+    scores = synth.gen_scores(wl, k, off, device="cuda")
+    del k, v
+    q = synth.gen_q(wl, device="cuda")
+    lens = torch.as_tensor(wl.lens, device="cuda")
+    L = int(wl.lens.max())
+    mask = torch.zeros((wl.B, wl.Hkv, (ptd.shape[1] * 16 + 31) // 32), dtype=torch.int32, device="cuda")
+    K.kv_topk_retain(scores, lens, permille, mask, None, max_len=L)
+    o = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device="cuda")
+    ws = cache.workspace(wl.B, wl.Hq)
+    page, _ = time_calls(lambda: K.kv4_decode_attn(cache.handle, q, lens, ptd, wl.softmax_scale, ws, o,
+                                                   retain_mask=mask), reps)
+    gath, _ = time_calls(lambda: cache.decode_masked(q, lens, ptd, wl.softmax_scale, mask, L * permille // 1000,
+                                                     out=o), reps)
+    unm, _ = time_calls(lambda: K.kv4_decode_attn(cache.handle, q, lens, ptd, wl.softmax_scale, ws, o), reps)
+    st = cache.get_error()[0]
+    cache.close()
+    return {"permille": permille, "page_path_us": page * 1e3, "gathered_us": gath * 1e3, "unmasked_us": unm * 1e3,
+            "device_error": st}
+
+
 def prefill_only(reps=20):
     """The prefill append of the qwen8b prompt (lengths L0 - 64) alone."""
     from compressed_kv_cache_kv4_b200 import synth
@@ -1069,6 +1101,10 @@ def main():
     if args.prefill_only:
         if rank == 0:
             print(json.dumps(prefill_only()), flush=True)
+        return
+    if args.masked_only:
+        if rank == 0:
+            print(json.dumps(masked_only()), flush=True)
         return
     wl, res = run_kv4(args, ws, rank)
     if rank == 0:
