@@ -471,25 +471,22 @@ kv4_status kv4_decode_partials(kv4_cache *cache, void *stream, const void *q, in
 
 namespace {
 
-// Workspace of kv4_decode_attn_masked: the ordinary decode workspace (for the
-// INT8 region), then counts [B*Hkv] | B zeros (empty page ranges) | word prefix
-// counts [B*Hkv*words] | partials [W+1][B][Hq][D+4] (one per warp of the
-// gathering kernel, then the INT8 region's).
+// Workspace of kv4_decode_attn_masked: counts [B*Hkv] | word prefix counts
+// [B*Hkv*words] | partials [W][B][Hq][D+4] (one per warp of the gathering
+// kernel).
 struct MaskedLayout {
-  size_t counts, lens, wpre, parts, total;
+  size_t counts, wpre, parts, total;
   int words, nparts;
 };
 
-MaskedLayout masked_layout(const kv4_cache *cache, const Kv4Plan &pl, int B, int Hq, int pt_stride) {
-  const int D = cache->cfg.head_dim, Hkv = cache->cfg.num_kv_heads, G = Hq / Hkv;
+MaskedLayout masked_layout(const kv4_cache *cache, int B, int Hq, int pt_stride) {
+  const int D = cache->cfg.head_dim, Hkv = cache->cfg.num_kv_heads;
   MaskedLayout l{};
   l.words = (pt_stride * kPageTokens + 31) / 32;
-  l.nparts = masked_decode_warps() + 1;
-  size_t o = round_up(kv4_ws_bytes(pl, G, D), kAlign);
+  l.nparts = masked_decode_warps();
+  size_t o = 0;
   l.counts = o;
   o += round_up((size_t)B * Hkv * 4, kAlign);
-  l.lens = o;
-  o += round_up((size_t)B * 4, kAlign);
   l.wpre = o;
   o += round_up((size_t)B * Hkv * l.words * 4, kAlign);
   l.parts = o;
@@ -519,7 +516,7 @@ kv4_status kv4_masked_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t
   Kv4Plan pl{};
   const kv4_status st = masked_check(cache, B, Hq, pt_stride, max_retained, &pl);
   if (st != KV4_OK) return st;
-  *bytes = masked_layout(cache, pl, B, Hq, pt_stride).total;
+  *bytes = masked_layout(cache, B, Hq, pt_stride).total;
   return KV4_OK;
 }
 
@@ -539,16 +536,12 @@ kv4_status kv4_decode_attn_masked(kv4_cache *cache, void *stream, const void *q,
   int dev = -1;
   if (bad(cudaGetDevice(&dev))) return KV4_ERR_CUDA;
   if (dev != cache->device) return KV4_ERR_INVALID;
-  const MaskedLayout l = masked_layout(cache, pl, B, Hq, pt_stride);
+  const MaskedLayout l = masked_layout(cache, B, Hq, pt_stride);
   if (ws_bytes < l.total) return KV4_ERR_INVALID;
   const int D = cache->cfg.head_dim, Hkv = cache->cfg.num_kv_heads, G = Hq / Hkv;
   uint8_t *w = static_cast<uint8_t *>(workspace);
-  const size_t dec_bytes = kv4_ws_bytes(pl, G, D);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int *zeros = reinterpret_cast<int *>(w + l.lens);
   float *parts = reinterpret_cast<float *>(w + l.parts);
-  const long long part_floats = (long long)B * Hq * (D + 4);
-  if (bad(cudaMemsetAsync(zeros, 0, (size_t)B * 4, s))) return KV4_ERR_CUDA;
   // 1. retained INT4-region rows per (sequence, head), and prefix counts per mask word
   GatherParams g{};
   g.mask = retain_mask;
@@ -583,18 +576,13 @@ kv4_status kv4_decode_attn_masked(kv4_cache *cache, void *stream, const void *q,
   dp.page_bytes = dp.head_bytes * Hkv;
   dp.scale_log2 = softmax_scale * 1.4426950408889634f;
   dp.err = cache->err;
+  dp.side = cache->side;
+  dp.side_stride = side_head_bytes(D, dp.sink, dp.recent);
+  dp.np8 = side_pages(dp.sink, dp.recent);
+  dp.int8_units = dp.sink + dp.recent > 0 ? 1 : 0;
   if (bad(launch_masked_decode(dp, g, parts, D, s))) return KV4_ERR_CUDA;
-  int nparts = l.nparts - 1;
-  // 3. the INT8 sink and recent positions from the side cache (no INT4 pages)
-  if (cache->cfg.sink + cache->cfg.recent > 0) {
-    const kv4_status s2 = decode_call(cache, stream, q, Hq, seq_lens, page_table, pt_stride, zeros, zeros, 1,
-                                      retain_mask, mask_stride, softmax_scale, 0, w, dec_bytes, nullptr, 0,
-                                      parts + nparts * part_floats, B);
-    if (s2 != KV4_OK) return s2;
-    ++nparts;
-  }
-  // 4. the exact merge of the partials
-  return cuda_status(launch_merge_partials(parts, nparts, (long long)B * Hq, D, out, out_is_fp32 ? 1 : 0, s));
+  // 3. the exact merge of the warps' partials
+  return cuda_status(launch_merge_partials(parts, l.nparts, (long long)B * Hq, D, out, out_is_fp32 ? 1 : 0, s));
 }
 
 kv4_status kv4_merge_partials(void *stream, const float *partials, int32_t N, int32_t B, int32_t Hq, int32_t D,

@@ -932,8 +932,10 @@ __global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
 // scales, and the 16-byte pieces of the V block that hold the row's bytes;
 // the V bytes are moved to the row's place in the fragment order) and runs
 // the ordinary page computation on it. Rows past the count are zero and not
-// attended. Reads and work follow the retained count; nothing is written back
-// but one (m, l, o) partial per warp, in the layout of kv4_decode_partials.
+// attended. The head's INT8 side pages (sink and recent window, under the
+// same mask) go through the same image and softmax state. Reads and work of
+// the INT4 region follow the retained count; nothing is written back but one
+// (m, l, o) partial per warp, in the layout of kv4_decode_partials.
 // ---------------------------------------------------------------------------
 constexpr int kMaskedWarps = 4, kMaskedChunk = 4096;
 
@@ -987,8 +989,9 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
   constexpr int NMT = D / 16, HEAD = 18 * D, KROW = D / 2, NP = D / 16, QB = kv4_q_bytes(D);
   extern __shared__ __align__(128) uint8_t msm[];
   int *list = reinterpret_cast<int *>(msm);                 // [kMaskedChunk]
-  uint8_t *qarea = msm + 4 * kMaskedChunk;                 // [QB], shared by the warps
-  uint8_t *img_all = qarea + QB;                           // [kMaskedWarps][HEAD]
+  uint8_t *qarea = msm + 4 * kMaskedChunk;                 // [QB] INT4 query format, shared by the warps
+  uint8_t *q8area = qarea + QB;                            // [QB] INT8 query format
+  uint8_t *img_all = q8area + QB;                          // [kMaskedWarps][HEAD]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NT = kMaskedWarps * 32;
   pdl_wait();
@@ -1005,6 +1008,7 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
   const int nw = (L + 31) / 32;
   uint8_t *im = img_all + warp * HEAD;
   if (warp == 0) load_q<D, G>(p, b, h, true, qarea, lane);
+  if (warp == 1 % kMaskedWarps && p.int8_units) load_q<D, G>(p, b, h, false, q8area, lane);
   SoftmaxState<NMT> st;
   st.reset();
   RangeCtx rc{};
@@ -1086,10 +1090,40 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
       __syncwarp();
     }
   }
+  // The INT8 region: this head's side pages, a warp per side page, the K half
+  // and then the V half through the page image, into the same softmax state.
+  if (p.int8_units) {
+    __syncthreads();   // the INT8 query is in place
+    RangeCtx r8{};
+    r8.b = b;
+    r8.h = h;
+    r8.L = L;
+    r8.lo_tok = p.sink;
+    r8.hi_tok = L - p.recent;
+    r8.r0 = max(p.sink, L - p.recent);
+    r8.mrow = mrow;
+    const uint32_t q8_u32 = smem_u32(q8area);
+    const uint8_t *sbase = p.side + ((long long)b * p.Hkv + h) * p.side_stride;
+    constexpr int KHALF = 16 * D + 64, VHALF = 16 * D, PAGE8 = 32 * D + 64;
+    uint32_t wb0 = 0, wb1 = 0;
+    for (int j = warp; j < p.np8; j += kMaskedWarps) {
+      if (!side_page_attended(j, L, p.sink, p.recent)) continue;
+      const uint4 *ks = reinterpret_cast<const uint4 *>(sbase + (long long)j * PAGE8);
+      for (int q = lane; q < KHALF / 16; q += 32) reinterpret_cast<uint4 *>(im)[q] = __ldg(ks + q);
+      __syncwarp();
+      int8k_item<D>(p, im_u32, q8_u32, j, r8, st, wb0, wb1, lane);
+      __syncwarp();
+      const uint4 *vs = reinterpret_cast<const uint4 *>(sbase + (long long)j * PAGE8 + KHALF);
+      for (int q = lane; q < VHALF / 16; q += 32) reinterpret_cast<uint4 *>(im)[q] = __ldg(vs + q);
+      __syncwarp();
+      int8v_item<D>(im_u32, st, wb0, wb1, lane);
+      __syncwarp();
+    }
+  }
   write_cp_partial<D, NMT>(G, st, parts + (((long long)warp * p.B + b) * p.Hq + h * G) * (D + 4), lane);
 }
 
-size_t masked_decode_smem(int D) { return 4 * kMaskedChunk + kv4_q_bytes(D) + (size_t)kMaskedWarps * 18 * D; }
+size_t masked_decode_smem(int D) { return 4 * kMaskedChunk + 2 * kv4_q_bytes(D) + (size_t)kMaskedWarps * 18 * D; }
 
 template <int D>
 static cudaError_t launch_masked_d(const DecodeParams &p, const GatherParams &g, float *parts, cudaStream_t s) {
