@@ -217,22 +217,21 @@ kv4_status kv4_decode_partials(kv4_cache *cache, void *stream, const void *q, in
  * and scales whole; a V row's bytes from the 16-byte pieces of the V block
  * that hold them) and attended there, so only the retained rows' K codes and
  * scales and the V pieces of their 4-row groups are read, and the work is
- * proportional to the retained rows. The INT8 region is attended from the side
- * cache under the same mask, and the partials are merged. The result is the
- * same attention as kv4_decode_attn with retain_mask (within rounding).
- * Each (sequence, head) is gathered by one CTA, page after page, so the call
- * gains on sparse masks (an H2O-style 10% budget: 0.45x the unmasked decode
- * time on the eviction workload) and loses on dense ones (beyond about a third
- * of the positions, kv4_decode_attn with retain_mask is faster).
+ * proportional to the retained rows. The INT8 region's side pages are attended
+ * by the same CTAs under the same mask, and the CTAs' partials are merged. The
+ * result is the same attention as kv4_decode_attn with retain_mask (within
+ * rounding). Each (sequence, head) is gathered by one CTA, page after page, so
+ * the call gains on sparse masks (an H2O-style 10% budget: 0.37x the unmasked
+ * decode time on the eviction workload) and loses on dense ones (beyond about a
+ * third of the positions, kv4_decode_attn with retain_mask is faster).
  *  retain_mask: device uint32 [B][Hkv][mask_stride], required; mask_stride *
  *    32 >= pt_stride * 16.
  *  max_retained: bound on the retained INT4-region positions [sink, L - recent)
  *    of any (sequence, head). A row with more sets KV4_ERR_CAPACITY and only
  *    its first max_retained positions are attended.
  *  workspace: device, >= kv4_masked_workspace_bytes(), 256-byte aligned.
- * Other arguments as kv4_decode_attn (the default worker count is used for the
- * INT8 region). Launches on `stream`: a count kernel, the gathering kernel, an
- * INT8-region worker and merge pair, and a partial merge.
+ * Other arguments as kv4_decode_attn. Launches on `stream`: a count kernel,
+ * the gathering kernel and a partial merge.
  */
 kv4_status kv4_masked_workspace_bytes(const kv4_cache *cache, int32_t B, int32_t Hq, int32_t pt_stride,
                                       int32_t max_retained, size_t *bytes);
