@@ -170,7 +170,7 @@ __device__ __forceinline__ uint16_t quant_group32(const float (&x)[kGroup], int 
 // forms, in shared memory, the prefix over sequences of their completely
 // filled pages, then maps its warps' units onto (sequence, page, head).
 template <int D>
-__global__ void __launch_bounds__(256, 3) append_pages_kernel(AppendParams p) {
+__global__ void __launch_bounds__(256, 4) append_pages_kernel(AppendParams p) {
   constexpr int WARPS = 8, NG = D / kGroup;
   __shared__ __align__(16) uint8_t img[WARPS][18 * D];
   __shared__ int wtot[WARPS];
