@@ -343,6 +343,7 @@ kv4_status kv4_append(kv4_cache *cache, void *stream, const void *k_new, const v
   p.page_bytes = p.head_bytes * p.Hkv;
   p.side_stride = side_head_bytes(D, p.sink, p.recent);
   p.err = cache->err;
+  p.num_sms = cache->num_sms;
   return cuda_status(launch_append(p, D, static_cast<cudaStream_t>(stream)));
 }
 

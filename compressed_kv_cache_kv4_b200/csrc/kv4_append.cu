@@ -13,23 +13,23 @@
 // quantises half a group (16 elements) of row l % 16 -- the two lanes of a
 // group combine their maxima with one shuffle -- into a shared-memory image
 // of the 18*D-byte head block, which the warp then writes out with 16-byte
-// stores. Codes are packed arithmetically: with u = c + 8 in [1, 15], four
-// codes make an exact fp32 integer u0 + 16 u1 + 256 u2 + 4096 u3 whose bits
-// an added 2^23 exposes, and XOR with 0x8 per nibble gives c mod 16.
-// append_kernel takes the rest: one warp per (new position, KV head, K or V),
-// lane l holding D/32 consecutive elements, for the INT4 slots of partially
-// filled pages and for every INT8 side-cache row.
+// stores. The rest -- the INT4 slots of partially filled pages and every INT8
+// side-cache row -- goes to append_tokens_kernel (one warp per new position,
+// over its KV heads and K / V), or, when no page is filled completely, to
+// append_kernel (one warp per new position, KV head and K or V); there lane l
+// holds D/32 consecutive elements of the row.
 //
 // Scale: fp32 IEEE division then round-up to fp16 equals rounding the exact
 // quotient a/7 (a/127) up: for a bf16 numerator the quotient is either exact
 // or has a periodic binary expansion whose bits past the fp16 precision are
-// never all zero, so the fp32 rounding cannot land on an fp16 value.
-// Code: x/s differs from every half-integer it is not equal to by at least
-// 2^-10, while x * r, with r = 1/s rounded (or approximated to an ulp or two),
-// differs from x/s by less than 2^-19 for |x/s| <= 7, so rounding x * r to the
-// nearest integer is exact except at true half-way points; those are detected
-// exactly through the residual c*s - x (exact in fp32) and resolved to the
-// even code.
+// never all zero, so the fp32 rounding cannot land on an fp16 value. The
+// division is one multiply and two fmas (div_by_const).
+// Code: x/s is either a half-integer or more than 2^-12 away from every
+// half-integer, so x * r (r an approximate 1/s) snapped to a 2^-13 grid keeps
+// the exact half-integers and the side of every other value, and one more
+// addition rounds it to the nearest integer with ties to even (biased_code2).
+// The codes stay biased by 1.5 * 2^23, whose low mantissa bits are then the
+// two's-complement code, so nibbles and bytes come straight from the bits.
 #include <algorithm>
 
 #include "kv4_common.cuh"
@@ -39,30 +39,16 @@ namespace kv4 {
 
 __device__ __forceinline__ uint32_t nib(int c) { return static_cast<uint32_t>(c) & 0xFu; }
 
-// Nearest-even integer to x/s (s > 0), given r = RN(1/s).
-__device__ __forceinline__ float round_code(float x, float s, float r) {
-  float c = rintf(x * r);
-  const float d = fmaf(c, s, -x);   // c*s - x, exact
-  if (2.f * fabsf(d) == s) {        // half-way: x/s = c - sign(d)/2; keep the even one
-    if (static_cast<int>(c) & 1) c -= copysignf(1.f, d);
-  }
-  return c;
-}
-
-// The same for two values with one scale (packed f32x2 arithmetic); r only
-// has to be within 2^-20 of 1/s (an approximate reciprocal will do): the
-// half-way test uses the exact residual, not r.
-__device__ __forceinline__ float2 round_code2(float2 x, float s, float r) {
-  const float2 q = __fmul2_rn(x, make_float2(r, r));
-  // nearest-even integer of q (|q| < 2^22): adding 1.5 * 2^23 rounds q to an
-  // integer in the last mantissa place, subtracting it again is exact
-  float2 c = __fadd2_rn(__fadd2_rn(q, make_float2(12582912.f, 12582912.f)), make_float2(-12582912.f, -12582912.f));
-  const float2 d = __ffma2_rn(c, make_float2(s, s), make_float2(-x.x, -x.y));   // c*s - x, exact
-  if (2.f * fabsf(d.x) == s || 2.f * fabsf(d.y) == s) {   // rare: an exact half-way point
-    if (2.f * fabsf(d.x) == s && (static_cast<int>(c.x) & 1)) c.x -= copysignf(1.f, d.x);
-    if (2.f * fabsf(d.y) == s && (static_cast<int>(c.y) & 1)) c.y -= copysignf(1.f, d.y);
-  }
-  return c;
+// a / d rounded to nearest for a constant d, given y = RN(1/d): q0 = RN(a*y)
+// is within an ulp of a/d, the residual a - d*q0 is exact in one fma, and the
+// corrected q0 + r*y rounds to the correctly rounded quotient (Markstein's
+// division by reciprocal with one fma correction). For d = 7 and d = 127 the
+// result equals IEEE division for every positive finite fp32 a (checked
+// exhaustively against the C library's division).
+__device__ __forceinline__ float div_by_const(float a, float d, float y) {
+  const float q0 = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-d, q0, a);
+  return __fmaf_rn(r, y, q0);
 }
 
 // 1/s to within an ulp or two (fp32 approximate reciprocal).
@@ -72,20 +58,39 @@ __device__ __forceinline__ float rcp_approx(float s) {
   return r;
 }
 
-// Codes c0..c3 in [-7, 7] -> 16 bits of four 4-bit two's-complement nibbles
-// (c0 lowest). With u = c + 8 in [1, 15], u0 + 16 u1 + 256 u2 + 4096 u3 is an
-// integer below 2^16, exact in fp32; adding 2^23 puts it in the low mantissa
-// bits, and nibble u ^ 8 = c mod 16 (the caller XORs 0x8888).
-__device__ __forceinline__ uint32_t nib4_biased(float c0, float c1, float c2, float c3) {
-  const float v = fmaf(c3, 4096.f, fmaf(c2, 256.f, fmaf(c1, 16.f, c0 + 34952.f)));   // 34952 = 8 * 0x1111
-  return __float_as_uint(v + 8388608.f);
+// Codes kept biased: kCodeBias + c is an fp32 integer in [2^23, 2^24), where
+// consecutive integers have consecutive bit patterns and the pattern of
+// kCodeBias ends in 4 zero bits, so its low 4 bits are c mod 16.
+constexpr float kCodeBias = 12582912.f;   // 1.5 * 2^23
+
+// kCodeBias + (x/s rounded to the nearest integer, ties to even) for two values,
+// given r within 4 ulps of 1/s (rcp.approx is within one) and |x/s| <= 127.5;
+// r = 0 gives 0 for x = 0. x/s is a half-integer or more than 2^-12 from every
+// half-integer: with x = X 2^ex (|X| < 2^8) and s = S 2^es (S < 2^11),
+// 2x - (2k+1)s is a multiple of 2^min(ex+1, es), which over 2s is at least
+// 1/(2S) if ex + 1 >= es, and otherwise, where |x/s| >= 1/4, at least 1/(4|X|).
+// x*r is within 127.5 * 2^-21 < 2^-14 of x/s, and x*r + 1536 is rounded once
+// to the 2^-13 spacing of fp32 in [1024, 2048): the result is exactly k + 1/2
+// at a half-integer x/s, and elsewhere it stays more than 2^-12 - 2^-14 - 2^-14
+// > 0 away on the same side of every half-integer. Adding 1.5 * 2^23 - 1536
+// then rounds to the nearest integer, ties to even. (Checked exhaustively on
+// the CPU: every positive fp16 s and every bf16 x with |x| <= 7s, and with
+// |x| <= 127s, for r = RN(1/s) and r moved by 2 and 4 ulps either way.)
+__device__ __forceinline__ float2 biased_code2(float2 x, float r) {
+  const float2 t = __ffma2_rn(x, make_float2(r, r), make_float2(1536.f, 1536.f));
+  return __fadd2_rn(t, make_float2(kCodeBias - 1536.f, kCodeBias - 1536.f));
+}
+
+// Byte of two biased codes: lo in the low nibble, hi in the high nibble.
+__device__ __forceinline__ uint32_t nib_pair(float lo, float hi) {
+  return (__float_as_uint(lo) & 0xFu) | ((__float_as_uint(hi) << 4) & 0xF0u);
 }
 
 // Quantise this lane's EPL values with a scale shared by `span` lanes
-// (span = lanes per group for INT4, 32 for INT8). Returns the fp16 scale bits.
-template <int EPL>
-__device__ __forceinline__ uint16_t quant_lane(const float (&x)[EPL], int span, float qmax, int (&c)[EPL],
-                                               uint32_t *err) {
+// (span = lanes per group for INT4, 32 for INT8) to codes in [-QMAX, QMAX].
+// Returns the fp16 scale bits.
+template <int EPL, int QMAX>
+__device__ __forceinline__ uint16_t quant_lane(const float (&x)[EPL], int span, int (&c)[EPL], uint32_t *err) {
   float a = 0.f;
 #pragma unroll
   for (int e = 0; e < EPL; ++e) a = fmaxf(a, fabsf(x[e]));
@@ -95,18 +100,28 @@ __device__ __forceinline__ uint16_t quant_lane(const float (&x)[EPL], int span, 
     for (int e = 0; e < EPL; ++e) c[e] = 0;
     return 0;
   }
-  uint16_t bits = __half_as_ushort(__float2half_ru(__fdiv_rn(a, qmax)));
-  if (bits == 0x7C00u) {           // a/qmax > 65504: saturate and flag
+  constexpr float qm = static_cast<float>(QMAX);
+  uint16_t bits = __half_as_ushort(__float2half_ru(div_by_const(a, qm, 1.f / qm)));
+  const bool sat = bits == 0x7C00u;
+  if (sat) {                       // a/qmax > 65504: saturate and flag
     bits = 0x7BFFu;
     set_error(err, kErrRange);
   }
-  const float s = half_bits_to_f32(bits);
-  const float r = __frcp_rn(s);
+  const float r = rcp_approx(half_bits_to_f32(bits));
+  float cb[EPL];
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    const float v = fminf(fmaxf(round_code(x[e], s, r), -qmax), qmax);
-    c[e] = static_cast<int>(v);
+  for (int e = 0; e < EPL; e += 2) {
+    const float2 v = biased_code2(make_float2(x[e], x[e + 1]), r);
+    cb[e] = v.x;
+    cb[e + 1] = v.y;
   }
+  // s >= max|x| / qmax makes |x / s| <= qmax: a clamp only when s saturated
+  if (sat) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) cb[e] = fminf(fmaxf(cb[e], kCodeBias - qm), kCodeBias + qm);
+  }
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) c[e] = static_cast<int>(__float_as_uint(cb[e]) - __float_as_uint(kCodeBias));
   return bits;
 }
 
@@ -137,45 +152,158 @@ __device__ __forceinline__ bool in_full_page(int pos, int L_old, int L_new) {
   return pos >= f0 && pos < f1;
 }
 
-// Scale bits and codes of one group of 32 values held by one thread (the same
-// quantiser as quant_lane, without lanes to combine).
-__device__ __forceinline__ uint16_t quant_group32(const float (&x)[kGroup], int (&c)[kGroup], uint32_t *err) {
-  float a = 0.f;
-#pragma unroll
-  for (int e = 0; e < kGroup; ++e) a = fmaxf(a, fabsf(x[e]));
-  if (a == 0.f) {
-#pragma unroll
-    for (int e = 0; e < kGroup; ++e) c[e] = 0;
-    return 0;
-  }
-  uint16_t bits = __half_as_ushort(__float2half_ru(__fdiv_rn(a, 7.f)));
-  const bool sat = bits == 0x7C00u;
-  if (sat) {                       // a/7 > 65504: saturate and flag
-    bits = 0x7BFFu;
-    set_error(err, kErrRange);
-  }
-  const float s = half_bits_to_f32(bits);
-  const float r = __frcp_rn(s);
-  // s >= max|x| / 7 makes |x / s| <= 7, so the codes need a clamp only when
-  // the scale saturated
-#pragma unroll
-  for (int e = 0; e < kGroup; ++e) {
-    const float v = round_code(x[e], s, r);
-    c[e] = static_cast<int>(sat ? fminf(fmaxf(v, -7.f), 7.f) : v);
-  }
-  return bits;
+constexpr int kAppendWarps = 8;
+
+// Shared-memory pitch of one staged bf16 row: 2*D bytes plus 16, so that the
+// 16 rows of a page start 4 banks apart and the lanes' 16-byte reads of one
+// instruction take the minimum of 4 wavefronts.
+template <int D>
+constexpr int kStageRow = 2 * D + 16;
+
+// append_pages_kernel's dynamic shared memory: per warp a stage of 16 rows and
+// the 18*D-byte image of one head block, per warp an mbarrier, then the plan.
+template <int D>
+constexpr size_t append_pages_smem(int B) {
+  return (size_t)kAppendWarps * (16 * kStageRow<D> + 18 * D + 8) + (size_t)(B + 1) * 4;
 }
 
-// One warp per (page the append fills completely, KV head). Every CTA first
-// forms, in shared memory, the prefix over sequences of their completely
-// filled pages, then maps its warps' units onto (sequence, page, head).
+// (page the append fills completely, KV head) number u -> sequence b, head h,
+// page index pg within the sequence, and j, the first of its 16 new rows.
+__device__ __forceinline__ void locate_page_unit(const AppendParams &p, const int *fplan, long long u, int &b,
+                                                 int &h, int &pg, long long &j) {
+  const int unit = static_cast<int>(u / p.Hkv);
+  h = static_cast<int>(u % p.Hkv);
+  int lo = 0, hi = p.B - 1;   // sequence: largest b with fplan[b] <= unit
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (fplan[mid] <= unit) lo = mid;
+    else hi = mid - 1;
+  }
+  b = lo;
+  const int L_old = p.lens_old[b];
+  pg = (L_old + kPageTokens - 1) / kPageTokens + (unit - fplan[b]);
+  j = p.offsets[b] + ((long long)pg * kPageTokens - L_old);
+}
+
+// Lanes 0..15 copy row j + lane of KV head h (K or V) into the warp's stage
+// with the bulk-copy engine; lane 0 arms the stage's barrier for the bytes.
 template <int D>
-__global__ void __launch_bounds__(256, 4) append_pages_kernel(AppendParams p) {
-  constexpr int WARPS = 8, NG = D / kGroup;
-  __shared__ __align__(16) uint8_t img[WARPS][18 * D];
+__device__ __forceinline__ void stage_rows(const AppendParams &p, long long j, int h, int kv, uint8_t *stage,
+                                           uint64_t *bar, int lane) {
+  if (lane == 0) mbar_arrive_expect_tx(bar, 16 * 2 * D);
+  if (lane < 16) {
+    const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + ((j + lane) * p.Hkv + h) * D;
+    bulk_g2s(stage + lane * kStageRow<D>, src, 2 * D, bar);
+  }
+}
+
+// Quantise the 16 rows of one KV head's K (kv = 0) or V (kv = 1) of a page
+// into the image of its head block. Lane (r, hh) holds row r, elements
+// [16 hh, 16 hh + 16) of every group of 32: raw[2i], raw[2i+1] for group i.
+template <int D>
+__device__ __forceinline__ void quant_page_rows(const uint4 (&raw)[D / 16], int kv, uint8_t *im, int r, int hh,
+                                                uint32_t *err) {
+  constexpr int NG = D / kGroup;
+  uint32_t kword[2][NG], sc_pair[(NG + 1) / 2] = {};
+#pragma unroll
+  for (int i = 0; i < NG; ++i) {
+    float x[16];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint4 w = raw[2 * i + q];
+      x[8 * q + 0] = bf16lo_to_f32(w.x);
+      x[8 * q + 1] = bf16hi_to_f32(w.x);
+      x[8 * q + 2] = bf16lo_to_f32(w.y);
+      x[8 * q + 3] = bf16hi_to_f32(w.y);
+      x[8 * q + 4] = bf16lo_to_f32(w.z);
+      x[8 * q + 5] = bf16hi_to_f32(w.z);
+      x[8 * q + 6] = bf16lo_to_f32(w.w);
+      x[8 * q + 7] = bf16hi_to_f32(w.w);
+    }
+    // scale of the group: max |x| over both lanes of the pair (lane ^ 16)
+    float a = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(x[e]));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
+    uint32_t sbits = 0;
+    float rc = 0.f;   // a == 0: every code is 0
+    bool sat = false;
+    if (a != 0.f) {
+      sbits = __half_as_ushort(__float2half_ru(div_by_const(a, 7.f, 1.f / 7.f)));
+      sat = sbits == 0x7C00u;
+      if (sat) {                       // a/7 > 65504: saturate and flag
+        sbits = 0x7BFFu;
+        if (hh == 0) set_error(err, kErrRange);
+      }
+      rc = rcp_approx(half_bits_to_f32(static_cast<uint16_t>(sbits)));
+    }
+    float cb[16];   // biased codes 1.5 * 2^23 + c
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const float2 v = biased_code2(make_float2(x[e], x[e + 1]), rc);
+      cb[e] = v.x;
+      cb[e + 1] = v.y;
+    }
+    // sc >= max|x| / 7 makes |x / sc| <= 7: a clamp only when sc saturated
+    if (sat) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) cb[e] = fminf(fmaxf(cb[e], kCodeBias - 7.f), kCodeBias + 7.f);
+    }
+    if (kv == 0) {
+      // K: element 32i + 8t + k of row r is nibble k of the word at
+      // r*D/2 + t*D/8 + 4i; this lane's elements are chunks t = 2hh, 2hh+1
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        kword[q][i] = nib_pair(cb[8 * q], cb[8 * q + 1]) | nib_pair(cb[8 * q + 2], cb[8 * q + 3]) << 8 |
+                      nib_pair(cb[8 * q + 4], cb[8 * q + 5]) << 16 | nib_pair(cb[8 * q + 6], cb[8 * q + 7]) << 24;
+    } else {
+      // V: the byte of (slot r, element d) pairs d and d+8 (low, high nibble);
+      // this lane's d = 32i + 16hh + e, e < 8 (m = 2i + hh, d mod 8 = e)
+      const int m = 2 * i + hh, tt = (r % 8) / 2;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int word = (m / 4) * 128 + (8 * tt + (e ^ (2 * tt))) * 4 + (m % 4);
+        im[8 * D + 4 * word + 2 * (r % 2) + r / 8] = static_cast<uint8_t>(nib_pair(cb[e], cb[e + 8]));
+      }
+    }
+    sc_pair[i / 2] |= sbits << (16 * (i % 2));
+  }
+  if (kv == 0) {
+    // chunk t = 2hh + q of row r: the words of groups 0 .. NG-1, 16 (D = 128) or 8 bytes
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint8_t *kd = im + r * (D / 2) + (2 * hh + q) * (D / 8);
+      if constexpr (NG == 4) *reinterpret_cast<uint4 *>(kd) = make_uint4(kword[q][0], kword[q][1], kword[q][2], kword[q][3]);
+      else *reinterpret_cast<uint2 *>(kd) = make_uint2(kword[q][0], kword[q][1]);
+    }
+  }
+  // the NG fp16 scales of row r, K at 16D, V at 17D
+  if (hh == 0) {
+    uint8_t *sd = im + (16 + kv) * D + 2 * NG * r;
+    if constexpr (NG == 4) *reinterpret_cast<uint2 *>(sd) = make_uint2(sc_pair[0], sc_pair[1]);
+    else *reinterpret_cast<uint32_t *>(sd) = sc_pair[0];
+  }
+}
+
+// One warp per (page the append fills completely, KV head) at a time, over a
+// grid of resident CTAs. Every CTA first forms, in shared memory, the prefix
+// over sequences of their completely filled pages, then maps its warps' units
+// onto (sequence, page, head). Each warp streams its units' rows through a
+// one-stage buffer: as soon as its lanes hold the staged K (V) rows in
+// registers, the bulk-copy engine fetches the V rows (the next unit's K rows)
+// into the same stage while the lanes quantise.
+template <int D>
+__global__ void __launch_bounds__(256, 3) append_pages_kernel(AppendParams p) {
+  constexpr int WARPS = kAppendWarps;
+  extern __shared__ __align__(16) uint8_t smem[];
   __shared__ int wtot[WARPS];
-  extern __shared__ int fplan[];   // [B + 1]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint8_t *stage = smem + warp * 16 * kStageRow<D>;
+  uint8_t *im = smem + WARPS * 16 * kStageRow<D> + warp * 18 * D;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + WARPS * (16 * kStageRow<D> + 18 * D));
+  int *fplan = reinterpret_cast<int *>(bars + WARPS);
+  if (tid < WARPS) mbar_init(&bars[tid], 1);
+  fence_mbar_init();
   pdl_wait();
   pdl_launch_dependents();
 
@@ -208,108 +336,63 @@ __global__ void __launch_bounds__(256, 4) append_pages_kernel(AppendParams p) {
   __syncthreads();
 
   const long long units = (long long)fplan[p.B] * p.Hkv;
-  uint8_t *im = img[warp];
-  // lane (r, hh): row r of the page, elements [16 hh, 16 hh + 16) of each group;
-  // K first, then V, so that the whole warp runs one code path at a time
+  const long long stride = (long long)gridDim.x * WARPS;
+  long long u = (long long)blockIdx.x * WARPS + warp;
+  if (u >= units) return;
+  uint64_t *bar = &bars[warp];
+  // lane (r, hh): row r of the page, elements [16 hh, 16 hh + 16) of each group
   const int r = lane & 15, hh = lane >> 4;
-  for (long long u = (long long)blockIdx.x * WARPS + warp; u < units; u += (long long)gridDim.x * WARPS) {
-    const int unit = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
-    int lo = 0, hi = p.B - 1;   // sequence: largest b with fplan[b] <= unit
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (fplan[mid] <= unit) lo = mid;
-      else hi = mid - 1;
-    }
-    const int b = lo;
-    const int L_old = p.lens_old[b];
-    const int pg = (L_old + kPageTokens - 1) / kPageTokens + (unit - fplan[b]);
-    if (pg >= p.pt_stride) {
-      if (lane == 0) set_error(p.err, kErrCapacity);
-      continue;
-    }
-    const int page = p.page_table[(long long)b * p.pt_stride + pg];
-    if (page < 0 || page >= p.num_pages) {
-      if (lane == 0) set_error(p.err, kErrBounds);
-      continue;
-    }
-    // rows j .. j+15 are the page's slots 0..15 (all new, all of sequence b)
-    const long long j = p.offsets[b] + (pg * kPageTokens - L_old);
+  const uint32_t sa = smem_u32(stage) + r * kStageRow<D> + 32 * hh;
+  int b, h, pg;
+  long long j;
+  locate_page_unit(p, fplan, u, b, h, pg, j);
+  stage_rows<D>(p, j, h, 0, stage, bar, lane);
+  uint32_t phase = 0;
+  for (;;) {
+    const long long un = u + stride;
+    int nb = 0, nh = 0, npg = 0;
+    long long nj = 0;
+    if (un < units) locate_page_unit(p, fplan, un, nb, nh, npg, nj);
+    const int page = pg < p.pt_stride ? p.page_table[(long long)b * p.pt_stride + pg] : -1;
 #pragma unroll 1
     for (int kv = 0; kv < 2; ++kv) {
-      const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + ((j + r) * p.Hkv + h) * D + 16 * hh;
-#pragma unroll
-      for (int i = 0; i < NG; ++i) {   // unrolled: the groups' loads are in flight together
-        float x[16];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(src + kGroup * i + 8 * q);
-          x[8 * q + 0] = bf16lo_to_f32(w.x);
-          x[8 * q + 1] = bf16hi_to_f32(w.x);
-          x[8 * q + 2] = bf16lo_to_f32(w.y);
-          x[8 * q + 3] = bf16hi_to_f32(w.y);
-          x[8 * q + 4] = bf16lo_to_f32(w.z);
-          x[8 * q + 5] = bf16hi_to_f32(w.z);
-          x[8 * q + 6] = bf16lo_to_f32(w.w);
-          x[8 * q + 7] = bf16hi_to_f32(w.w);
-        }
-        // scale of the group: max |x| over both lanes of the pair (lane ^ 16)
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(x[e]));
-        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
-        uint16_t sbits = 0;
-        float c[16];
-        if (a == 0.f) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) c[e] = 0.f;
-        } else {
-          sbits = __half_as_ushort(__float2half_ru(__fdiv_rn(a, 7.f)));
-          const bool sat = sbits == 0x7C00u;
-          if (sat) {                       // a/7 > 65504: saturate and flag
-            sbits = 0x7BFFu;
-            if (hh == 0) set_error(p.err, kErrRange);
-          }
-          const float sc = half_bits_to_f32(sbits);
-          const float rc = rcp_approx(sc);
-          // sc >= max|x| / 7 makes |x / sc| <= 7: a clamp only when sc saturated
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float2 v = round_code2(make_float2(x[e], x[e + 1]), sc, rc);
-            if (sat) v = make_float2(fminf(fmaxf(v.x, -7.f), 7.f), fminf(fmaxf(v.y, -7.f), 7.f));
-            c[e] = v.x;
-            c[e + 1] = v.y;
-          }
-        }
-        if (kv == 0) {
-          // K: element 32i + 8t + k of row r is nibble k of the word at
-          // r*D/2 + t*D/8 + 4i; this lane's elements are chunks t = 2hh, 2hh+1
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const uint32_t w = __byte_perm(nib4_biased(c[8 * q], c[8 * q + 1], c[8 * q + 2], c[8 * q + 3]),
-                                           nib4_biased(c[8 * q + 4], c[8 * q + 5], c[8 * q + 6], c[8 * q + 7]),
-                                           0x5410) ^ 0x88888888u;
-            *reinterpret_cast<uint32_t *>(im + r * (D / 2) + (2 * hh + q) * (D / 8) + 4 * i) = w;
-          }
-          if (hh == 0) *reinterpret_cast<uint16_t *>(im + 16 * D + 2 * (r * NG + i)) = sbits;
-        } else {
-          // V: the byte of (slot r, element d) pairs d and d+8 (low, high nibble);
-          // this lane's d = 32i + 16hh + e, e < 8 (m = 2i + hh, d mod 8 = e)
-          const int m = 2 * i + hh, tt = (r % 8) / 2;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int word = (m / 4) * 128 + (8 * tt + (e ^ (2 * tt))) * 4 + (m % 4);
-            const uint32_t byte = (__float_as_uint(fmaf(c[e + 8], 16.f, c[e] + 136.f) + 8388608.f) & 0xFFu) ^ 0x88u;
-            im[8 * D + 4 * word + 2 * (r % 2) + r / 8] = static_cast<uint8_t>(byte);
-          }
-          if (hh == 0) *reinterpret_cast<uint16_t *>(im + 17 * D + 2 * (r * NG + i)) = sbits;
-        }
+      const bool ok = mbar_wait_bounded(bar, phase, kDefaultWaitCycles);
+      if (!__all_sync(0xffffffffu, ok)) {   // the copy did not land: flag, drain it, stop
+        if (lane == 0) set_error(p.err, kErrTimeout);
+        mbar_wait_bounded(bar, phase, kDefaultWaitCycles);
+        return;
       }
+      phase ^= 1u;
+      uint4 raw[D / 16];
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        raw[2 * i] = lds128(sa + 64 * i);
+        raw[2 * i + 1] = lds128(sa + 64 * i + 16);
+      }
+      // the stage is read: order the reads before the next bulk write into it
+      fence_proxy_async();
+      __syncwarp();
+      if (kv == 0) stage_rows<D>(p, j, h, 1, stage, bar, lane);
+      else if (un < units) stage_rows<D>(p, nj, nh, 0, stage, bar, lane);
+      quant_page_rows<D>(raw, kv, im, r, hh, p.err);
     }
     __syncwarp();
-    uint4 *dst = reinterpret_cast<uint4 *>(p.pool + (long long)page * p.page_bytes + (long long)h * p.head_bytes);
-    const uint4 *srci = reinterpret_cast<const uint4 *>(im);
-    for (int q = lane; q < 18 * D / 16; q += 32) dst[q] = srci[q];
+    if (pg >= p.pt_stride) {
+      if (lane == 0) set_error(p.err, kErrCapacity);
+    } else if (page < 0 || page >= p.num_pages) {
+      if (lane == 0) set_error(p.err, kErrBounds);
+    } else {
+      uint4 *dst = reinterpret_cast<uint4 *>(p.pool + (long long)page * p.page_bytes + (long long)h * p.head_bytes);
+      const uint4 *srci = reinterpret_cast<const uint4 *>(im);
+      for (int q = lane; q < 18 * D / 16; q += 32) dst[q] = srci[q];
+    }
     __syncwarp();
+    if (un >= units) break;
+    u = un;
+    b = nb;
+    h = nh;
+    pg = npg;
+    j = nj;
   }
 }
 
@@ -356,7 +439,7 @@ __device__ __forceinline__ void append_row(const AppendParams &p, long long j, i
 
     // ---- INT4 copy, one scale per group of 32
     int c[EPL];
-    const uint16_t s4 = skip4 ? 0 : quant_lane<EPL>(x, LPG, 7.f, c, p.err);
+    const uint16_t s4 = skip4 ? 0 : quant_lane<EPL, 7>(x, LPG, c, p.err);
     if (skip4) {
     } else if (kv == 0) {
       // K: element d at row r, chunk (d%32)/8, word d/32, nibble d%8
@@ -389,7 +472,7 @@ __device__ __forceinline__ void append_row(const AppendParams &p, long long j, i
     // ---- INT8 side cache (sink row and/or ring row), one scale per token row
     if (sink_row >= 0 || ring_row >= 0) {
       int c8[EPL];
-      const uint16_t s8 = quant_lane<EPL>(x, 32, 127.f, c8, p.err);
+      const uint16_t s8 = quant_lane<EPL, 127>(x, 32, c8, p.err);
       int partner8[EPL];
 #pragma unroll
       for (int e = 0; e < EPL; ++e) partner8[e] = __shfl_down_sync(0xffffffffu, c8[e], 8 / EPL);
@@ -532,6 +615,15 @@ __global__ void __launch_bounds__(256) append_tokens_kernel(AppendParams p) {
   }
 }
 
+template <int D>
+cudaError_t launch_append_pages(unsigned blocks, const AppendParams &p, cudaStream_t stream) {
+  const size_t smem = append_pages_smem<D>(p.B);
+  const cudaError_t attr = cudaFuncSetAttribute(append_pages_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)smem);
+  if (attr != cudaSuccess) return attr;
+  return launch_pdl(append_pages_kernel<D>, dim3(blocks), dim3(32 * kAppendWarps), smem, stream, p);
+}
+
 cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream) {
   AppendParams p = p_in;
   const long long tasks = p.T * p.Hkv * 2;
@@ -540,21 +632,19 @@ cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream) 
   // Pages can only be filled completely by a multi-position append; the page
   // kernel reads rows with 16-byte loads and keeps its plan in shared memory.
   const bool aligned16 = ((reinterpret_cast<uintptr_t>(p.k) | reinterpret_cast<uintptr_t>(p.v)) & 15u) == 0;
-  // (the plan, 4 bytes per sequence, stays within the default 48 KB with the page images)
+  // (the plan, 4 bytes per sequence, and the stages stay within 227 KB of shared memory)
   p.page_kernel = (p.offsets && p.T >= kPageTokens && aligned16 && p.B <= 7168) ? 1 : 0;
   if (!p.page_kernel) {
     const unsigned blocks = static_cast<unsigned>((tasks + warps_per_block - 1) / warps_per_block);
     if (D == 128) return launch_pdl(append_kernel<128>, dim3(blocks), dim3(32 * warps_per_block), 0, stream, p);
     return launch_pdl(append_kernel<64>, dim3(blocks), dim3(32 * warps_per_block), 0, stream, p);
   }
+  // resident CTAs only (3 per SM): each warp keeps its stage busy over several units
   const long long units = (p.T / kPageTokens) * p.Hkv;   // upper bound on (full page, head) units
-  const unsigned pblocks = static_cast<unsigned>(
-      std::max(1LL, std::min((units + warps_per_block - 1) / warps_per_block, 8192LL)));
+  const unsigned pblocks = static_cast<unsigned>(std::max(
+      1LL, std::min((units + warps_per_block - 1) / warps_per_block, 3LL * std::max(p.num_sms, 1))));
   const size_t plan_bytes = (size_t)(p.B + 1) * 4;
-  cudaError_t e = D == 128 ? launch_pdl(append_pages_kernel<128>, dim3(pblocks), dim3(32 * warps_per_block),
-                                        plan_bytes, stream, p)
-                           : launch_pdl(append_pages_kernel<64>, dim3(pblocks), dim3(32 * warps_per_block),
-                                        plan_bytes, stream, p);
+  cudaError_t e = D == 128 ? launch_append_pages<128>(pblocks, p, stream) : launch_append_pages<64>(pblocks, p, stream);
   if (e != cudaSuccess) return e;
   // upper bound on the positions with work left: all of them, or per sequence
   // two partial pages plus the sink and ring rows

@@ -25,6 +25,7 @@ struct AppendParams {
   long long page_bytes, head_bytes, side_stride;
   uint32_t *err;
   int page_kernel;          // 1: pages filled completely by this append go through append_pages_kernel
+  int num_sms;              // SMs of the device (grid of the page kernel)
 };
 
 struct DecodeParams {
