@@ -31,6 +31,7 @@
 // The codes stay biased by 1.5 * 2^23, whose low mantissa bits are then the
 // two's-complement code, so nibbles and bytes come straight from the bits.
 #include <algorithm>
+#include <type_traits>
 
 #include "kv4_common.cuh"
 #include "kv4_internal.h"
@@ -396,47 +397,71 @@ __global__ void __launch_bounds__(256, 3) append_pages_kernel(AppendParams p) {
   }
 }
 
-// Quantise and store row (j, head h, K or V) of position pos of sequence b:
-// the INT4 slot (unless the page kernel owns the page) and the INT8 side rows.
-// One warp; lane l holds D/32 consecutive elements.
+// Where the rows of position pos of sequence b go: the INT4 slot r of `page`
+// (unless the page kernel owns the page) and the INT8 sink and ring rows.
+struct RowTarget {
+  int sink_row, ring_row, r, page;
+  bool skip4;
+};
+
+// False if the position has nothing to write here, or if its page id is out
+// of range (flagged).
+__device__ __forceinline__ bool row_target(const AppendParams &p, int b, int pos, int L_new, int lane, RowTarget &t) {
+  const int S = p.sink, R = p.recent;
+  t.sink_row = pos < S ? pos : -1;
+  t.ring_row = (R > 0 && pos >= L_new - R) ? (S > 0 ? 16 : 0) + pos % R : -1;
+  // INT4 slots of pages this append fills completely belong to append_pages_kernel
+  t.skip4 = p.page_kernel && in_full_page(pos, p.lens_old[b], L_new);
+  if (t.skip4 && t.sink_row < 0 && t.ring_row < 0) return false;
+  t.page = p.page_table[(long long)b * p.pt_stride + pos / kPageTokens];
+  if (t.page < 0 || t.page >= p.num_pages) {
+    if (lane == 0) set_error(p.err, kErrBounds);
+    return false;
+  }
+  t.r = pos % kPageTokens;
+  return true;
+}
+
+// This lane's D/32 consecutive bf16 elements of row (j, head h, K or V), packed.
 template <int D>
-__device__ __forceinline__ void append_row(const AppendParams &p, long long j, int h, int kv, int b, int pos,
-                                           int L_new, int lane) {
+using RowRaw = typename std::conditional<D / 32 == 4, uint2, uint32_t>::type;
+
+template <int D>
+__device__ __forceinline__ RowRaw<D> load_row_raw(const AppendParams &p, long long j, int h, int kv, int lane) {
+  const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + (j * p.Hkv + h) * D + lane * (D / 32);
+  return *reinterpret_cast<const RowRaw<D> *>(src);
+}
+
+__device__ __forceinline__ void unpack_row(uint2 raw, float (&x)[4]) {
+  x[0] = bf16lo_to_f32(raw.x);
+  x[1] = bf16hi_to_f32(raw.x);
+  x[2] = bf16lo_to_f32(raw.y);
+  x[3] = bf16hi_to_f32(raw.y);
+}
+
+__device__ __forceinline__ void unpack_row(uint32_t raw, float (&x)[2]) {
+  x[0] = bf16lo_to_f32(raw);
+  x[1] = bf16hi_to_f32(raw);
+}
+
+// Quantise and store one row (head h, K or V) of position pos of sequence b,
+// given by its lanes' elements x: the INT4 slot (unless the page kernel owns
+// the page) and the INT8 side rows. One warp; lane l holds D/32 consecutive
+// elements.
+template <int D>
+__device__ __forceinline__ void store_row(const AppendParams &p, const RowTarget &t, const float (&x)[D / 32], int h,
+                                          int kv, int b, int lane) {
   constexpr int EPL = D / 32;              // elements per lane
   constexpr int LPG = kGroup / EPL;        // lanes per INT4 group
-  const int S = p.sink, R = p.recent;
-  const int sink_row = pos < S ? pos : -1;
-  const int ring_row = (R > 0 && pos >= L_new - R) ? (S > 0 ? 16 : 0) + pos % R : -1;
-  // INT4 slots of pages this append fills completely belong to append_pages_kernel
-  const bool skip4 = p.page_kernel && in_full_page(pos, p.lens_old[b], L_new);
-  if (skip4 && sink_row < 0 && ring_row < 0) return;
-  const int page = p.page_table[(long long)b * p.pt_stride + pos / kPageTokens];
-  if (page < 0 || page >= p.num_pages) {
-    if (lane == 0 && kv == 0) set_error(p.err, kErrBounds);
-    return;
-  }
-  const int r = pos % kPageTokens;
-  uint8_t *blk = p.pool + (long long)page * p.page_bytes + (long long)h * p.head_bytes;
+  const int sink_row = t.sink_row, ring_row = t.ring_row, r = t.r;
+  const bool skip4 = t.skip4;
+  uint8_t *blk = p.pool + (long long)t.page * p.page_bytes + (long long)h * p.head_bytes;
   const int d0 = lane * EPL;
   const int grp = d0 / kGroup;
   uint8_t *sblk = p.side + ((long long)b * p.Hkv + h) * p.side_stride;
   const long long spage = 32LL * D + 64;
 
   {
-    const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + (j * p.Hkv + h) * D + d0;
-    float x[EPL];
-    if constexpr (EPL == 4) {
-      const uint2 raw = *reinterpret_cast<const uint2 *>(src);
-      x[0] = bf16lo_to_f32(raw.x);
-      x[1] = bf16hi_to_f32(raw.x);
-      x[2] = bf16lo_to_f32(raw.y);
-      x[3] = bf16hi_to_f32(raw.y);
-    } else {
-      const uint32_t raw = *reinterpret_cast<const uint32_t *>(src);
-      x[0] = bf16lo_to_f32(raw);
-      x[1] = bf16hi_to_f32(raw);
-    }
-
     // ---- INT4 copy, one scale per group of 32
     int c[EPL];
     const uint16_t s4 = skip4 ? 0 : quant_lane<EPL, 7>(x, LPG, c, p.err);
@@ -535,7 +560,11 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     if (lane == 0) set_error(p.err, kErrCapacity);
     return;
   }
-  append_row<D>(p, j, h, kv, b, pos, L_new, lane);
+  RowTarget t;
+  if (!row_target(p, b, pos, L_new, lane, t)) return;
+  float x[D / 32];
+  unpack_row(load_row_raw<D>(p, j, h, kv, lane), x);
+  store_row<D>(p, t, x, h, kv, b, lane);
 }
 
 // Positions of sequence b that have work outside the pages the append fills
@@ -561,7 +590,7 @@ __device__ __forceinline__ int token_work(const AppendParams &p, int b, int &L_o
 }
 
 // Used with append_pages_kernel: one warp per position that has work outside
-// the pages the append fills completely, looping over the KV heads and K / V.
+// the pages the append fills completely, over its KV heads and K / V.
 // Every CTA forms the prefix of those positions over sequences in shared memory.
 template <int D>
 __global__ void __launch_bounds__(256) append_tokens_kernel(AppendParams p) {
@@ -611,7 +640,24 @@ __global__ void __launch_bounds__(256) append_tokens_kernel(AppendParams p) {
       if (lane == 0) set_error(p.err, kErrCapacity);
       continue;
     }
-    for (int hk = 0; hk < 2 * p.Hkv; ++hk) append_row<D>(p, j, hk >> 1, hk & 1, b, pos, L_new, lane);
+    RowTarget t;
+    if (!row_target(p, b, pos, L_new, lane, t)) continue;
+    // the position's rows (KV head, K / V) in batches of 8, each batch's loads in flight together
+    for (int hk0 = 0; hk0 < 2 * p.Hkv; hk0 += 8) {
+      RowRaw<D> raw[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (hk0 + e < 2 * p.Hkv) raw[e] = load_row_raw<D>(p, j, (hk0 + e) >> 1, (hk0 + e) & 1, lane);
+      const int n = min(8, 2 * p.Hkv - hk0);
+#pragma unroll 1
+      for (int e = 0; e < n; ++e) {   // row hk0 + e sits in raw[0]: the batch shifts down
+        float x[D / 32];
+        unpack_row(raw[0], x);
+        store_row<D>(p, t, x, (hk0 + e) >> 1, (hk0 + e) & 1, b, lane);
+#pragma unroll
+        for (int k = 0; k < 7; ++k) raw[k] = raw[k + 1];
+      }
+    }
   }
 }
 
