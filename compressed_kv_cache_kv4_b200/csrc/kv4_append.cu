@@ -397,6 +397,24 @@ __global__ void __launch_bounds__(256, 3) append_pages_kernel(AppendParams p) {
   }
 }
 
+// INT8 side pages that an append with the page kernel writes whole, one warp
+// per (page, KV head) in append_tokens_kernel instead of row by row: the sink
+// page when the sequence starts with this append and fills all 16 of its rows,
+// and, when every position of the recent window is new, each ring page whose
+// 16 rows all hold a position (all of them once L_new >= recent). Every other
+// INT8 row is written by the row path, so no byte outside a row is touched.
+__device__ __forceinline__ bool sink_whole(const AppendParams &p, int L_old, int L_new) {
+  return p.page_kernel && p.sink == kPageTokens && L_old == 0 && L_new >= kPageTokens;
+}
+// Number of whole ring pages (ring pages 0 .. n-1).
+__device__ __forceinline__ int ring_whole(const AppendParams &p, int L_old, int L_new) {
+  const bool fresh = p.page_kernel && p.recent > 0 && L_old >= 0 && L_old <= max(L_new - p.recent, 0);
+  return fresh ? min(p.recent, L_new) / kPageTokens : 0;
+}
+__device__ __forceinline__ int side_pages_whole(const AppendParams &p, int L_old, int L_new) {
+  return (sink_whole(p, L_old, L_new) ? 1 : 0) + ring_whole(p, L_old, L_new);
+}
+
 // Where the rows of position pos of sequence b go: the INT4 slot r of `page`
 // (unless the page kernel owns the page) and the INT8 sink and ring rows.
 struct RowTarget {
@@ -407,11 +425,13 @@ struct RowTarget {
 // False if the position has nothing to write here, or if its page id is out
 // of range (flagged).
 __device__ __forceinline__ bool row_target(const AppendParams &p, int b, int pos, int L_new, int lane, RowTarget &t) {
-  const int S = p.sink, R = p.recent;
-  t.sink_row = pos < S ? pos : -1;
-  t.ring_row = (R > 0 && pos >= L_new - R) ? (S > 0 ? 16 : 0) + pos % R : -1;
+  const int S = p.sink, R = p.recent, L_old = p.lens_old[b];
+  t.sink_row = (pos < S && !sink_whole(p, L_old, L_new)) ? pos : -1;
+  t.ring_row = (R > 0 && pos >= L_new - R && (pos % R) / kPageTokens >= ring_whole(p, L_old, L_new))
+                   ? (S > 0 ? 16 : 0) + pos % R
+                   : -1;
   // INT4 slots of pages this append fills completely belong to append_pages_kernel
-  t.skip4 = p.page_kernel && in_full_page(pos, p.lens_old[b], L_new);
+  t.skip4 = p.page_kernel && in_full_page(pos, L_old, L_new);
   if (t.skip4 && t.sink_row < 0 && t.ring_row < 0) return false;
   t.page = p.page_table[(long long)b * p.pt_stride + pos / kPageTokens];
   if (t.page < 0 || t.page >= p.num_pages) {
@@ -569,8 +589,8 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
 
 // Positions of sequence b that have work outside the pages the append fills
 // completely: the slots of partly filled pages and the INT8 sink and ring
-// rows. They form [L_old, a_end) and [b_start, L_new) (one range if these
-// meet); returns their number.
+// rows not written page-wise. They form [L_old, a_end) and [b_start, L_new)
+// (one range if these meet); returns their number.
 __device__ __forceinline__ int token_work(const AppendParams &p, int b, int &L_old, int &a_end, int &b_start) {
   L_old = p.lens_old[b];
   const int L_new = L_old + (p.offsets[b + 1] - p.offsets[b]);
@@ -580,8 +600,9 @@ __device__ __forceinline__ int token_work(const AppendParams &p, int b, int &L_o
   }
   const int f0 = (L_old + kPageTokens - 1) / kPageTokens * kPageTokens;
   const int f1 = L_new / kPageTokens * kPageTokens;
-  a_end = min(L_new, max(f0, min(p.sink, f1)));
-  b_start = max(L_old, min(f1, max(L_new - p.recent, f0)));
+  // (ring rows of positions below f1 sit in whole ring pages when any ring page is whole)
+  a_end = min(L_new, max(f0, sink_whole(p, L_old, L_new) ? 0 : min(p.sink, f1)));
+  b_start = max(L_old, min(f1, max(ring_whole(p, L_old, L_new) > 0 ? f1 : L_new - p.recent, f0)));
   if (a_end >= b_start) {
     a_end = b_start = L_new;
     return L_new - L_old;
@@ -589,50 +610,191 @@ __device__ __forceinline__ int token_work(const AppendParams &p, int b, int &L_o
   return (a_end - L_old) + (L_new - b_start);
 }
 
-// Used with append_pages_kernel: one warp per position that has work outside
-// the pages the append fills completely, over its KV heads and K / V.
-// Every CTA forms the prefix of those positions over sequences in shared memory.
+// One INT8 side page j of (sequence b, KV head h) written whole (one warp):
+// lane (r, hh) quantises row r -- elements [16 hh, 16 hh + 16) of every group
+// of 32 -- of K, then of V, into a shared-memory image of the 32*D + 64-byte
+// page, written out with 16-byte stores. Row r of the sink page holds
+// position r; row r of ring page k holds the position of the recent window
+// congruent to 16 k + r modulo recent.
+template <int D>
+__device__ void append_side_page(const AppendParams &p, int b, int h, int j, int L_old, int L_new, uint8_t *im,
+                                 int lane) {
+  constexpr int NG = D / kGroup;
+  const int r = lane & 15, hh = lane >> 4;
+  const int js = p.sink > 0 ? 1 : 0;
+  // (every row of a whole page holds a position)
+  const int pos = j < js ? r : L_new - 1 - (L_new - 1 - (kPageTokens * (j - js) + r)) % p.recent;
+  const long long row = p.offsets[b] + (pos - L_old);
+#pragma unroll 1
+  for (int kv = 0; kv < 2; ++kv) {
+    uint4 raw[D / 16];
+    const __nv_bfloat16 *src = (kv == 0 ? p.k : p.v) + (row * p.Hkv + h) * D + 16 * hh;
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        raw[2 * i + q] = *reinterpret_cast<const uint4 *>(src + kGroup * i + 8 * q);
+    }
+    // row scale: max |x| over the row (this lane's half, then lane ^ 16)
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+      const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a = fmaxf(a, fmaxf(fabsf(bf16lo_to_f32(w[e])), fabsf(bf16hi_to_f32(w[e]))));
+    }
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 16));
+    uint32_t sbits = 0;
+    float rc = 0.f;   // a == 0: every code is 0
+    bool sat = false;
+    if (a != 0.f) {
+      sbits = __half_as_ushort(__float2half_ru(div_by_const(a, 127.f, 1.f / 127.f)));
+      sat = sbits == 0x7C00u;
+      if (sat) {                       // a/127 > 65504: saturate and flag
+        sbits = 0x7BFFu;
+        if (hh == 0) set_error(p.err, kErrRange);
+      }
+      rc = rcp_approx(half_bits_to_f32(static_cast<uint16_t>(sbits)));
+    }
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+      float cb[16];   // biased codes of elements d = 32i + 16hh + e
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const uint4 w = raw[2 * i + q];
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 v = biased_code2(make_float2(bf16lo_to_f32(ww[e]), bf16hi_to_f32(ww[e])), rc);
+          cb[8 * q + 2 * e] = v.x;
+          cb[8 * q + 2 * e + 1] = v.y;
+        }
+      }
+      if (sat) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) cb[e] = fminf(fmaxf(cb[e], kCodeBias - 127.f), kCodeBias + 127.f);
+      }
+      const int d0 = kGroup * i + 16 * hh;
+      if (kv == 0) {
+        // K row r, element d: byte d%4 of word (r/8)*(D/16) + (d%(D/4))/4 of
+        // lane 4*(r%8) + d/(D/4); 4 consecutive elements make one word
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int d = d0 + 4 * c;
+          const int lk = 4 * (r % 8) + d / (D / 4), w = (r / 8) * (D / 16) + (d % (D / 4)) / 4;
+          const uint32_t lo = __byte_perm(__float_as_uint(cb[4 * c]), __float_as_uint(cb[4 * c + 1]), 0x0040);
+          const uint32_t hi = __byte_perm(__float_as_uint(cb[4 * c + 2]), __float_as_uint(cb[4 * c + 3]), 0x0040);
+          *reinterpret_cast<uint32_t *>(im + (w / 4) * 512 + lk * 16 + (w % 4) * 4) = __byte_perm(lo, hi, 0x5410);
+        }
+      } else {
+        // V row r, element d (d%16 < 8): bytes 2(r%2) and 2(r%2)+1 of word
+        // 2(d/16) + r/8 of lane 4(d%8) + (r%8)/2 hold the codes of d and d+8
+        const int w = 2 * (d0 / 16) + r / 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int lv = 4 * e + (r % 8) / 2;
+          const uint32_t pair = __byte_perm(__float_as_uint(cb[e]), __float_as_uint(cb[e + 8]), 0x0040);
+          *reinterpret_cast<uint16_t *>(im + 16 * D + 64 + (w / 4) * 512 + lv * 16 + (w % 4) * 4 + 2 * (r % 2)) =
+              static_cast<uint16_t>(pair);
+        }
+      }
+    }
+    if (hh == 0) *reinterpret_cast<uint16_t *>(im + 16 * D + 32 * kv + 2 * r) = static_cast<uint16_t>(sbits);
+  }
+  __syncwarp();
+  uint4 *dst = reinterpret_cast<uint4 *>(p.side + ((long long)b * p.Hkv + h) * p.side_stride +
+                                         (long long)j * (32 * D + 64));
+  const uint4 *srci = reinterpret_cast<const uint4 *>(im);
+  for (int q = lane; q < (32 * D + 64) / 16; q += 32) dst[q] = srci[q];
+  __syncwarp();
+}
+
+// Used with append_pages_kernel: one warp per INT8 side page written whole
+// (append_side_page), then one warp per position that has work outside the
+// pages the append fills completely, over its KV heads and K / V. Every CTA
+// forms the prefixes over sequences of both counts in shared memory.
 template <int D>
 __global__ void __launch_bounds__(256) append_tokens_kernel(AppendParams p) {
   constexpr int WARPS = 8;
-  __shared__ int wtot[WARPS];
-  extern __shared__ int tplan[];   // [B + 1]
+  __shared__ int wtot[2][WARPS];
+  __shared__ __align__(16) uint8_t img[WARPS][32 * D + 64];
+  extern __shared__ int tplan[];   // [B + 1] positions, then [B + 1] side pages
+  int *splan = tplan + p.B + 1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
   pdl_launch_dependents();
+  auto side_count = [&](int b) {
+    const int L_old = p.lens_old[b];
+    return side_pages_whole(p, L_old, L_old + (p.offsets[b + 1] - p.offsets[b]));
+  };
   const int chunk = (p.B + WARPS * 32 - 1) / (WARPS * 32);
   const int b0 = min(p.B, tid * chunk), b1 = min(p.B, b0 + chunk);
-  int mine = 0, lo_, ae_, bs_;
-  for (int b = b0; b < b1; ++b) mine += token_work(p, b, lo_, ae_, bs_);
-  int incl = mine;
+  int mine = 0, mine_s = 0, lo_, ae_, bs_;
+  for (int b = b0; b < b1; ++b) {
+    mine += token_work(p, b, lo_, ae_, bs_);
+    mine_s += side_count(b);
+  }
+  int incl = mine, incl_s = mine_s;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+    const int z = __shfl_up_sync(0xffffffffu, incl_s, o);
+    if (lane >= o) {
+      incl += y;
+      incl_s += z;
+    }
   }
-  if (lane == 31) wtot[warp] = incl;
+  if (lane == 31) {
+    wtot[0][warp] = incl;
+    wtot[1][warp] = incl_s;
+  }
   __syncthreads();
-  int run = incl - mine;
-  for (int w = 0; w < warp; ++w) run += wtot[w];
+  int run = incl - mine, run_s = incl_s - mine_s;
+  for (int w = 0; w < warp; ++w) {
+    run += wtot[0][w];
+    run_s += wtot[1][w];
+  }
   for (int b = b0; b < b1; ++b) {
     tplan[b] = run;
+    splan[b] = run_s;
     run += token_work(p, b, lo_, ae_, bs_);
+    run_s += side_count(b);
   }
-  if (tid == WARPS * 32 - 1) tplan[p.B] = run;
+  if (tid == WARPS * 32 - 1) {
+    tplan[p.B] = run;
+    splan[p.B] = run_s;
+  }
   __syncthreads();
 
-  const int total = tplan[p.B];
+  const long long nside = (long long)splan[p.B] * p.Hkv;
+  const long long total = nside + tplan[p.B];
   for (long long u = (long long)blockIdx.x * WARPS + warp; u < total; u += (long long)gridDim.x * WARPS) {
-    int lo = 0, hi = p.B - 1;   // sequence: largest b with tplan[b] <= u
+    if (u < nside) {
+      const int q = static_cast<int>(u / p.Hkv), h = static_cast<int>(u % p.Hkv);
+      int lo = 0, hi = p.B - 1;   // sequence: largest b with splan[b] <= q
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (splan[mid] <= q) lo = mid;
+        else hi = mid - 1;
+      }
+      const int b = lo, L_old = p.lens_old[b], L_new = L_old + (p.offsets[b + 1] - p.offsets[b]);
+      const int js = p.sink > 0 ? 1 : 0;
+      const int k = q - splan[b];   // which of the sequence's whole side pages
+      const int j = sink_whole(p, L_old, L_new) ? (k == 0 ? 0 : js + (k - 1)) : js + k;
+      append_side_page<D>(p, b, h, j, L_old, L_new, img[warp], lane);
+      continue;
+    }
+    const int tu = static_cast<int>(u - nside);
+    int lo = 0, hi = p.B - 1;   // sequence: largest b with tplan[b] <= tu
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (tplan[mid] <= u) lo = mid;
+      if (tplan[mid] <= tu) lo = mid;
       else hi = mid - 1;
     }
     const int b = lo;
     int L_old, a_end, b_start;
     token_work(p, b, L_old, a_end, b_start);
-    const int k = static_cast<int>(u - tplan[b]);
+    const int k = tu - tplan[b];
     const int pos = k < a_end - L_old ? L_old + k : b_start + (k - (a_end - L_old));
     const int L_new = L_old + (p.offsets[b + 1] - p.offsets[b]);
     const long long j = p.offsets[b] + (pos - L_old);
@@ -670,6 +832,15 @@ cudaError_t launch_append_pages(unsigned blocks, const AppendParams &p, cudaStre
   return launch_pdl(append_pages_kernel<D>, dim3(blocks), dim3(32 * kAppendWarps), smem, stream, p);
 }
 
+template <int D>
+cudaError_t launch_append_tokens(unsigned blocks, const AppendParams &p, cudaStream_t stream) {
+  const size_t smem = (size_t)(p.B + 1) * 8;   // the two plans
+  const cudaError_t attr = cudaFuncSetAttribute(append_tokens_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)smem);
+  if (attr != cudaSuccess) return attr;
+  return launch_pdl(append_tokens_kernel<D>, dim3(blocks), dim3(32 * kAppendWarps), smem, stream, p);
+}
+
 cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream) {
   AppendParams p = p_in;
   const long long tasks = p.T * p.Hkv * 2;
@@ -689,17 +860,16 @@ cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream) 
   const long long units = (p.T / kPageTokens) * p.Hkv;   // upper bound on (full page, head) units
   const unsigned pblocks = static_cast<unsigned>(std::max(
       1LL, std::min((units + warps_per_block - 1) / warps_per_block, 3LL * std::max(p.num_sms, 1))));
-  const size_t plan_bytes = (size_t)(p.B + 1) * 4;
   cudaError_t e = D == 128 ? launch_append_pages<128>(pblocks, p, stream) : launch_append_pages<64>(pblocks, p, stream);
   if (e != cudaSuccess) return e;
-  // upper bound on the positions with work left: all of them, or per sequence
-  // two partial pages plus the sink and ring rows
-  const long long tw = std::min<long long>(p.T, (long long)p.B * (2 * kPageTokens + p.sink + p.recent));
+  // upper bound on the warp units left: per sequence and KV head the whole side
+  // pages, then the positions with work left (all of them, or per sequence two
+  // partial pages plus the sink and ring rows)
+  const long long tw = std::min<long long>(p.T, (long long)p.B * (2 * kPageTokens + p.sink + p.recent)) +
+                       (long long)p.B * p.Hkv * (1 + p.recent / kPageTokens);
   const unsigned tblocks = static_cast<unsigned>(
       std::max(1LL, std::min((tw + warps_per_block - 1) / warps_per_block, 8192LL)));
-  if (D == 128)
-    return launch_pdl(append_tokens_kernel<128>, dim3(tblocks), dim3(32 * warps_per_block), plan_bytes, stream, p);
-  return launch_pdl(append_tokens_kernel<64>, dim3(tblocks), dim3(32 * warps_per_block), plan_bytes, stream, p);
+  return D == 128 ? launch_append_tokens<128>(tblocks, p, stream) : launch_append_tokens<64>(tblocks, p, stream);
 }
 
 }  // namespace kv4
