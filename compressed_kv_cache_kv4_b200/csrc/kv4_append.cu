@@ -867,8 +867,9 @@ cudaError_t launch_append(const AppendParams &p_in, int D, cudaStream_t stream) 
   // partial pages plus the sink and ring rows)
   const long long tw = std::min<long long>(p.T, (long long)p.B * (2 * kPageTokens + p.sink + p.recent)) +
                        (long long)p.B * p.Hkv * (1 + p.recent / kPageTokens);
+  // resident CTAs only (2 per SM), so that each CTA's plan serves several units
   const unsigned tblocks = static_cast<unsigned>(
-      std::max(1LL, std::min((tw + warps_per_block - 1) / warps_per_block, 8192LL)));
+      std::max(1LL, std::min((tw + warps_per_block - 1) / warps_per_block, 2LL * std::max(p.num_sms, 1))));
   return D == 128 ? launch_append_tokens<128>(tblocks, p, stream) : launch_append_tokens<64>(tblocks, p, stream);
 }
 
