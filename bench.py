@@ -695,6 +695,7 @@ def masked_only(permille=100, reps=20):
     k, v, off = prefill(cache, wl, wl.lens, ptd)
     scores = synth.gen_scores(wl, k, off, device="cuda")
     del k, v
+    torch.cuda.empty_cache()   # the prompt's K/V are not needed again
     q = synth.gen_q(wl, device="cuda")
     lens = torch.as_tensor(wl.lens, device="cuda")
     L = int(wl.lens.max())

@@ -986,7 +986,7 @@ __device__ __forceinline__ void write_cp_partial(int G, SoftmaxState<NMT> &st, f
 template <int D, int G>
 __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(DecodeParams p, GatherParams gp,
                                                                              float *parts) {
-  constexpr int NMT = D / 16, HEAD = 18 * D, KROW = D / 2, NP = D / 16, QB = kv4_q_bytes(D);
+  constexpr int NMT = D / 16, HEAD = 18 * D, KROW = D / 2, QB = kv4_q_bytes(D);
   extern __shared__ __align__(128) uint8_t msm[];
   int *list = reinterpret_cast<int *>(msm);                 // [kMaskedChunk]
   uint8_t *qarea = msm + 4 * kMaskedChunk;                 // [QB] INT4 query format, shared by the warps
@@ -1035,50 +1035,89 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
     }
     __syncthreads();
     const int pg_end = min(npg, (t0 + kMaskedChunk) / kPageTokens);
-    for (int j = t0 / kPageTokens + warp; j < pg_end; j += kMaskedWarps) {
-      for (int q = lane; q < HEAD / 16; q += 32) reinterpret_cast<uint4 *>(im)[q] = make_uint4(0, 0, 0, 0);
-      const int t = kPageTokens * j + i;
-      int page = -1, r = 0;
-      if (t < n) {
-        const int pos = list[t - t0];
-        r = pos % kPageTokens;
-        page = p.page_table[(long long)b * p.pt_stride + pos / kPageTokens];
-        if (page < 0 || page >= p.num_pages) {
-          if (half == 0) set_error(p.err, kErrBounds);
-          page = -1;   // the row stays zero
+    // Software pipeline over the warp's compact pages j, j + W, ...: the page
+    // ids of page j + 2W and the row data of page j + W are in flight while
+    // page j is attended. Row i of a compact page is retained position
+    // 16 j + i; lanes i and i + 16 look its page up, as pr = page * 16 + slot
+    // (-1: no position, or a page id out of range).
+    auto row_page = [&](int jj) -> int {
+      const int t = kPageTokens * jj + i;
+      if (jj >= pg_end || t >= n) return -1;
+      const int pos = list[t - t0];
+      const int page = p.page_table[(long long)b * p.pt_stride + pos / kPageTokens];
+      if (page < 0 || page >= p.num_pages) {
+        if (half == 0) set_error(p.err, kErrBounds);
+        return -1;   // the row stays zero
+      }
+      return page * kPageTokens + pos % kPageTokens;
+    };
+    // The loads are spread so that one warp instruction touches few 128-byte
+    // lines: K, 16-byte piece Q = 32u + lane of the page's 16 rows (D/32 per
+    // row); V, the 128-byte group span of line L = 4u + lane/8 (row L % 16,
+    // 512-byte block L / 16), piece lane % 8; scales, lane (i, half): the K
+    // (half 0) or V (half 1) scale row of row i.
+    // V layout: word (m/4)*128 + 4*P + m%4 with P = 8*tt + (g ^ 2*tt),
+    // tt = (r%8)/2, holds byte 2*(r%2) + r/8 of row r; a row's bytes in a
+    // 512-byte block lie in the 8 pieces of its group span [128 tt, 128 tt + 128).
+    constexpr int KPR = D / 32, NK = D / 64, NV = D / 16;
+    uint4 kc[NK], vp[NV];
+    uint2 sc = make_uint2(0, 0);
+    auto row_src = [&](int pr) -> const uint8_t * {
+      return p.pool + (long long)(pr / kPageTokens) * p.page_bytes + (long long)h * p.head_bytes;
+    };
+    auto issue_rows = [&](int prl) {   // prl: this lane's row (lane & 15)
+#pragma unroll
+      for (int u = 0; u < NK; ++u) {
+        const int q = 32 * u + lane, row = q / KPR, y = q % KPR;
+        const int pr = __shfl_sync(0xffffffffu, prl, row);
+        if (pr >= 0) kc[u] = __ldg(reinterpret_cast<const uint4 *>(row_src(pr) + (pr % kPageTokens) * KROW) + y);
+      }
+      if (prl >= 0) {
+        const int sb = half ? 17 * D : 16 * D;   // K scales (half 0) or V scales (half 1)
+        const uint8_t *src = row_src(prl) + sb + (prl % kPageTokens) * (D / 16);
+        if constexpr (D == 128) sc = __ldg(reinterpret_cast<const uint2 *>(src));
+        else sc.x = __ldg(reinterpret_cast<const uint32_t *>(src));
+      }
+#pragma unroll
+      for (int u = 0; u < NV; ++u) {
+        const int line = 4 * u + (lane >> 3), row = line % kPageTokens, m4 = line / kPageTokens;
+        const int pr = __shfl_sync(0xffffffffu, prl, row);
+        if (pr >= 0) {
+          const int tts = (pr % 8) / 2;
+          vp[u] = __ldg(reinterpret_cast<const uint4 *>(row_src(pr) + 8 * D + m4 * 512 + 128 * tts) + (lane & 7));
         }
       }
-      __syncwarp();
-      if (page >= 0) {
-        const uint8_t *src = p.pool + (long long)page * p.page_bytes + (long long)h * p.head_bytes;
-        uint4 kc[D / 64];
+    };
+    int j = t0 / kPageTokens + warp;
+    int pra = row_page(j), prb = row_page(j + kMaskedWarps);
+    issue_rows(pra);
+    for (; j < pg_end; j += kMaskedWarps) {
+      const int prc = row_page(j + 2 * kMaskedWarps);
+      // the image of page j: zero first unless every row holds a position
+      if (!__all_sync(0xffffffffu, pra >= 0)) {
+        for (int q = lane; q < HEAD / 16; q += 32) reinterpret_cast<uint4 *>(im)[q] = make_uint4(0, 0, 0, 0);
+        __syncwarp();
+      }
 #pragma unroll
-        for (int u = 0; u < D / 64; ++u)
-          kc[u] = __ldg(reinterpret_cast<const uint4 *>(src + r * KROW + half * (KROW / 2)) + u);
-        const int sb = half ? 17 * D : 16 * D;   // K scales (half 0) or V scales (half 1)
-        uint2 sc = make_uint2(0, 0);
-        if constexpr (D == 128) sc = __ldg(reinterpret_cast<const uint2 *>(src + sb + r * (D / 16)));
-        else sc.x = __ldg(reinterpret_cast<const uint32_t *>(src + sb + r * (D / 16)));
-        // V: word (m/4)*128 + 4*P + m%4 with P = 8*tt + (dm8 ^ 2*tt), tt =
-        // (r%8)/2, holds the row's byte 2*(r%2) + r/8; a 16-byte piece (m/4,
-        // dm8) has four of the row's bytes, and the pieces of the row's 4-row
-        // group are 128 contiguous bytes of each 512-byte block
-        const int tts = (r % 8) / 2, ttd = (i % 8) / 2;
-        uint4 vp[NP];
-#pragma unroll
-        for (int u = 0; u < NP; ++u) {
-          const int m4 = D == 128 ? half : 0, dm8 = D == 128 ? u : 4 * half + u;
-          vp[u] = __ldg(reinterpret_cast<const uint4 *>(src + 8 * D + 16 * (m4 * 32 + 8 * tts + (dm8 ^ (2 * tts)))));
-        }
-#pragma unroll
-        for (int u = 0; u < D / 64; ++u) reinterpret_cast<uint4 *>(im + i * KROW + half * (KROW / 2))[u] = kc[u];
+      for (int u = 0; u < NK; ++u) {
+        const int q = 32 * u + lane, row = q / KPR, y = q % KPR;
+        if (__shfl_sync(0xffffffffu, pra, row) >= 0) reinterpret_cast<uint4 *>(im + row * KROW)[y] = kc[u];
+      }
+      if (pra >= 0) {
+        const int sb = half ? 17 * D : 16 * D;
         if constexpr (D == 128) *reinterpret_cast<uint2 *>(im + sb + i * (D / 16)) = sc;
         else *reinterpret_cast<uint32_t *>(im + sb + i * (D / 16)) = sc.x;
-        const int sh_src = 8 * (2 * (r % 2) + r / 8), b_dst = 2 * (i % 2) + i / 8;
+      }
 #pragma unroll
-        for (int u = 0; u < NP; ++u) {
-          const int m4 = D == 128 ? half : 0, dm8 = D == 128 ? u : 4 * half + u;
-          uint8_t *dst = im + 8 * D + 16 * (m4 * 32 + 8 * ttd + (dm8 ^ (2 * ttd))) + b_dst;
+      for (int u = 0; u < NV; ++u) {
+        const int line = 4 * u + (lane >> 3), row = line % kPageTokens, m4 = line / kPageTokens;
+        const int pr = __shfl_sync(0xffffffffu, pra, row);
+        if (pr >= 0) {
+          // source piece x = lane % 8 of the row's span holds g = x ^ 2 tt;
+          // the row's byte of word k goes to the image piece of g for row `row`
+          const int r = pr % kPageTokens, tts = (r % 8) / 2, g = (lane & 7) ^ (2 * tts);
+          const int ttd = (row % 8) / 2, sh_src = 8 * (2 * (r % 2) + r / 8), b_dst = 2 * (row % 2) + row / 8;
+          uint8_t *dst = im + 8 * D + m4 * 512 + 16 * (8 * ttd + (g ^ (2 * ttd))) + b_dst;
           dst[0] = static_cast<uint8_t>(vp[u].x >> sh_src);
           dst[4] = static_cast<uint8_t>(vp[u].y >> sh_src);
           dst[8] = static_cast<uint8_t>(vp[u].z >> sh_src);
@@ -1086,8 +1125,12 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
         }
       }
       __syncwarp();
+      // the rows of page j + W load while page j is attended
+      issue_rows(prb);
       int4_item<D, G>(p, im_u32, q_u32, j, rc, st, lane);
       __syncwarp();
+      pra = prb;
+      prb = prc;
     }
   }
   // The INT8 region: this head's side pages, a warp per side page, the K half
