@@ -1053,9 +1053,9 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
     };
     // The loads are spread so that one warp instruction touches few 128-byte
     // lines: K, 16-byte piece Q = 32u + lane of the page's 16 rows (D/32 per
-    // row); V, the 128-byte group span of line L = 4u + lane/8 (row L % 16,
-    // 512-byte block L / 16), piece lane % 8; scales, lane (i, half): the K
-    // (half 0) or V (half 1) scale row of row i.
+    // row); V, piece lane % 8 of the 128-byte group span of row 4k + lane/8 in
+    // each 512-byte block (k < 4); scales, lane (i, half): the K (half 0) or V
+    // (half 1) scale row of row i.
     // V layout: word (m/4)*128 + 4*P + m%4 with P = 8*tt + (g ^ 2*tt),
     // tt = (r%8)/2, holds byte 2*(r%2) + r/8 of row r; a row's bytes in a
     // 512-byte block lie in the 8 pieces of its group span [128 tt, 128 tt + 128).
@@ -1078,13 +1078,14 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
         if constexpr (D == 128) sc = __ldg(reinterpret_cast<const uint2 *>(src));
         else sc.x = __ldg(reinterpret_cast<const uint32_t *>(src));
       }
+      // V: rows k*4 + lane/8 (k < 4), each over its D/64 blocks
 #pragma unroll
-      for (int u = 0; u < NV; ++u) {
-        const int line = 4 * u + (lane >> 3), row = line % kPageTokens, m4 = line / kPageTokens;
-        const int pr = __shfl_sync(0xffffffffu, prl, row);
+      for (int k = 0; k < 4; ++k) {
+        const int pr = __shfl_sync(0xffffffffu, prl, 4 * k + (lane >> 3));
         if (pr >= 0) {
-          const int tts = (pr % 8) / 2;
-          vp[u] = __ldg(reinterpret_cast<const uint4 *>(row_src(pr) + 8 * D + m4 * 512 + 128 * tts) + (lane & 7));
+          const uint4 *src = reinterpret_cast<const uint4 *>(row_src(pr) + 8 * D + 128 * ((pr % 8) / 2)) + (lane & 7);
+#pragma unroll
+          for (int m4 = 0; m4 < D / 64; ++m4) vp[4 * m4 + k] = __ldg(src + 32 * m4);
         }
       }
     };
@@ -1109,19 +1110,23 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
         else *reinterpret_cast<uint32_t *>(im + sb + i * (D / 16)) = sc.x;
       }
 #pragma unroll
-      for (int u = 0; u < NV; ++u) {
-        const int line = 4 * u + (lane >> 3), row = line % kPageTokens, m4 = line / kPageTokens;
+      for (int k = 0; k < 4; ++k) {
+        const int row = 4 * k + (lane >> 3);
         const int pr = __shfl_sync(0xffffffffu, pra, row);
         if (pr >= 0) {
           // source piece x = lane % 8 of the row's span holds g = x ^ 2 tt;
-          // the row's byte of word k goes to the image piece of g for row `row`
+          // the row's byte of word c goes to the image piece of g for row `row`
           const int r = pr % kPageTokens, tts = (r % 8) / 2, g = (lane & 7) ^ (2 * tts);
           const int ttd = (row % 8) / 2, sh_src = 8 * (2 * (r % 2) + r / 8), b_dst = 2 * (row % 2) + row / 8;
-          uint8_t *dst = im + 8 * D + m4 * 512 + 16 * (8 * ttd + (g ^ (2 * ttd))) + b_dst;
-          dst[0] = static_cast<uint8_t>(vp[u].x >> sh_src);
-          dst[4] = static_cast<uint8_t>(vp[u].y >> sh_src);
-          dst[8] = static_cast<uint8_t>(vp[u].z >> sh_src);
-          dst[12] = static_cast<uint8_t>(vp[u].w >> sh_src);
+          uint8_t *dst = im + 8 * D + 16 * (8 * ttd + (g ^ (2 * ttd))) + b_dst;
+#pragma unroll
+          for (int m4 = 0; m4 < D / 64; ++m4) {
+            const uint4 w = vp[4 * m4 + k];
+            dst[512 * m4 + 0] = static_cast<uint8_t>(w.x >> sh_src);
+            dst[512 * m4 + 4] = static_cast<uint8_t>(w.y >> sh_src);
+            dst[512 * m4 + 8] = static_cast<uint8_t>(w.z >> sh_src);
+            dst[512 * m4 + 12] = static_cast<uint8_t>(w.w >> sh_src);
+          }
         }
       }
       __syncwarp();
