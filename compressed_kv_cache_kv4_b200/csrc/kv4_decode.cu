@@ -928,10 +928,11 @@ __global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
 // One CTA per (sequence, KV head). Its retained INT4-region positions, in
 // order, form "compact pages" of 16 rows; a warp at a time gathers one compact
 // page of the head into a shared-memory image of the ordinary head-block
-// layout (lanes i and i + 16 load the two halves of row i: K codes, the K or V
-// scales, and the 16-byte pieces of the V block that hold the row's bytes;
-// the V bytes are moved to the row's place in the fragment order) and runs
-// the ordinary page computation on it. Rows past the count are zero and not
+// layout (the K rows, the K and V scale rows, and the 16-byte pieces of the
+// V block that hold each row's bytes, loaded with the lanes spread over few
+// lines per instruction; the V bytes are moved to the row's place in the
+// fragment order) and runs the ordinary page computation on it, with the next
+// page's rows already in flight. Rows past the count are zero and not
 // attended. The head's INT8 side pages (sink and recent window, under the
 // same mask) go through the same image and softmax state. Reads and work of
 // the INT4 region follow the retained count; nothing is written back but one

@@ -221,9 +221,9 @@ kv4_status kv4_decode_partials(kv4_cache *cache, void *stream, const void *q, in
  * by the same CTAs under the same mask, and the CTAs' partials are merged. The
  * result is the same attention as kv4_decode_attn with retain_mask (within
  * rounding). Each (sequence, head) is gathered by one CTA, page after page, so
- * the call gains on sparse masks (an H2O-style 10% budget: 0.37x the unmasked
- * decode time on the eviction workload) and loses on dense ones (beyond about a
- * third of the positions, kv4_decode_attn with retain_mask is faster).
+ * the call gains on sparse masks (an H2O-style 10% budget: 0.31x the unmasked
+ * decode time on the eviction workload) and loses on dense ones (beyond about
+ * half of the positions, kv4_decode_attn with retain_mask is faster).
  *  retain_mask: device uint32 [B][Hkv][mask_stride], required; mask_stride *
  *    32 >= pt_stride * 16.
  *  max_retained: bound on the retained INT4-region positions [sink, L - recent)
