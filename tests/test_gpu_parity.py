@@ -45,6 +45,30 @@ def test_append_bytes_match_oracle(name, chunks):
     assert np.array_equal(gs, side), "side cache differs at %s" % np.flatnonzero(gs != side)[:10]
 
 
+@pytest.mark.parametrize("sink,recent,D", [(16, 128, 128), (5, 16, 64), (0, 0, 64), (16, 0, 64), (0, 32, 128),
+                                            (16, 48, 64)])
+@pytest.mark.parametrize("chunks", [1, 3])
+def test_append_side_windows_match_oracle(sink, recent, D, chunks):
+    """INT8 side pages written whole by the page path (a sink page of 16 rows,
+    ring pages whose rows all hold a position) and by rows (a shorter sink,
+    partly filled ring pages, appends that do not renew the whole window),
+    every pool and side byte against the oracle."""
+    wl = small_wl([3, 16, 20, 47, 130, 257, 700], Hq=8, Hkv=2, D=D, seed=sink + recent + chunks, sink=sink,
+                  recent=recent)
+    c = Case(wl)
+    c.make_cache()
+    c.append_all(chunks=chunks)
+    pool, side, flags = c.oracle_cache()
+    assert flags == 0
+    st, bits = c.cache.get_error()
+    assert st == K.KV4_OK, bits
+    gp = c.cache.pool.cpu().numpy()
+    assert np.array_equal(gp, pool), "page pool differs at %s" % np.flatnonzero(gp != pool)[:10]
+    if c.cache.side is not None:
+        gs = c.cache.side.cpu().numpy()
+        assert np.array_equal(gs, side), "side cache differs at %s" % np.flatnonzero(gs != side)[:10]
+
+
 def test_append_unaligned_rows_match_oracle():
     """k_new / v_new 8- but not 16-byte aligned: whole pages go through the
     per-position kernel instead of the page kernel; the bytes are the same."""
