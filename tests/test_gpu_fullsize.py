@@ -201,6 +201,10 @@ def test_evict_full_size():
                           mask=np.ascontiguousarray(m_ref[seqs]))
             assert_close(out32[seqs].cpu().numpy(), ref, what="evict %d" % permille)
             assert_bf16_output(out16[seqs], out32[seqs], ref)
+            # the gathered path at full size, under the same mask
+            g32 = cache.decode_masked(q, lens, ptd, wl.softmax_scale, mask, L * permille // 1000, out_fp32=True)
+            assert_close(g32[seqs].cpu().numpy(), ref, what="evict gathered %d" % permille)
+            assert_close(g32.cpu().numpy(), out32.cpu().numpy(), what="evict gathered vs page path %d" % permille)
         if permille == 1000:
             full = cache.decode(q, lens, ptd, wl.softmax_scale, out_fp32=True, retain_mask=mask)
             assert torch.equal(full, unmasked)
