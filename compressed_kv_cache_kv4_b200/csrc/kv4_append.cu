@@ -574,6 +574,8 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   const int kv = static_cast<int>(task & 1);   // 0: K, 1: V
   const long long j = (task >> 1) / p.Hkv;
   const int h = static_cast<int>((task >> 1) % p.Hkv);
+  // the row's load is in flight while its place in the cache is looked up
+  const RowRaw<D> raw = load_row_raw<D>(p, j, h, kv, lane);
   int b, pos, L_new;
   locate_row(p, j, b, pos, L_new);
   if (pos < 0 || pos >= p.pt_stride * kPageTokens) {
@@ -583,7 +585,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
   RowTarget t;
   if (!row_target(p, b, pos, L_new, lane, t)) return;
   float x[D / 32];
-  unpack_row(load_row_raw<D>(p, j, h, kv, lane), x);
+  unpack_row(raw, x);
   store_row<D>(p, t, x, h, kv, b, lane);
 }
 
