@@ -513,23 +513,26 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
   // (their full keys are fetched after the pass, from L2).
   // A warp covers 128 positions (4 words) per step: lane l positions 4l..4l+3
   // from one 8-byte load; the 8 lanes of a word OR their 4-bit pieces.
-  // Bin d0 holds the prefixes [lo16, lo16 + 2^s); with four candidates per
-  // lane the bounds are compared two prefixes at a time.
+  // Bin d0 holds the prefixes [lo16, lo16 + W), W = 2^s: with u = prefix - lo16
+  // as an unsigned 32-bit difference (a prefix below the bin wraps past 2^31),
+  // the prefix is in the bin iff u < W and above it iff W <= u < 2^31 (no
+  // prefix lies above the top bin).
   const int sub = lane & 7;
   const uint32_t lo16 = pmin + (d0 << sh16), hi16 = lo16 + (1u << sh16);
   const bool top = hi16 > 0xFFFFu;   // no prefix lies above bin d0
-  const uint32_t lo2 = lo16 * 0x10001u, hi2 = (top ? 0xFFFFu : hi16) * 0x10001u;
+  const uint32_t W = 1u << sh16;   // bin d0 is [lo16, lo16 + W)
   for (int it = warp; 4 * it < nt; it += NWARP) {
     const int pos = 128 * it + 4 * lane;
     uint32_t sel = 0, lst = 0;
     if (pos >= c0 && pos + 4 <= c1) {
       const uint2 k2 = *reinterpret_cast<const uint2 *>(keys16 + pos);
-      // 0xFFFF in a half where its prefix is >= the bound
-      const uint32_t gl0 = __vcmpgeu2(k2.x, lo2), gl1 = __vcmpgeu2(k2.y, lo2);
-      const uint32_t gh0 = top ? 0u : __vcmpgeu2(k2.x, hi2), gh1 = top ? 0u : __vcmpgeu2(k2.y, hi2);
-      const uint32_t in0 = gl0 & ~gh0, in1 = gl1 & ~gh1;
-      sel = (gh0 & 1u) | ((gh0 >> 15) & 2u) | ((gh1 & 1u) << 2) | ((gh1 >> 13) & 8u);
-      lst = (in0 & 1u) | ((in0 >> 15) & 2u) | ((in1 & 1u) << 2) | ((in1 >> 13) & 8u);
+      const uint32_t kp[4] = {k2.x & 0xFFFFu, k2.x >> 16, k2.y & 0xFFFFu, k2.y >> 16};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t u = kp[e] - lo16;   // below the bin: wraps past 2^31
+        sel |= static_cast<uint32_t>(u - W < 0x80000000u - W) << e;
+        lst |= static_cast<uint32_t>(u < W) << e;
+      }
     } else {
       uint2 k2 = make_uint2(0, 0);
       if (pos + 4 > c0 && pos < c1) k2 = *reinterpret_cast<const uint2 *>(keys16 + pos);
