@@ -7,17 +7,21 @@
 // head_dim elements, INT8 per token row; scale = max|x| / qmax rounded toward
 // +inf to fp16; code = x / scale rounded to nearest-even.
 //
-// Two kernels. append_pages_kernel takes every page the append fills
+// Three kernels. append_pages_kernel takes every page the append fills
 // completely (a prefill, or a multi-token append that crosses page
-// boundaries): one warp per (page, KV head); for K, then for V, lane l
-// quantises half a group (16 elements) of row l % 16 -- the two lanes of a
-// group combine their maxima with one shuffle -- into a shared-memory image
-// of the 18*D-byte head block, which the warp then writes out with 16-byte
-// stores. The rest -- the INT4 slots of partially filled pages and every INT8
-// side-cache row -- goes to append_tokens_kernel (one warp per new position,
-// over its KV heads and K / V), or, when no page is filled completely, to
-// append_kernel (one warp per new position, KV head and K or V); there lane l
-// holds D/32 consecutive elements of the row.
+// boundaries): one warp per (page, KV head) at a time on resident CTAs, the
+// page's 16 bf16 rows of K, then of V, brought into a per-warp shared-memory
+// stage by the bulk-copy engine one half-unit ahead; lane l quantises half a
+// group (16 elements) of row l % 16 -- the two lanes of a group combine their
+// maxima with one shuffle -- into a shared-memory image of the 18*D-byte head
+// block, which the warp writes out with 16-byte stores. append_tokens_kernel
+// follows: one warp per INT8 side page that the append writes whole (the sink
+// page, ring pages whose rows all hold a position), then one warp per new
+// position with other work left (INT4 slots of partly filled pages, INT8 rows
+// of partly filled side pages), over its KV heads and K / V. When no page is
+// filled completely (a decode step) append_kernel takes everything: one warp
+// per new position, KV head and K or V. In the row paths lane l holds D/32
+// consecutive elements of the row.
 //
 // Scale: fp32 IEEE division then round-up to fp16 equals rounding the exact
 // quotient a/7 (a/127) up: for a bf16 numerator the quotient is either exact
