@@ -1,6 +1,6 @@
 // kv4_common.cuh -- device helpers shared by the libkv4 kernels (sm_100a).
 //
-// Inline PTX for: mbarrier + 1-D bulk copies (the TMA engine, no multicast),
+// Inline PTX for: mbarrier + 1-D bulk copies (the TMA engine, one CTA per copy),
 // warp-level bf16 tensor-core MMA (m16n8k16) and 8x8 fragment transposes,
 // LOP3 nibble -> bf16 unpacking, ex2.approx.
 #pragma once
