@@ -425,28 +425,79 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
   uint32_t *list_key = maskw + NTW;
   uint16_t *list_pos = reinterpret_cast<uint16_t *>(list_key + kListCap);
 
-  // A. stage the key prefixes and find the candidates' prefix range
+  // A. stage the key prefixes and count them into the first histogram as
+  // they arrive, so that its shared-memory atomics overlap the row's loads.
+  // The bins need the candidates' prefix range before the last loads land:
+  // the first step's vectors (one block of NT in every kFastStageVec, spread
+  // over the row) give an estimate [emin, emax], widened by a quarter of its
+  // span on each side to [P0, P0 + 2048 * 2^S); a prefix outside it counts in
+  // the end bin on its side. The exact range follows from the whole pass: a
+  // threshold in an end bin that received such prefixes takes the general
+  // path, every other bin holds exactly the prefixes of its nominal range.
   for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
   if (tid == 0) sh.listn = 0;
-  uint32_t kmin = 0xFFFFu, kmax = 0u;
+  uint32_t kmin = 0xFFFFu, kmax = 0u;   // candidate prefix range of this thread
   const int base = c0 & ~3;
   const int nvec = (c1 - base + 3) >> 2;
+  const int nblk = (nvec + NT - 1) / NT, nstep = (nblk + kFastStageVec - 1) / kFastStageVec;
   const float4 *src = reinterpret_cast<const float4 *>(srow + base);
-  for (int v0 = tid; v0 < nvec; v0 += kFastStageVec * NT) {
+  uint32_t P0 = 0, S = 0;
+  auto bin_of = [&](uint32_t kp) -> uint32_t {
+    const int d = static_cast<int>(kp) - static_cast<int>(P0);
+    return min(static_cast<uint32_t>(max(d, 0)) >> S, static_cast<uint32_t>(kTopkBins - 1));
+  };
+  // candidates among the 4 positions from i (all of them inside the range)
+  auto count4 = [&](int i, uint32_t p01, uint32_t p23) {
+    const uint32_t kp[4] = {p01 & 0xFFFFu, p01 >> 16, p23 & 0xFFFFu, p23 >> 16};
+    if (i >= c0 && i + 4 <= c1) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) atomicAdd(&sh.hist[bin_of(kp[e])], 1u);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (i + e >= c0 && i + e < c1) atomicAdd(&sh.hist[bin_of(kp[e])], 1u);
+    }
+  };
+  // block-wide min / max of the threads' kmin / kmax into sh.kmin / sh.kmax
+  auto reduce_range = [&]() {
+    uint32_t a = kmin, z = kmax;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+      z = max(z, __shfl_xor_sync(0xffffffffu, z, o));
+    }
+    if (lane == 0) {
+      sh.wsum[warp] = static_cast<int>(a);
+      sh.wsum[16 + warp] = static_cast<int>(z);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int x = sh.wsum[0], y = sh.wsum[16];
+      for (int w = 1; w < NWARP; ++w) {
+        x = min(x, sh.wsum[w]);
+        y = max(y, sh.wsum[16 + w]);
+      }
+      sh.kmin = x;
+      sh.kmax = y;
+    }
+    __syncthreads();
+  };
+  for (int st = 0; st < nstep; ++st) {
     float4 buf[kFastStageVec];
 #pragma unroll
     for (int u = 0; u < kFastStageVec; ++u) {
-      const int v = v0 + u * NT;
+      const int v = (st + nstep * u) * NT + tid;
       if (v < nvec) buf[u] = __ldg(src + v);
     }
 #pragma unroll
     for (int u = 0; u < kFastStageVec; ++u) {
-      const int v = v0 + u * NT;
+      const int v = (st + nstep * u) * NT + tid;
       if (v < nvec) {
         const int i = base + 4 * v;
         const uint32_t k0 = score_key2(buf[u].x), k1 = score_key2(buf[u].y), k2 = score_key2(buf[u].z),
                        k3 = score_key2(buf[u].w);
-        *reinterpret_cast<uint2 *>(keys16 + i) = make_uint2(__byte_perm(k0, k1, 0x7632), __byte_perm(k2, k3, 0x7632));
+        const uint2 pk = make_uint2(__byte_perm(k0, k1, 0x7632), __byte_perm(k2, k3, 0x7632));
+        *reinterpret_cast<uint2 *>(keys16 + i) = pk;
         if (i >= c0 && i + 4 <= c1) {
           kmin = min(kmin, min(min(k0, k1), min(k2, k3)) >> 16);
           kmax = max(kmax, max(max(k0, k1), max(k2, k3)) >> 16);
@@ -459,52 +510,38 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
               kmax = max(kmax, ka[e] >> 16);
             }
         }
+        if (st > 0) count4(i, pk.x, pk.y);
+      }
+    }
+    if (st == 0) {
+      // the bins, from the first step's range (it holds position c0)
+      reduce_range();
+      const int emin = sh.kmin, emax = sh.kmax, q = (emax - emin) >> 2;
+      const int lo = max(emin - q, 0), hi = min(emax + q + 1, 0x10000);
+      P0 = static_cast<uint32_t>(lo);
+      while (static_cast<uint32_t>(hi - lo) > (static_cast<uint32_t>(kTopkBins) << S)) ++S;
+#pragma unroll
+      for (int u = 0; u < kFastStageVec; ++u) {
+        const int v = nstep * u * NT + tid;
+        if (v < nvec) {
+          const uint2 k2 = *reinterpret_cast<const uint2 *>(keys16 + base + 4 * v);
+          count4(base + 4 * v, k2.x, k2.y);
+        }
       }
     }
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  if (lane == 0) {
-    sh.wsum[warp] = static_cast<int>(kmin);
-    sh.wsum[16 + warp] = static_cast<int>(kmax);
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int a = sh.wsum[0], z = sh.wsum[16];
-    for (int w = 1; w < NWARP; ++w) {
-      a = min(a, sh.wsum[w]);
-      z = max(z, sh.wsum[16 + w]);
-    }
-    sh.kmin = a;
-    sh.kmax = z;
-  }
-  __syncthreads();
-  const uint32_t pmin = static_cast<uint32_t>(sh.kmin);
-  int sh16 = 0;   // bin of a candidate: (prefix - pmin) >> sh16 < kTopkBins
-  while (((static_cast<uint32_t>(sh.kmax) - pmin) >> sh16) >= static_cast<uint32_t>(kTopkBins)) ++sh16;
-  // B. histogram of the bins (prefixes from shared memory, 4 per load), the
-  // threshold bin d0 and the rank left inside it
-  for (int i = base + 4 * tid; i < c1; i += 4 * NT) {
-    const uint2 k2 = *reinterpret_cast<const uint2 *>(keys16 + i);
-    const uint32_t kp[4] = {k2.x & 0xFFFFu, k2.x >> 16, k2.y & 0xFFFFu, k2.y >> 16};
-    if (i >= c0 && i + 4 <= c1) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) atomicAdd(&sh.hist[(kp[e] - pmin) >> sh16], 1u);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (i + e >= c0 && i + e < c1) atomicAdd(&sh.hist[(kp[e] - pmin) >> sh16], 1u);
-    }
-  }
+  reduce_range();   // the exact range: were prefixes counted in an end bin from outside it?
+  const bool low_out = static_cast<uint32_t>(sh.kmin) < P0;
+  const bool high_out = static_cast<uint32_t>(sh.kmax) >= P0 + (static_cast<uint32_t>(kTopkBins) << S);
+  const uint32_t pmin = P0;
+  const int sh16 = static_cast<int>(S);
   __syncthreads();
   select_bin<NT>(sh, static_cast<int>(ksel), tid);
   const uint32_t d0 = static_cast<uint32_t>(sh.digit);
   const int rem0 = sh.rem, n0 = sh.cnt;
-  if (n0 > kListCap) {
-    // a crowded threshold bin: the general path, keys re-read from global memory
+  if (n0 > kListCap || (d0 == 0 && low_out) || (d0 == kTopkBins - 1 && high_out)) {
+    // a crowded threshold bin, or an end bin wider than its nominal range:
+    // the general path, keys re-read from global memory
     __syncthreads();
     topk_row<false, NT>(p, row, reinterpret_cast<uint32_t *>(dynb), sh);
     return;

@@ -270,6 +270,35 @@ def test_topk_crowded_threshold_bin(permille):
     assert np.array_equal(count.cpu().numpy(), c_ref)
 
 
+@pytest.mark.parametrize("permille", [10, 100, 990])
+def test_topk_range_off_the_first_loads(permille):
+    """Rows whose values depend strongly on the position, so that a part of the
+    row alone misjudges the range of the whole: tail outliers far above or far
+    below the rest, an exponential ramp, and blocks of 1024 positions with
+    scales from 1e-20 to 1e20. Thresholds among the outliers fall outside any
+    range estimated without them; the masks must still equal the oracle's."""
+    rng = np.random.default_rng(permille + 31)
+    B, Hkv, Lmax = 2, 4, 16384
+    lens = np.array([16384, 9001], np.int32)
+    sc = rng.standard_normal((B, Hkv, Lmax)).astype(np.float32)
+    for b, L in enumerate(lens):
+        sc[b, 0, L - 428:L - 128] = np.float32(1e30) * (1.0 + rng.random(300)).astype(np.float32)
+        sc[b, 1, L - 428:L - 128] = np.float32(-1e30) * (1.0 + rng.random(300)).astype(np.float32)
+        sc[b, 2, :] = np.exp2(np.arange(Lmax) / 256.0).astype(np.float32)
+        scale = 10.0 ** rng.uniform(-20, 20, (Lmax + 1023) // 1024)
+        sc[b, 3, :] = (sc[b, 3, :] * np.repeat(scale, 1024)[:Lmax]).astype(np.float32)
+    mstride = (Lmax + 31) // 32
+    mask = torch.zeros((B, Hkv, mstride), dtype=torch.int32, device="cuda")
+    count = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+    K.kv_topk_retain(torch.as_tensor(sc, device="cuda"), torch.as_tensor(lens, device="cuda"), permille, mask, count)
+    m_ref, c_ref = O.topk(sc, lens, permille)
+    got = mask.cpu().numpy().view(np.uint32)
+    for b in range(B):
+        nw = (int(lens[b]) + 31) // 32
+        assert np.array_equal(got[b, :, :nw], m_ref[b, :, :nw]), b
+    assert np.array_equal(count.cpu().numpy(), c_ref)
+
+
 def test_topk_long_rows_global_path():
     rng = np.random.default_rng(9)
     B, Hkv, Lmax = 1, 2, 70000
