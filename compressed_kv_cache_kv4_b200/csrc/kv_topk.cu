@@ -446,18 +446,16 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
     const int d = static_cast<int>(kp) - static_cast<int>(P0);
     return min(static_cast<uint32_t>(max(d, 0)) >> S, static_cast<uint32_t>(kTopkBins - 1));
   };
-  // candidates among the 4 positions from i (all of them inside the range)
-  auto count4 = [&](int i, uint32_t p01, uint32_t p23) {
-    const uint32_t kp[4] = {p01 & 0xFFFFu, p01 >> 16, p23 & 0xFFFFu, p23 >> 16};
-    if (i >= c0 && i + 4 <= c1) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) atomicAdd(&sh.hist[bin_of(kp[e])], 1u);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (i + e >= c0 && i + e < c1) atomicAdd(&sh.hist[bin_of(kp[e])], 1u);
-    }
+  // the 4 prefixes of a vector whose positions are all candidates
+  auto count4 = [&](uint32_t p01, uint32_t p23) {
+    atomicAdd(&sh.hist[bin_of(p01 & 0xFFFFu)], 1u);
+    atomicAdd(&sh.hist[bin_of(p01 >> 16)], 1u);
+    atomicAdd(&sh.hist[bin_of(p23 & 0xFFFFu)], 1u);
+    atomicAdd(&sh.hist[bin_of(p23 >> 16)], 1u);
   };
+  // vectors [v_in0, v_in1) hold candidates only; the first and the last
+  // vector may also hold forced positions and are finished after the pass
+  const int v_in0 = base < c0 ? 1 : 0, v_in1 = (c1 - base) >> 2;
   // block-wide min / max of the threads' kmin / kmax into sh.kmin / sh.kmax
   auto reduce_range = [&]() {
     uint32_t a = kmin, z = kmax;
@@ -493,39 +491,52 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
     for (int u = 0; u < kFastStageVec; ++u) {
       const int v = (st + nstep * u) * NT + tid;
       if (v < nvec) {
-        const int i = base + 4 * v;
         const uint32_t k0 = score_key2(buf[u].x), k1 = score_key2(buf[u].y), k2 = score_key2(buf[u].z),
                        k3 = score_key2(buf[u].w);
         const uint2 pk = make_uint2(__byte_perm(k0, k1, 0x7632), __byte_perm(k2, k3, 0x7632));
-        *reinterpret_cast<uint2 *>(keys16 + i) = pk;
-        if (i >= c0 && i + 4 <= c1) {
+        *reinterpret_cast<uint2 *>(keys16 + base + 4 * v) = pk;
+        if (v >= v_in0 && v < v_in1) {
           kmin = min(kmin, min(min(k0, k1), min(k2, k3)) >> 16);
           kmax = max(kmax, max(max(k0, k1), max(k2, k3)) >> 16);
-        } else {
-          const uint32_t ka[4] = {k0, k1, k2, k3};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (i + e >= c0 && i + e < c1) {
-              kmin = min(kmin, ka[e] >> 16);
-              kmax = max(kmax, ka[e] >> 16);
-            }
+          if (st > 0) count4(pk.x, pk.y);
         }
-        if (st > 0) count4(i, pk.x, pk.y);
       }
     }
     if (st == 0) {
-      // the bins, from the first step's range (it holds position c0)
+      // the bins, from the first step's range (no candidate there: the whole
+      // prefix range)
       reduce_range();
-      const int emin = sh.kmin, emax = sh.kmax, q = (emax - emin) >> 2;
-      const int lo = max(emin - q, 0), hi = min(emax + q + 1, 0x10000);
+      int lo = 0, hi = 0x10000;
+      if (sh.kmin <= sh.kmax) {
+        const int emin = sh.kmin, emax = sh.kmax, q = (emax - emin) >> 2;
+        lo = max(emin - q, 0);
+        hi = min(emax + q + 1, 0x10000);
+      }
       P0 = static_cast<uint32_t>(lo);
       while (static_cast<uint32_t>(hi - lo) > (static_cast<uint32_t>(kTopkBins) << S)) ++S;
 #pragma unroll
       for (int u = 0; u < kFastStageVec; ++u) {
         const int v = nstep * u * NT + tid;
-        if (v < nvec) {
+        if (v >= v_in0 && v < v_in1) {
           const uint2 k2 = *reinterpret_cast<const uint2 *>(keys16 + base + 4 * v);
-          count4(base + 4 * v, k2.x, k2.y);
+          count4(k2.x, k2.y);
+        }
+      }
+    }
+  }
+  __syncthreads();   // the last vector may have been staged by another thread
+  if (tid < 2) {
+    // the first and the last vector when they hold forced positions
+    const int v = tid == 0 ? 0 : nvec - 1;
+    if ((v < v_in0 || v >= v_in1) && (tid == 0 || v > 0)) {
+      const uint2 k2 = *reinterpret_cast<const uint2 *>(keys16 + base + 4 * v);
+      const uint32_t kp[4] = {k2.x & 0xFFFFu, k2.x >> 16, k2.y & 0xFFFFu, k2.y >> 16};
+      for (int e = 0; e < 4; ++e) {
+        const int q = base + 4 * v + e;
+        if (q >= c0 && q < c1) {
+          kmin = min(kmin, kp[e]);
+          kmax = max(kmax, kp[e]);
+          atomicAdd(&sh.hist[bin_of(kp[e])], 1u);
         }
       }
     }
@@ -552,44 +563,15 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
   // from one 8-byte load; the 8 lanes of a word OR their 4-bit pieces.
   // Bin d0 holds the prefixes [lo16, lo16 + W), W = 2^s: with u = prefix - lo16
   // as an unsigned 32-bit difference (a prefix below the bin wraps past 2^31),
-  // the prefix is in the bin iff u < W and above it iff W <= u < 2^31 (no
-  // prefix lies above the top bin).
+  // the prefix is in the bin iff u < W and above it iff W <= u < 2^31 (every
+  // prefix is below 2^16).
   const int sub = lane & 7;
   const uint32_t lo16 = pmin + (d0 << sh16), hi16 = lo16 + (1u << sh16);
-  const bool top = hi16 > 0xFFFFu;   // no prefix lies above bin d0
   const uint32_t W = 1u << sh16;   // bin d0 is [lo16, lo16 + W)
-  for (int it = warp; 4 * it < nt; it += NWARP) {
-    const int pos = 128 * it + 4 * lane;
-    uint32_t sel = 0, lst = 0;
-    if (pos >= c0 && pos + 4 <= c1) {
-      const uint2 k2 = *reinterpret_cast<const uint2 *>(keys16 + pos);
-      const uint32_t kp[4] = {k2.x & 0xFFFFu, k2.x >> 16, k2.y & 0xFFFFu, k2.y >> 16};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t u = kp[e] - lo16;   // below the bin: wraps past 2^31
-        sel |= static_cast<uint32_t>(u - W < 0x80000000u - W) << e;
-        lst |= static_cast<uint32_t>(u < W) << e;
-      }
-    } else {
-      uint2 k2 = make_uint2(0, 0);
-      if (pos + 4 > c0 && pos < c1) k2 = *reinterpret_cast<const uint2 *>(keys16 + pos);
-      const uint32_t kp[4] = {k2.x & 0xFFFFu, k2.x >> 16, k2.y & 0xFFFFu, k2.y >> 16};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int q = pos + e;
-        const bool cand = q >= c0 && q < c1;
-        const bool above = !top && kp[e] >= hi16, inbin = kp[e] >= lo16 && !above;
-        sel |= static_cast<uint32_t>((q < L && !cand) || (cand && above)) << e;
-        lst |= static_cast<uint32_t>(cand && inbin) << e;
-      }
-    }
-    sel <<= 4 * sub;
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) sel |= __shfl_xor_sync(0xffffffffu, sel, o);
-    const int w = 4 * it + (lane >> 3);
-    if (sub == 0 && w < nt) maskw[w] = sel;
-    if (!__any_sync(0xffffffffu, lst != 0)) continue;
-    // list bin d0: warp-wide slots, one shared-memory atomic per warp
+  // bin d0's positions p + stride * e of the set bits e of lst listed
+  // (warp-wide slots, one shared-memory atomic per warp)
+  auto list_lane = [&](uint32_t lst, int p, int stride) {
+    if (!__any_sync(0xffffffffu, lst != 0)) return;
     const int nl = __popc(lst);
     int excl = nl;
 #pragma unroll
@@ -605,8 +587,57 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
     while (lst) {
       const int e = __ffs(lst) - 1;
       lst &= lst - 1;
-      list_pos[at++] = static_cast<uint16_t>(pos + e);
+      list_pos[at++] = static_cast<uint16_t>(p + stride * e);
     }
+  };
+  // the word pieces of a step (lane l: positions 4l..4l+3) ORed and stored
+  auto store_pieces = [&](int it, uint32_t sel) {
+    sel <<= 4 * sub;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) sel |= __shfl_xor_sync(0xffffffffu, sel, o);
+    const int w = 4 * it + (lane >> 3);
+    if (sub == 0 && w < nt) maskw[w] = sel;
+  };
+  // steps [it_in0, it_in1) lie inside [c0, c1)
+  const int nstp = (nt + 3) / 4;
+  const int it_in0 = min((c0 + 127) / 128, nstp), it_in1 = max(it_in0, c1 / 128);
+  // (lane l takes positions l, l + 32, l + 64, l + 96 of the step, so that a
+  // ballot is a whole mask word)
+  for (int it = it_in0 + warp; it < it_in1; it += NWARP) {
+    const int p0 = 128 * it + lane;
+    uint32_t sw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t u = static_cast<uint32_t>(keys16[p0 + 32 * e]) - lo16;   // below the bin: wraps past 2^31
+      sw[e] = __ballot_sync(0xffffffffu, u - W < 0x80000000u - W);
+      lw[e] = __ballot_sync(0xffffffffu, u < W);
+    }
+    if (lane == 0) *reinterpret_cast<uint4 *>(maskw + 4 * it) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+    if ((lw[0] | lw[1] | lw[2] | lw[3]) == 0u) continue;
+    uint32_t lst = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) lst |= ((lw[e] >> lane) & 1u) << e;
+    list_lane(lst, p0, 32);
+  }
+  // the other steps: forced positions, the ends of the candidate range
+  const int n_edge = it_in0 + (nstp - it_in1);
+  for (int j = warp; j < n_edge; j += NWARP) {
+    const int it = j < it_in0 ? j : it_in1 + (j - it_in0);
+    const int pos = 128 * it + 4 * lane;
+    uint2 k2 = make_uint2(0, 0);
+    if (pos + 4 > c0 && pos < c1) k2 = *reinterpret_cast<const uint2 *>(keys16 + pos);
+    const uint32_t kp[4] = {k2.x & 0xFFFFu, k2.x >> 16, k2.y & 0xFFFFu, k2.y >> 16};
+    uint32_t sel = 0, lst = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int q = pos + e;
+      const bool cand = q >= c0 && q < c1;
+      const bool above = kp[e] >= hi16, inbin = kp[e] >= lo16 && !above;
+      sel |= static_cast<uint32_t>((q < L && !cand) || (cand && above)) << e;
+      lst |= static_cast<uint32_t>(cand && inbin) << e;
+    }
+    store_pieces(it, sel);
+    list_lane(lst, pos, 1);
   }
   __syncthreads();
   // the listed positions' full keys, all loads in flight together
