@@ -326,15 +326,17 @@ __device__ void topk_row(const TopkParams &p, int row, uint32_t *dyn, TopkShared
 // Rows of up to kFastMaxLen positions with 16-byte aligned scores: the row is
 // staged as the top 16 bits of its keys (so four CTAs share an SM and a batch
 // of rows runs in one wave). The first histogram bins the candidates' key
-// prefixes relative to the row's own range, (prefix - min) >> s with the
-// smallest s that fits 2048 bins: scores that span a few octaves spread over
-// about a thousand counters instead of the few dozen that fixed sign and
-// exponent bits would give, so the shared-memory atomics rarely collide. One
-// pass over the staged prefixes then writes every mask bit except those of the
-// threshold bin and lists that bin's positions; the exact threshold is
+// prefixes relative to the row's own range, (prefix - P0) >> s over 2048 bins:
+// scores that span a few octaves spread over about a thousand counters instead
+// of the few dozen that fixed sign and exponent bits would give, so the
+// shared-memory atomics rarely collide. The prefixes are counted as they are
+// staged, with the range estimated from the first step of loads (see phase A).
+// One pass over the staged prefixes then writes every mask bit except those of
+// the threshold bin and lists that bin's positions; the exact threshold is
 // selected among the listed keys (full keys re-read from global memory, cached
 // in L2 by then) and their bits are set last. A threshold bin larger than
-// kListCap falls back to the general path.
+// kListCap, or an end bin that also counted prefixes outside the estimated
+// range, falls back to the general path.
 // ---------------------------------------------------------------------------
 constexpr int kFastThreads = 256;
 constexpr int kFastMaxLen = 16384;
