@@ -127,25 +127,26 @@ __device__ __forceinline__ void weights_bf16(float2 w01, float2 w23, float2 neg_
   b1 = movmatrix_t(pack_bf16x2(r23.x, r23.y));
 }
 
-// fp16 variant of weights_bf16 (hi + lo carry 22 significant bits).
-__device__ __forceinline__ void weights_f16x2(float2 w01, float2 w23, float2 neg_sel, uint32_t &b0, uint32_t &b1) {
+// fp16 variant of weights_bf16 (hi + lo carry 22 significant bits). The
+// remainder w - hi comes from a mixed-precision FMA (fp16 factors, fp32
+// addend, one rounding), so the hi halves need no conversion back to fp32.
+// neg_sel is -1 (0xBC00) on the "lo" lanes and 0 on the "hi" lanes.
+__device__ __forceinline__ float fma_f16_f32(uint16_t a, uint16_t b, float c) {
+  float d;
+  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ void weights_f16x2(float2 w01, float2 w23, uint16_t neg_sel, uint32_t &b0, uint32_t &b1) {
   const uint32_t h01 = pack_f16x2(w01.x, w01.y);
   const uint32_t h23 = pack_f16x2(w23.x, w23.y);
-  const float2 r01 = __ffma2_rn(neg_sel, f16x2_to_f32x2(h01), w01);
-  const float2 r23 = __ffma2_rn(neg_sel, f16x2_to_f32x2(h23), w23);
-  b0 = movmatrix_t(pack_f16x2(r01.x, r01.y));
-  b1 = movmatrix_t(pack_f16x2(r23.x, r23.y));
+  const float r0 = fma_f16_f32(static_cast<uint16_t>(h01), neg_sel, w01.x);
+  const float r1 = fma_f16_f32(static_cast<uint16_t>(h01 >> 16), neg_sel, w01.y);
+  const float r2 = fma_f16_f32(static_cast<uint16_t>(h23), neg_sel, w23.x);
+  const float r3 = fma_f16_f32(static_cast<uint16_t>(h23 >> 16), neg_sel, w23.y);
+  b0 = movmatrix_t(pack_f16x2(r0, r1));
+  b1 = movmatrix_t(pack_f16x2(r2, r3));
 }
-
-__device__ __forceinline__ void weights_f16(float w0, float w1, float w2, float w3, float lo_sel, uint32_t &b0,
-                                            uint32_t &b1) {
-  uint32_t h01 = pack_f16x2(w0, w1);
-  uint32_t h23 = pack_f16x2(w2, w3);
-  h01 = pack_f16x2(fmaf(-lo_sel, f16lo_to_f32(h01), w0), fmaf(-lo_sel, f16hi_to_f32(h01), w1));
-  h23 = pack_f16x2(fmaf(-lo_sel, f16lo_to_f32(h23), w2), fmaf(-lo_sel, f16hi_to_f32(h23), w3));
-  b0 = movmatrix_t(h01);
-  b1 = movmatrix_t(h23);
-}
+__device__ __forceinline__ uint16_t f16_neg_sel(bool lo) { return lo ? static_cast<uint16_t>(0xBC00u) : 0; }
 
 // Reduce and write the worker's partial for one piece.
 template <int D, int NMT>
@@ -635,7 +636,7 @@ __device__ __forceinline__ void int4_item(const DecodeParams &p, uint32_t stg, u
   float pr[4];
   softmax_update<NMT, 0>(st, sl, pr);
 
-  const float2 neg_sel = t >= 2 ? make_float2(-1.f, -1.f) : make_float2(0.f, 0.f);
+  const uint16_t neg_sel = f16_neg_sel(t >= 2);
   uint32_t wb[NG][2];
 #pragma unroll
   for (int i = 0; i < NG; ++i) {
@@ -719,7 +720,8 @@ __device__ __forceinline__ void int8k_item(const DecodeParams &p, uint32_t stg, 
   softmax_update<NMT, 0>(st, sl, pr);
   const float s0 = half_bits_to_f32(lds16(stg + 16 * D + 32 + 2 * g));
   const float s1 = half_bits_to_f32(lds16(stg + 16 * D + 32 + 2 * (g + 8)));
-  weights_f16(pr[0] * s0, pr[1] * s0, pr[2] * s1, pr[3] * s1, t >= 2 ? 1.f : 0.f, wb0, wb1);
+  weights_f16x2(make_float2(pr[0] * s0, pr[1] * s0), make_float2(pr[2] * s1, pr[3] * s1), f16_neg_sel(t >= 2), wb0,
+                wb1);
 }
 
 // V half of an INT8 side page: P.V on fp16 tiles with the weights of the K half.
