@@ -132,14 +132,15 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// D = A * B + C with separate C inputs (c0, c1, c0, c1: the same start for
-// both row halves), A 16x16 (row), B 16x8 (col) bf16, C/D fp32.
-__device__ __forceinline__ void mma_bf16_c(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, float c0,
-                                           float c1) {
+// D = A * B + C with the four C registers given (fp32 bit patterns), A 16x16
+// (row), B 16x8 (col) bf16, C/D fp32.
+__device__ __forceinline__ void mma_bf16_c4(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                            uint4 c) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%10,%11,%10,%11};"
+      "{%10,%11,%12,%13};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(__uint_as_float(c.x)),
+        "f"(__uint_as_float(c.y)), "f"(__uint_as_float(c.z)), "f"(__uint_as_float(c.w)));
 }
 
 // Transpose an 8x8 matrix of 16-bit elements held one row per 4 lanes.

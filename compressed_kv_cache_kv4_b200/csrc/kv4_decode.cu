@@ -311,7 +311,7 @@ constexpr int kItemInt4 = 0, kItemInt8K = 1, kItemInt8V = 2;
 // Per-warp query area: D/32 chunks of 512 bytes (the B fragments of the q.K
 // tiles, one 16-byte piece per lane) and, for INT4 ranges, the accumulator
 // start of every (group, query head): D/32 x 4 floats.
-__host__ __device__ constexpr int kv4_q_bytes(int D) { return (D / 32) * 512 + (D / 32) * 16; }
+__host__ __device__ constexpr int kv4_q_bytes(int D) { return (D / 32) * 512 + (D / 32) * 32; }
 
 // Shared-memory layout of the KV4 kernel (bytes), for HB heads, NS stages and
 // NVB virtual sequences.
@@ -500,8 +500,10 @@ __device__ void mark_ranges(const DecodeParams &p, const int *plan, int n8, long
 // Query fragments of one (virtual sequence, head) into the warp's q area.
 // INT4 format (per group i, 512 bytes): q as the B operand of the two q.K
 // tiles -- bf16 pairs of the even elements, fp16 pairs of the odd ones --
-// then, after the NG group chunks, a table [group][query head] of the
-// accumulator starts -(136 * sum of even q + 72 * sum of odd q).
+// then, after the NG group chunks, the accumulator starts
+// -(136 * sum of even q + 72 * sum of odd q) of each group as ready-made C
+// register quads [group][t & 1] = {c(h), c(h + 1), c(h), c(h + 1)}, h = 2 (t & 1),
+// which one 16-byte load hands to the MMA without register moves.
 // INT8 format: fp16 fragments of the D/16 tiles of the side-page q.K.
 // Every query element must lie in the fp16 range (it enters fp16 tiles);
 // one that does not is reported as KV4_ERR_RANGE.
@@ -530,7 +532,13 @@ __device__ __forceinline__ void load_q(const DecodeParams &p, int b, int h, bool
       part += __shfl_xor_sync(0xffffffffu, part, 1);
       part += __shfl_xor_sync(0xffffffffu, part, 2);
       // lanes 4c..4c+3 now hold the offset of column c, i.e. of query head c & 3
-      if (t == 0 && g < 4) reinterpret_cast<float *>(qsm + NG * 512)[4 * i + g] = part;
+      if (t == 0 && g < 4) {
+        // the accumulator start of MMA columns (2t, 2t + 1) for rows g and g + 8,
+        // as the four C registers {c0, c1, c0, c1} of lanes with t & 1 = g >> 1
+        float *quad = reinterpret_cast<float *>(qsm + NG * 512) + 8 * i + 4 * (g >> 1) + (g & 1);
+        quad[0] = part;
+        quad[2] = part;
+      }
     }
   } else {
     constexpr int NJ = D / 16;
@@ -552,6 +560,7 @@ __device__ __forceinline__ void load_q(const DecodeParams &p, int b, int h, bool
 // Per-range context of a warp.
 struct RangeCtx {
   int b, h, L, lo_tok, hi_tok, r0;
+  int pin0, pspan;   // pages [pin0, pin0 + pspan) have every slot attended (none under a mask)
   const uint32_t *mrow;
 };
 
@@ -600,12 +609,12 @@ __device__ __forceinline__ void int4_item(const DecodeParams &p, uint32_t stg, u
   for (int i = 0; i < NG; ++i) {
     const uint4 qv = lds128(qsm + i * 512 + lane * 16);
     // accumulator start of columns 2t, 2t+1 (query heads 2t & 3, (2t & 3) + 1)
-    const float2 qi = lds64f(qsm + NG * 512 + 16 * i + 8 * (t & 1));
+    const uint4 qi = lds128(qsm + NG * 512 + 32 * i + 16 * (t & 1));
     float acc[4];
     const uint32_t k80 = kw0[i] >> 8, k81 = kw1[i] >> 8;
     {   // elements 0, 4 (k-slots 2t, 2t+1) and 2, 6 (2t+8, 2t+9): bf16, 136 + c
       const uint32_t a[4] = {i4x2_biased(kw0[i]), i4x2_biased(kw1[i]), i4x2_biased(k80), i4x2_biased(k81)};
-      mma_bf16_c(acc, a, qv.x, qv.y, qi.x, qi.y);
+      mma_bf16_c4(acc, a, qv.x, qv.y, qi);
     }
     {   // elements 1, 5 and 3, 7: fp16, 72 + c (bits 4-7 convert in place)
       const uint32_t a[4] = {i4x2_hi_biased_f16(kw0[i]), i4x2_hi_biased_f16(kw1[i]), i4x2_hi_biased_f16(k80),
@@ -621,7 +630,7 @@ __device__ __forceinline__ void int4_item(const DecodeParams &p, uint32_t stg, u
   sc23 = __fmul2_rn(sc23, sl2);
   float sl[4] = {sc01.x, sc01.y, sc23.x, sc23.y};
   // which of the page's slots are attended (all of them on interior pages)
-  if (rc.mrow || pg * kPageTokens < rc.lo_tok || pg * kPageTokens + kPageTokens > rc.hi_tok) {
+  if (static_cast<uint32_t>(pg - rc.pin0) >= static_cast<uint32_t>(rc.pspan)) {
     const int tok0 = pg * kPageTokens + g, tok1 = tok0 + 8;
     bool v0 = tok0 >= rc.lo_tok && tok0 < rc.hi_tok;
     bool v1 = tok1 >= rc.lo_tok && tok1 < rc.hi_tok;
@@ -870,6 +879,8 @@ __global__ void __launch_bounds__(256, 2) kv4_decode_kernel(DecodeParams p) {
         rc.hi_tok = rc.L - p.recent;
         rc.r0 = max(p.sink, rc.L - p.recent);
         rc.mrow = p.mask ? p.mask + ((long long)rc.b * p.Hkv + rc.h) * p.mask_stride : nullptr;
+        rc.pin0 = (rc.lo_tok + kPageTokens - 1) / kPageTokens;
+        rc.pspan = rc.mrow ? 0 : max(0, (rc.hi_tok >= 0 ? rc.hi_tok / kPageTokens : -1) - rc.pin0);
         load_q<D, G>(p, rc.b, rc.h, kind == kItemInt4, qsm, lane);
       }
       const bool ok = p.wait_cap != 0 && mbar_wait_bounded(&full[s], (phase >> s) & 1u, p.wait_cap);
@@ -1021,6 +1032,8 @@ __global__ void __launch_bounds__(kMaskedWarps * 32, 4) masked_decode_kernel(Dec
   rc.lo_tok = 0;
   rc.hi_tok = n;   // rows of compact page j are retained indices 16 j .. 16 j + 15
   rc.mrow = nullptr;
+  rc.pin0 = 0;
+  rc.pspan = n / kPageTokens;
   const uint32_t im_u32 = smem_u32(im), q_u32 = smem_u32(qarea);
   const int i = lane & 15, half = lane >> 4;
   for (int t0 = 0; t0 < npg * kPageTokens; t0 += kMaskedChunk) {
