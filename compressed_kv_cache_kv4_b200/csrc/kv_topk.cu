@@ -439,14 +439,16 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
   for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
   if (tid == 0) sh.listn = 0;
   uint32_t kmin = 0xFFFFu, kmax = 0u;   // candidate prefix range of this thread
+  uint32_t kmin2 = 0xFFFFFFFFu, kmax2 = 0u;   // the same over whole vectors, two 16-bit lanes
   const int base = c0 & ~3;
   const int nvec = (c1 - base + 3) >> 2;
   const int nblk = (nvec + NT - 1) / NT, nstep = (nblk + kFastStageVec - 1) / kFastStageVec;
   const float4 *src = reinterpret_cast<const float4 *>(srow + base);
   uint32_t P0 = 0, S = 0;
+  int negP0 = 0, top = 0;   // -P0, and the last prefix offset of the top bin
   auto bin_of = [&](uint32_t kp) -> uint32_t {
-    const int d = static_cast<int>(kp) - static_cast<int>(P0);
-    return min(static_cast<uint32_t>(max(d, 0)) >> S, static_cast<uint32_t>(kTopkBins - 1));
+    // max(min(kp - P0, top), 0) >> S: one clamped add, one shift
+    return static_cast<uint32_t>(__viaddmin_s32_relu(static_cast<int>(kp), negP0, top)) >> S;
   };
   // the 4 prefixes of a vector whose positions are all candidates
   auto count4 = [&](uint32_t p01, uint32_t p23) {
@@ -460,7 +462,7 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
   const int v_in0 = base < c0 ? 1 : 0, v_in1 = (c1 - base) >> 2;
   // block-wide min / max of the threads' kmin / kmax into sh.kmin / sh.kmax
   auto reduce_range = [&]() {
-    uint32_t a = kmin, z = kmax;
+    uint32_t a = min(kmin, min(kmin2 & 0xFFFFu, kmin2 >> 16)), z = max(kmax, max(kmax2 & 0xFFFFu, kmax2 >> 16));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
@@ -498,8 +500,8 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
         const uint2 pk = make_uint2(__byte_perm(k0, k1, 0x7632), __byte_perm(k2, k3, 0x7632));
         *reinterpret_cast<uint2 *>(keys16 + base + 4 * v) = pk;
         if (v >= v_in0 && v < v_in1) {
-          kmin = min(kmin, min(min(k0, k1), min(k2, k3)) >> 16);
-          kmax = max(kmax, max(max(k0, k1), max(k2, k3)) >> 16);
+          kmin2 = __vimin3_u16x2(kmin2, pk.x, pk.y);
+          kmax2 = __vimax3_u16x2(kmax2, pk.x, pk.y);
           if (st > 0) count4(pk.x, pk.y);
         }
       }
@@ -516,6 +518,8 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
       }
       P0 = static_cast<uint32_t>(lo);
       while (static_cast<uint32_t>(hi - lo) > (static_cast<uint32_t>(kTopkBins) << S)) ++S;
+      negP0 = -lo;
+      top = (kTopkBins << S) - 1;
 #pragma unroll
       for (int u = 0; u < kFastStageVec; ++u) {
         const int v = nstep * u * NT + tid;
