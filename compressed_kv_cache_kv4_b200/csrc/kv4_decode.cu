@@ -46,6 +46,12 @@ struct Bf16Cfg {
 // Partial slot: m[G] | l[G] | pad | o[G][D]   (m in log2 units, o normalised)
 // ---------------------------------------------------------------------------
 
+// Running-max start: the lowest finite float, so that score - max needs no
+// test for an empty state. Only -inf (excluded) scores and scores equal to it
+// leave it in place; they get weights 0 and 1, as against a true maximum. A
+// state that attended nothing keeps l = 0 and is written as empty.
+constexpr float kNoMax = -3.40282347e38f;
+
 // Online-softmax state of one warp for the 8 MMA columns (4 "hi" + 4 "lo"
 // copies of up to 4 query heads). Thread (g, t) owns columns 2t and 2t+1.
 template <int NMT>
@@ -53,7 +59,7 @@ struct SoftmaxState {
   float m[2], l[2];
   float o[NMT][4];   // O^T fragments: rows = head_dim, columns = MMA columns
   __device__ __forceinline__ void reset() {
-    m[0] = m[1] = -INFINITY;
+    m[0] = m[1] = kNoMax;
     l[0] = l[1] = 0.f;
 #pragma unroll
     for (int mt = 0; mt < NMT; ++mt)
@@ -101,7 +107,7 @@ __device__ __forceinline__ void softmax_update(SoftmaxState<NMT> &st, const floa
       st.m[1] = mx1;
     }
   }
-  const float2 r = make_float2(st.m[0] == -INFINITY ? 0.f : st.m[0], st.m[1] == -INFINITY ? 0.f : st.m[1]);
+  const float2 r = make_float2(st.m[0], st.m[1]);   // kNoMax while nothing is attended: every p is 0
   const float2 d01 = __fadd2_rn(make_float2(s[0], s[1]), make_float2(-r.x, -r.y));
   const float2 d23 = __fadd2_rn(make_float2(s[2], s[3]), make_float2(-r.x, -r.y));
   pr[0] = ex2(d01.x);
