@@ -41,6 +41,15 @@ constexpr int kTcThreads = 128;   // one warpgroup: TMEM lanes 0..127
 constexpr int kTcRows = 128;      // tile rows (M of every MMA)
 constexpr int kKeyBlock = 64;     // keys per block (N of S, K of P V)
 
+// x - hi for a bf16 hi: a mixed-precision FMA (bf16 factors, fp32 addend, one
+// rounding), so hi needs no conversion back to fp32.
+constexpr uint16_t kBf16MinusOne = 0xBF80u;
+__device__ __forceinline__ float fma_bf16_f32(uint16_t a, uint16_t b, float c) {
+  float d;
+  asm("fma.rn.f32.bf16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
@@ -330,7 +339,8 @@ __global__ void __launch_bounds__(kTcThreads) smd_attn_kernel(SmdParams p) {
       for (int e = 0; e < 4; ++e) {
         const float x0 = x[c * 8 + 2 * e], x1 = x[c * 8 + 2 * e + 1];
         hw[e] = pack_bf16x2(x0, x1);
-        lw[e] = pack_bf16x2(x0 - bf16lo_to_f32(hw[e]), x1 - bf16hi_to_f32(hw[e]));
+        lw[e] = pack_bf16x2(fma_bf16_f32(static_cast<uint16_t>(hw[e]), kBf16MinusOne, x0),
+                            fma_bf16_f32(static_cast<uint16_t>(hw[e] >> 16), kBf16MinusOne, x1));
       }
       const int off = (c * 16 + r / 8) * 128 + (r % 8) * 16;
       *reinterpret_cast<uint4 *>(sph + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
