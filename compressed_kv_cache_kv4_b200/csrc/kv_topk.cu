@@ -334,7 +334,8 @@ __device__ void topk_row(const TopkParams &p, int row, uint32_t *dyn, TopkShared
 // One pass over the staged prefixes then writes every mask bit except those of
 // the threshold bin and lists that bin's positions; the exact threshold is
 // selected among the listed keys (full keys re-read from global memory, cached
-// in L2 by then) and their bits are set last. A threshold bin larger than
+// in L2 by then; one warp ranks them when at most 32 are listed) and their
+// bits are set last. A threshold bin larger than
 // kListCap, or an end bin that also counted prefixes outside the estimated
 // range, falls back to the general path.
 // ---------------------------------------------------------------------------
@@ -649,29 +650,59 @@ __global__ void __launch_bounds__(kFastThreads, 4) topk_fast_kernel(TopkParams p
   // the listed positions' full keys, all loads in flight together
   for (int i = tid; i < n0; i += NT) list_key[i] = score_key2(srow[list_pos[i]]);
   __syncthreads();
-  // D. the exact threshold inside bin d0: its keys lie in [kbase, kbase + 2^(16+s))
-  // with s <= 5, so two 11-bit digits of key - kbase finish the selection
+  // D. the exact threshold inside bin d0. Up to 32 listed keys: one warp
+  // ranks them against each other (keys above and equal to each). More: its
+  // keys lie in [kbase, kbase + 2^(16+s)) with s <= 5, so two 11-bit digits of
+  // key - kbase finish the selection.
   const int n = n0;
-  const uint32_t kbase = (pmin + (d0 << sh16)) << 16;
-  for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += NT) atomicAdd(&sh.hist[(list_key[i] - kbase) >> 11], 1u);
-  __syncthreads();
-  select_bin<NT>(sh, rem0, tid);
-  const uint32_t d1 = static_cast<uint32_t>(sh.digit);
-  const int rem1 = sh.rem;
-  __syncthreads();
-  for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += NT) {
-    const uint32_t k = list_key[i] - kbase;
-    if ((k >> 11) == d1) atomicAdd(&sh.hist[k & 2047u], 1u);
+  uint32_t T;
+  int need_eq;
+  bool ties;
+  if (n <= 32) {
+    if (warp == 0) {
+      const bool valid = lane < n;
+      const uint32_t k = valid ? list_key[lane] : 0u;
+      int gt = 0, eq = 0;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t kj = __shfl_sync(0xffffffffu, k, j);
+        gt += kj > k ? 1 : 0;
+        eq += kj == k ? 1 : 0;
+      }
+      // T: the key with gt < rem0 <= gt + eq (every lane holding it agrees)
+      const uint32_t bal = __ballot_sync(0xffffffffu, valid && gt < rem0 && rem0 <= gt + eq);
+      const int src = __ffs(bal) - 1;
+      const uint32_t t_key = __shfl_sync(0xffffffffu, k, src);
+      const int t_gt = __shfl_sync(0xffffffffu, gt, src), t_eq = __shfl_sync(0xffffffffu, eq, src);
+      if (lane == 0) {
+        sh.digit = static_cast<int>(t_key);
+        sh.rem = rem0 - t_gt;
+        sh.cnt = t_eq;
+      }
+    }
+    __syncthreads();
+    T = static_cast<uint32_t>(sh.digit);
+  } else {
+    const uint32_t kbase = (pmin + (d0 << sh16)) << 16;
+    for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += NT) atomicAdd(&sh.hist[(list_key[i] - kbase) >> 11], 1u);
+    __syncthreads();
+    select_bin<NT>(sh, rem0, tid);
+    const uint32_t d1 = static_cast<uint32_t>(sh.digit);
+    const int rem1 = sh.rem;
+    __syncthreads();
+    for (int i = tid; i < kTopkBins; i += NT) sh.hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += NT) {
+      const uint32_t k = list_key[i] - kbase;
+      if ((k >> 11) == d1) atomicAdd(&sh.hist[k & 2047u], 1u);
+    }
+    __syncthreads();
+    select_bin<NT>(sh, rem1, tid);
+    T = kbase + (d1 << 11) + static_cast<uint32_t>(sh.digit);
   }
-  __syncthreads();
-  select_bin<NT>(sh, rem1, tid);
-  const uint32_t T = kbase + (d1 << 11) + static_cast<uint32_t>(sh.digit);
-  const int need_eq = sh.rem;
-  const bool ties = need_eq < sh.cnt;
+  need_eq = sh.rem;
+  ties = need_eq < sh.cnt;
   // E. bits of the listed positions: keys above T, and keys equal to T by
   // index order (ranks from a bitmap of the equal keys and a scan over words)
   if (!ties) {

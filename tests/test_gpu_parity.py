@@ -299,6 +299,36 @@ def test_topk_range_off_the_first_loads(permille):
     assert np.array_equal(count.cpu().numpy(), c_ref)
 
 
+@pytest.mark.parametrize("permille", [100, 300])
+def test_topk_threshold_bin_sizes(permille):
+    """Rows whose threshold bin holds few keys (the exact selection among them
+    by one warp) or a few dozen to a few hundred (by digit histograms): a
+    block of equal scores of 8, 31, 33 or 60 positions placed at the budget's
+    quantile, and a coarse value grid (about 128 equal keys per value)."""
+    rng = np.random.default_rng(permille + 41)
+    B, Hkv, Lmax = 2, 5, 16384
+    lens = np.array([16384, 7001], np.int32)
+    sc = rng.standard_normal((B, Hkv, Lmax)).astype(np.float32)
+    for b, L in enumerate(lens):
+        c = np.arange(16, L - 128)
+        for h, run in enumerate((8, 31, 33, 60)):
+            row = sc[b, h]
+            q = np.sort(row[c])[::-1][int(L) * permille // 1000 - 144]
+            pos = rng.choice(c, run, replace=False)
+            row[pos] = q
+        sc[b, 4, :] = (np.round(sc[b, 4, :] * 16) / 16).astype(np.float32)
+    mstride = (Lmax + 31) // 32
+    mask = torch.zeros((B, Hkv, mstride), dtype=torch.int32, device="cuda")
+    count = torch.zeros((B, Hkv), dtype=torch.int32, device="cuda")
+    K.kv_topk_retain(torch.as_tensor(sc, device="cuda"), torch.as_tensor(lens, device="cuda"), permille, mask, count)
+    m_ref, c_ref = O.topk(sc, lens, permille)
+    got = mask.cpu().numpy().view(np.uint32)
+    for b in range(B):
+        nw = (int(lens[b]) + 31) // 32
+        assert np.array_equal(got[b, :, :nw], m_ref[b, :, :nw]), b
+    assert np.array_equal(count.cpu().numpy(), c_ref)
+
+
 def test_topk_long_rows_global_path():
     rng = np.random.default_rng(9)
     B, Hkv, Lmax = 1, 2, 70000
